@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Benchmark of the 4-bit quantized MoE expert layer on B200.
+
+Metric: MoE-layer prefill tokens/s (with TFLOP/s and the fraction of the
+layer roofline) for one Qwen3.6-35B-A3B-shaped layer: hidden 2048, 256
+routed experts, top-8, expert intermediate 512, one sigmoid-gated shared
+expert, symmetric int4 weights in groups of 128; default batch T = 512
+tokens of synthetic bf16 N(0,1) activations and seeded random weights.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+One process per GPU (torchrun for N > 1).  Each rank runs its own
+replica on its own tokens (the layer shards by token with no exchange), so
+the whole-job value is N * T tokens per step ("weak" scaling).  Rank 0
+prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+FLOP_PER_TOKEN_TERMS = "2*k*3*H*I + 2*3*H*I (shared) + 2*H*E (router) + 2*H (shared gate)"
+
+
+def flops_per_token(cfg) -> int:
+    f = 2 * cfg.k * 3 * cfg.H * cfg.I + 2 * cfg.H * cfg.E
+    if cfg.has_shared:
+        f += 2 * 3 * cfg.H * cfg.I + 2 * cfg.H
+    return f
+
+
+def expert_bytes(cfg) -> tuple:
+    """(gate/up, down) algorithmic bytes of one expert: codes + scales / headers."""
+    if cfg.wfmt == 1:
+        gu = 2 * cfg.I * (cfg.H // 256) * 144
+        dn = cfg.H * (cfg.I // 256) * 144
+    else:
+        gu = 2 * cfg.I * cfg.H // 2 + 2 * cfg.I * (cfg.H // cfg.G) * 2
+        dn = cfg.H * cfg.I // 2 + cfg.H * (cfg.I // cfg.G) * 2
+    return gu, dn
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "quantized_moe_expert_warp_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_tag: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", f"ncu_{kernel_tag}_{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return int(float(vals["dram_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """SM clock and throttle reasons sampled through NVML while work runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.ok = False
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ oracle arm
+
+def oracle_sample_rate(layer, n_tokens: int):
+    """Time the CPU oracle (as it stands) on the first n_tokens of the batch.
+
+    Routing and the permutation still cover the whole batch (that is how
+    the oracle is written); the expert FFNs and the combine run for the
+    sampled tokens only.  Returns (tokens/s, seconds)."""
+    import oracle
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.layer_forward(layer, sample=np.arange(n_tokens))
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, dt
+
+
+def run_reference(args, cfg, rank, world):
+    if rank != 0:
+        return
+    import synth
+    layer = synth.make_layer(cfg)
+    n = args.ref_sample
+    for _ in range(args.warmup):
+        oracle_sample_rate(layer, n)
+    rates, secs = [], 0.0
+    for _ in range(args.steps):
+        r, dt = oracle_sample_rate(layer, n)
+        rates.append(r)
+        secs += dt
+    value = args.steps * n / secs
+    line = {
+        "metric": "MoE-layer prefill tokens/s", "impl": "reference", "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights quantised)",
+        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k, "I": cfg.I},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"first {n} of {cfg.T} tokens per step (routing of all {cfg.T})"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------- our arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="a3b_t512")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-sample", type=int, default=8, help="tokens per oracle step (reference arm)")
+    ap.add_argument("--cpu-sample", type=int, default=96, help="tokens of the CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true", help="short run for ncu: no e2e / cpu legs")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if not args.profile else args.warmup
+
+    import synth
+    rank, world, local = dist_setup()
+    cfg = synth.get_config(args.config)
+
+    if args.impl == "reference":
+        if world > 1:
+            import torch.distributed as dist
+            import datetime
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+        run_reference(args, cfg, rank, world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    import torch
+    import quantized_moe_expert_warp_b200 as mq
+    from quantized_moe_expert_warp_b200.host import upload_layer, x_to_device
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    # every rank: the same layer weights, its own tokens
+    rcfg = cfg if rank == 0 else cfg.with_(x_stream=cfg.x_stream + 7919 * rank)
+    layer = synth.make_layer(rcfg)
+    packed = upload_layer(layer, dev)
+    T, H, E, k = cfg.T, cfg.H, cfg.E, cfg.k
+    x = x_to_device(layer["x"], dev)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    nbytes = mq.moe_layer_workspace_size(cfg, T)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mq.moe_layer_forward(packed, x, T, y, ws, nbytes, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st, det = mq.moe_read_status(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({det}) after warm-up")
+
+    # ---------------------------------------------------------- timed region
+    sampler = ClockSampler(local)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with sampler:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        launches0 = mq.moe_kernel_launches()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        ev1.synchronize()
+        launches = mq.moe_kernel_launches() - launches0
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        # keep the same work running for a short window so that the clock
+        # sampler also sees a sustained load when the timed region is short
+        t_end = time.perf_counter() + (0.5 if not args.profile else 0.0)
+        while time.perf_counter() < t_end:
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize(dev)
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms_max = max_over_ranks(ms, world, dev)
+    st, det = mq.moe_read_status(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({det}) in the timed region")
+
+    value = world * T / (ms_max * 1e-3)
+    fpt = flops_per_token(cfg)
+    tflops = value * fpt / 1e12
+
+    # ------------------------------------------- per-kernel times (same stream)
+    # the composed path (same kernels as the fused call), events between steps
+    e32 = lambda *s: torch.empty(s, dtype=torch.float32, device=dev)
+    i32 = lambda *s: torch.empty(s, dtype=torch.int32, device=dev)
+    logits, gl, ids, tw = e32(T, E), e32(T), i32(T, k), e32(T, k)
+    counts, offsets, ss, dp = i32(E), i32(E + 1), i32(T * k), i32(T * k)
+    pn = mq.moe_permute_workspace_size(T, E, k)
+    pws = torch.zeros(pn, dtype=torch.uint8, device=dev)
+    fn = mq.moe_expert_ffn_workspace_size(cfg, T)
+    fws = torch.zeros(fn, dtype=torch.uint8, device=dev)
+    h = torch.empty((T * k + T, cfg.I), dtype=torch.bfloat16, device=dev)
+    y_perm = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
+    sh = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    names = ["router_logits", "route", "permute", "gate_up_gemm", "down_gemm", "combine"]
+    calls = [
+        lambda: mq.moe_router_logits(packed, x, T, logits, gl, stream),
+        lambda: mq.moe_route(logits, T, E, k, cfg.renorm, ids, tw, stream),
+        lambda: mq.moe_permute(ids, T, E, k, counts, offsets, ss, dp, pws, pn, stream),
+        lambda: mq.moe_expert_gate_up_q4(packed, x, T, ss, offsets, h, fws, fn, stream),
+        lambda: mq.moe_expert_down_q4(packed, h, T, offsets, y_perm, sh, fws, fn, stream),
+        lambda: mq.moe_combine(y_perm, dp, tw, sh, gl, T, H, k, y, stream),
+    ]
+    for _ in range(2):
+        for c in calls:
+            c()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    for s in range(args.steps):
+        evs[s][0].record(stream)
+        for i, c in enumerate(calls):
+            c()
+            evs[s][i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    per_kernel_ms = {n: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps))
+                     for i, n in enumerate(names)}
+    composed_ms = sum(per_kernel_ms.values())
+    touched = int((counts.cpu().numpy() > 0).sum()) + (1 if cfg.has_shared else 0)
+    gu_b, dn_b = expert_bytes(cfg)
+    alg = {
+        "gate_up_gemm": touched * gu_b + 2 * T * H,
+        "down_gemm": touched * dn_b,
+    }
+    dominant = max(("gate_up_gemm", "down_gemm"), key=lambda n: per_kernel_ms[n])
+    peaks = {}
+    mp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(mp):
+        peaks = json.load(open(mp))
+    hbm_peak = peaks.get("hbm_gbs")
+    peak_src = "measured"
+    if not hbm_peak:
+        hbm_peak, peak_src = 6650.0, "fallback"
+    achieved = alg[dominant] / (per_kernel_ms[dominant] * 1e-3) / 1e9
+    tag = {"gate_up_gemm": "gate_up", "down_gemm": "down"}[dominant]
+    roofline = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": ncu_traffic(tag, cfg.name),
+                "algorithmic_bytes_per_launch": alg[dominant], "ms_per_launch": per_kernel_ms[dominant],
+                "peak_source": peak_src}
+    # whole-layer roofline: max(FLOPs at tensor peak, bytes at HBM peak)
+    layer_bytes = touched * (gu_b + dn_b) + E * H * 4 + 4 * T * H
+    t_hbm = layer_bytes / (hbm_peak * 1e9)
+    tc_peak = peaks.get("bf16_tflops", 1590.0)
+    t_tc = T * fpt / (tc_peak * 1e12)
+    layer_roof = {"bound": "hbm" if t_hbm >= t_tc else "tensor", "roofline_ms": 1e3 * max(t_hbm, t_tc),
+                  "frac": 1e3 * max(t_hbm, t_tc) / ms, "bytes": layer_bytes, "flops": T * fpt,
+                  "hbm_gbs_achieved": layer_bytes / (ms * 1e-3) / 1e9}
+
+    # ------------------------------------------------------------------ e2e
+    e2e = None
+    if not args.profile:
+        x_host = torch.from_numpy(np.ascontiguousarray(layer["x"]).view(np.int16)).pin_memory()
+        y_host = torch.empty((T, H), dtype=torch.int16).pin_memory()
+        x_in = torch.empty((T, H), dtype=torch.int16, device=dev)
+        y_out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+
+        def e2e_step():
+            x_in.copy_(x_host, non_blocking=True)
+            mq.moe_layer_forward(packed, x_in, T, y_out, ws, nbytes, stream)
+            y_host.copy_(y_out.view(torch.int16), non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        a1.record(stream)
+        a1.synchronize()
+        e_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps, world, dev)
+        e2e = {"value": world * T / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
+               "d2h_bytes_per_step": T * H * 2, "ms_per_step": e_ms}
+
+    # ---------------------------------------------------------- cpu baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
+        n = min(args.cpu_sample, T)
+        rate, dt = oracle_sample_rate(layer, n)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"first {n} of {T} tokens ({dt:.1f} s; routing and permutation of all {T})"}
+
+    if rank == 0:
+        line = {
+            "metric": "MoE-layer prefill tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 activations; N(0,0.02) weights, int4-sym quantised)",
+            "config": {"workload": cfg.name, "T": T, "H": H, "E": E, "k": k, "I": cfg.I,
+                       "shared_expert": bool(cfg.has_shared), "weights": "int4-sym" if cfg.wfmt == 0 else "q4k",
+                       "G": cfg.G, "tokens_per_rank": T, "parallelism": f"replicas x{world} (token-sharded)",
+                       "l2": "inputs larger than L2 (expert weights %.0f MB)" % (packed.weight_bytes() / 1e6)},
+            "tflops": tflops, "flop_per_token": fpt,
+            "roofline": roofline, "layer_roofline": layer_roof,
+            "per_kernel_ms": per_kernel_ms, "composed_ms_per_step": composed_ms,
+            "experts_touched": touched,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,239 @@
+/*
+ * moeq4 -- C ABI of the 4-bit weight-quantized Mixture-of-Experts FFN layer
+ * for NVIDIA B200 (sm_100a).  Library: libmoeq4.so.
+ *
+ * The layer is the routed-expert FFN of a Qwen3.6-35B-A3B-style model, the
+ * model the hipfire 0.4.3 benchmarks page measures ("Qwen3.6-35B-A3B
+ * prefill on the R9700" table; its "Read this before comparing columns"
+ * table names the MoE prefill routes: per-expert buffers, and the
+ * symmetric IU4 MoE route for files with symmetric int4 experts).  The
+ * hipEngine post ("GGUF" section) adds the Q4_K super-block format.  The
+ * pages give no equations; the layer computed here is the plain reading:
+ *
+ *   logits[t,e] = x[t,:] . Wr[e,:] + bias[e]                (moe_router_logits)
+ *   ids[t,:]    = the k largest logits, ties to the lower id, descending
+ *   w[t,j]      = exp(L[ids[t,j]] - L_max) / sum_{i<k} exp(L[ids[t,i]] - L_max)
+ *                 (renorm = 1; renorm = 0 divides by the sum over all E) (moe_route)
+ *   slots s = t*k + j are sorted by expert, stably in s        (moe_permute)
+ *   Y[p] = (silu(x[t_p] Wg_e^T) * (x[t_p] Wu_e^T)) Wd_e^T      (moe_expert_ffn_q4)
+ *   y[t] = sum_j w[t,j] Y[dest_pos[t*k+j]] + sigmoid(x[t].g) S[t]  (moe_combine)
+ *
+ * where S is the same FFN with the shared expert's weights on every token.
+ * moe_layer_forward runs all steps in order on one stream.
+ *
+ * Conventions for every call:
+ *  - Returns MOE_OK (0) or a negative MOE_ERR_* code; moe_last_error()
+ *    then gives a message (thread-local, valid until the next call).
+ *  - Tensor pointers are DEVICE pointers owned by the caller; arrays are
+ *    row-major and contiguous.  Pointers handed to kernels must be 16-byte
+ *    aligned (MOE_ERR_INVALID_ARG otherwise).  The library never
+ *    allocates device memory; scratch comes from a caller workspace whose
+ *    size a *_workspace_size call returns.
+ *  - `stream` is a cudaStream_t (NULL: the legacy default stream).  Calls
+ *    enqueue kernels and return without synchronising.  Failures detected
+ *    inside kernels (a wait that exceeded its time budget) are recorded in
+ *    a status word inside the workspace; moe_read_status() reads it.
+ *  - bf16 tensors are passed as uint16_t bit patterns.
+ */
+#ifndef MOEQ4_H
+#define MOEQ4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1) /* null / misaligned pointer, bad size                  */
+#define MOE_ERR_UNSUPPORTED (-2) /* shape or format the kernels do not admit              */
+#define MOE_ERR_CUDA (-3)        /* a CUDA runtime call failed (message has the cause)    */
+#define MOE_ERR_TIMEOUT (-4)     /* a device-side wait ran out of its budget               */
+#define MOE_ERR_WORKSPACE (-5)   /* workspace missing or smaller than required            */
+
+/* Expert weight formats. */
+#define MOE_WFMT_INT4_SYM 0 /* int4 two's complement, one bf16 scale per G weights along K */
+#define MOE_WFMT_Q4K 1      /* Q4_K-style 256-weight super-blocks (see moe_pack_weights)   */
+
+/* Shapes of one layer.  Admitted: H % 128 == 0, I % 128 == 0, 1 <= k <= E <= 1024,
+ * int4-sym: G % 32 == 0 and G divides H and I; Q4K: H % 256 == 0, I % 256 == 0. */
+typedef struct moe_config {
+    int32_t H;          /* hidden size                                   */
+    int32_t I;          /* expert intermediate size (shared expert too)  */
+    int32_t E;          /* routed experts                                */
+    int32_t k;          /* experts per token                             */
+    int32_t G;          /* int4-sym group size along K (ignored for Q4K) */
+    int32_t has_shared; /* 1: one always-on shared expert                */
+    int32_t renorm;     /* 1: renormalise the top-k weights to sum to 1  */
+    int32_t wfmt;       /* MOE_WFMT_*                                    */
+} moe_config_t;
+
+/* Device pointers of one layer's weights (caller-owned). */
+typedef struct moe_layer {
+    moe_config_t cfg;
+    const float *router_w;    /* [E, H] fp32                                     */
+    const float *router_bias; /* [E] fp32 or NULL                                */
+    const float *shared_gate; /* [H] fp32 (required when has_shared)             */
+    const void *gu_q;         /* gate/up codes in the kernel layout (moe_pack_weights) */
+    const void *gu_meta;      /* gate/up scales or super-block headers           */
+    const void *dn_q;         /* down codes in the kernel layout                 */
+    const void *dn_meta;      /* down scales or super-block headers              */
+} moe_layer_t;
+
+/* Optional exports / overrides of moe_layer_forward (all device pointers,
+ * each may be NULL).  When override_ids is set, routing is skipped and
+ * override_ids / override_w [T, k] are used instead. */
+typedef struct moe_debug {
+    float *logits;            /* [T, E]  */
+    float *gate_logit;        /* [T]     */
+    int32_t *topk_ids;        /* [T, k]  */
+    float *topk_w;            /* [T, k]  */
+    int32_t *counts;          /* [E]     */
+    int32_t *offsets;         /* [E + 1] */
+    int32_t *sorted_slot;     /* [T k]   */
+    int32_t *dest_pos;        /* [T k]   */
+    const int32_t *override_ids;
+    const float *override_w;
+} moe_debug_t;
+
+/* Message of the last failed call on this thread ("" if none). */
+const char *moe_last_error(void);
+
+/* ABI version (increments on incompatible change). */
+int moe_version(void);
+
+/* Number of kernels this library has enqueued in this process (host-side count). */
+uint64_t moe_kernel_launches(void);
+
+/* --------------------------------------------------------------- weights */
+
+/* Bytes of the four kernel-layout buffers for all E (+1 shared) experts.
+ * Returns MOE_ERR_UNSUPPORTED for shapes the kernels do not admit. */
+int moe_packed_sizes(const moe_config_t *cfg, size_t *gu_q_bytes, size_t *gu_meta_bytes, size_t *dn_q_bytes,
+                     size_t *dn_meta_bytes);
+
+/*
+ * Convert canonical expert weights (device memory) to the kernel layout.
+ * Canonical, per expert e in [0, E + has_shared) (the shared expert last):
+ *   gate/up matrix [2I, H] (gate rows first), down matrix [H, I];
+ *   int4-sym: codes uint8 [rows, K/2] (element 2i in the low nibble,
+ *             two's complement) and scales bf16 [rows, K/G];
+ *   Q4K:      uint8 [rows, K/256 * 144] super-blocks: fp16 d, fp16 dmin,
+ *             12 bytes of sixteen 6-bit fields (little-endian bit stream:
+ *             sc_0..7 then m_0..7), 128 bytes of unsigned 4-bit q (weight
+ *             i in byte i/2, low nibble when i is even);
+ *             w = d*sc_j*q - dmin*m_j for sub-block j = i / 32.
+ *   gu_scale / dn_scale are ignored (may be NULL) for Q4K.
+ * Outputs go to caller buffers of the sizes moe_packed_sizes() returns.
+ * Source: hipfire 0.4.3 benchmarks, "Read this before comparing columns"
+ * (symmetric-expert mq4rs file); hipEngine post, "GGUF" (Q4_K).  The bit
+ * layouts are this library's own; the pages give none.
+ */
+int moe_pack_weights(const moe_config_t *cfg, const void *gu_canon, const void *gu_scale, const void *dn_canon,
+                     const void *dn_scale, void *gu_q, void *gu_meta, void *dn_q, void *dn_meta, void *stream);
+
+/*
+ * Dequantised weights of one matrix of one expert, decoded from the kernel
+ * layout exactly as the GEMM kernels decode them.  which = 0: gate/up
+ * [2I, H]; which = 1: down [H, I].  out_f32 gets the exact values (fp32),
+ * out_bf16 (optional) the bf16 operand the tensor cores consume.
+ */
+int moe_dequant_export(const moe_config_t *cfg, const void *q, const void *meta, int which, int expert,
+                       float *out_f32, uint16_t *out_bf16, void *stream);
+
+/* ------------------------------------------------------------ the steps */
+
+/*
+ * Router logits and the shared expert's gate logit.
+ *   x [T, H] bf16, logits [T, E] fp32 (bias added when L->router_bias),
+ *   gate_logit [T] fp32 = x . shared_gate (may be NULL; ignored without a
+ *   shared expert).  fp32 accumulation.
+ */
+int moe_router_logits(const moe_layer_t *L, const uint16_t *x, int T, float *logits, float *gate_logit,
+                      void *stream);
+
+/*
+ * Top-k routing, one warp per token.  logits [T, E] fp32 (finite),
+ * topk_ids [T, k] int32 (descending logit, ties to the lower id),
+ * topk_w [T, k] fp32.  1 <= k <= min(E, 32), E <= 1024.
+ */
+int moe_route(const float *logits, int T, int E, int k, int renorm, int32_t *topk_ids, float *topk_w,
+              void *stream);
+
+/* Workspace bytes of moe_permute for T tokens. */
+size_t moe_permute_workspace_size(int T, int E, int k);
+
+/*
+ * Stable counting sort of the T*k slots by expert.
+ *   counts [E], offsets [E + 1] (offsets[E] = T k), sorted_slot [T k]
+ *   (slot t*k + j at position p), dest_pos [T k] (inverse).  Ids outside
+ *   [0, E) are a device error (status word).  ws: moe_permute_workspace_size.
+ */
+int moe_permute(const int32_t *topk_ids, int T, int E, int k, int32_t *counts, int32_t *offsets,
+                int32_t *sorted_slot, int32_t *dest_pos, void *ws, size_t ws_bytes, void *stream);
+
+/* Workspace bytes of moe_expert_ffn_q4 for T tokens. */
+size_t moe_expert_ffn_workspace_size(const moe_config_t *cfg, int T);
+
+/*
+ * Grouped expert FFN on 4-bit weights (tensor cores, bf16 operands, fp32
+ * accumulation): for every permuted row p of expert e,
+ *   y_perm[p] = bf16( (silu(x[t] Wg_e^T) * (x[t] Wu_e^T)) Wd_e^T ),
+ *   t = sorted_slot[p] / k, and the intermediate rounded to bf16;
+ * and with a shared expert shared_out[t] the same FFN with its weights for
+ * every token t.  x [T, H], y_perm [T k, H], shared_out [T, H] (bf16).
+ * offsets [E + 1] from moe_permute.
+ */
+int moe_expert_ffn_q4(const moe_layer_t *L, const uint16_t *x, int T, const int32_t *sorted_slot,
+                      const int32_t *offsets, uint16_t *y_perm, uint16_t *shared_out, void *ws, size_t ws_bytes,
+                      void *stream);
+
+/*
+ * The two passes of moe_expert_ffn_q4, for callers that want them apart
+ * (same kernels, same results):
+ *   gate/up:  h[p] = bf16( silu(x[t] Wg_e^T) * (x[t] Wu_e^T) ),  h [T k (+ T), I]
+ *             (rows T k .. T k + T - 1 are the shared expert's, token t = p - T k)
+ *   down:     y_perm[p] = bf16( h[p] Wd_e^T ), shared_out[t] = bf16( h[T k + t] Wd_s^T )
+ * ws: moe_expert_ffn_workspace_size (the h buffer inside it is not used).
+ */
+int moe_expert_gate_up_q4(const moe_layer_t *L, const uint16_t *x, int T, const int32_t *sorted_slot,
+                          const int32_t *offsets, uint16_t *h, void *ws, size_t ws_bytes, void *stream);
+int moe_expert_down_q4(const moe_layer_t *L, const uint16_t *h, int T, const int32_t *offsets, uint16_t *y_perm,
+                       uint16_t *shared_out, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Weighted combine: y[t] = bf16( sum_j topk_w[t,j] y_perm[dest_pos[t k + j]]
+ *                                + sigmoid(shared_gate_logit[t]) shared_out[t] )
+ * summed in fp32 in j order; shared_out / shared_gate_logit may be NULL.
+ */
+int moe_combine(const uint16_t *y_perm, const int32_t *dest_pos, const float *topk_w, const uint16_t *shared_out,
+                const float *shared_gate_logit, int T, int H, int k, uint16_t *y, void *stream);
+
+/* --------------------------------------------------------- fused layer */
+
+/* Workspace bytes of moe_layer_forward for up to T_max tokens. */
+size_t moe_layer_workspace_size(const moe_config_t *cfg, int T_max);
+
+/*
+ * The whole layer: router logits, routing, permutation, expert FFNs and
+ * combine, in that order on `stream`, with all intermediates in `ws`.
+ * x [T, H] bf16 -> y [T, H] bf16.  Same kernels as the separate calls, so
+ * the result is bitwise equal to running them one after another.
+ */
+int moe_layer_forward(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *y, void *ws, size_t ws_bytes,
+                      void *stream, const moe_debug_t *dbg);
+
+/*
+ * Read (and, when clear != 0, reset) the device status word kept in a
+ * workspace of moe_layer_forward / moe_expert_ffn_q4 / moe_permute.
+ * Synchronises `stream`.  *status = MOE_OK or the first MOE_ERR_* code a
+ * kernel recorded; *detail (optional) = where it was recorded.
+ */
+int moe_read_status(void *ws, void *stream, int clear, int *status, int *detail);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEQ4_H */

@@ -64,6 +64,7 @@ def lib():
             L.oracle_route.argtypes = [vp, i64, i64, i64, C.c_int, vp, vp, vp]
             L.oracle_permute.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp]
             L.oracle_layer_forward.argtypes = [C.POINTER(_LayerArgs)]
+            L.oracle_combine.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
             _lib = L
     return _lib
 
@@ -129,6 +130,20 @@ def permute(ids, E):
     dp = np.empty(T * k, np.int32)
     _check(lib().oracle_permute(_p(ids), T, E, k, _p(counts), _p(offsets), _p(ss), _p(dp)), "permute")
     return counts, offsets, ss, dp
+
+
+def combine(Y, dest_pos, w, S=None, z=None):
+    """y [T, H] fp64 from expert rows Y [T k, H], dest_pos [T k], w [T, k]."""
+    Y = _c(Y, np.float64)
+    dp = _c(dest_pos, np.int32).reshape(-1)
+    w = _c(w, np.float64)
+    T, k = w.shape
+    H = Y.shape[1]
+    S = _c(S, np.float64)
+    z = _c(z, np.float64)
+    y = np.empty((T, H), np.float64)
+    _check(lib().oracle_combine(_p(Y), _p(dp), _p(w), _p(S), _p(z), T, H, k, _p(y)), "combine")
+    return y
 
 
 def layer_forward(layer: dict, sample=None, override_ids=None, override_w=None):

@@ -249,6 +249,35 @@ int oracle_permute(const int32_t *ids, int64_t T, int64_t E, int64_t k, int32_t 
     return ORACLE_OK;
 }
 
+/* -------------------------------------------------------------- combine */
+
+/*
+ * y[t] = sum_{j<k} w[t][j] * Y[dest_pos[t k + j]] + sigmoid(z[t]) * S[t]
+ * for given expert outputs Y [T k, H] and shared outputs S [T, H] (S and z
+ * may be NULL: no shared term).  Sums in fp64, j in order.
+ */
+int oracle_combine(const double *Y, const int32_t *dest_pos, const double *w, const double *S,
+                   const double *z, int64_t T, int64_t H, int64_t k, double *y)
+{
+    if (!Y || !dest_pos || !w || !y || T < 0 || H <= 0 || k <= 0)
+        return ORACLE_EINVAL;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t c = 0; c < H; ++c) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < k; ++j) {
+                int32_t p = dest_pos[t * k + j];
+                if (p < 0 || p >= T * k)
+                    return ORACLE_EINVAL;
+                acc += w[t * k + j] * Y[(int64_t)p * H + c];
+            }
+            if (S && z)
+                acc += 1.0 / (1.0 + exp(-z[t])) * S[t * H + c];
+            y[t * H + c] = acc;
+        }
+    }
+    return ORACLE_OK;
+}
+
 /* ------------------------------------------------------------ expert FFN */
 
 static double silu(double a) { return a / (1.0 + exp(-a)); }

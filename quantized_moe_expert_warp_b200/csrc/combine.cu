@@ -1,0 +1,77 @@
+// Weighted combine: y[t] = sum_j w[t,j] Y[dest_pos[t k + j]] + sigmoid(g_t) S[t].
+//
+// The pages state no combine rule; reading: the standard top-k mixture of
+// the routed experts' outputs plus the sigmoid-gated shared expert of the
+// Qwen3-Next-style layers run on the hipfire 0.4.3 benchmarks page.
+// One CTA per token pair; each thread owns 8 consecutive features and reads
+// them with 16-byte loads (coalesced across the warp); fp32 sums in j order.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+
+namespace moeq4 {
+
+__device__ __forceinline__ void add8(float (&acc)[8], const uint4 v, float w)
+{
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = fmaf(w, __uint_as_float(u[i] << 16), acc[2 * i]);
+        acc[2 * i + 1] = fmaf(w, __uint_as_float(u[i] & 0xFFFF0000u), acc[2 * i + 1]);
+    }
+}
+
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict__ y_perm,
+                                                      const int32_t *__restrict__ dest_pos,
+                                                      const float *__restrict__ w,
+                                                      const uint16_t *__restrict__ shared_out,
+                                                      const float *__restrict__ gate_logit, int T, int H, int k,
+                                                      uint16_t *__restrict__ y)
+{
+    const int chunks = H / 8;
+    const int per_cta_tokens = blockDim.x / chunks > 0 ? blockDim.x / chunks : 1;
+    if ((int)threadIdx.x / chunks >= per_cta_tokens)
+        return;
+    const int t = blockIdx.x * per_cta_tokens + threadIdx.x / chunks;
+    if (t >= T)
+        return;
+    const int S = T * k;
+    for (int c = threadIdx.x % chunks; c < chunks; c += blockDim.x) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < k; ++j) {
+            const int p = dest_pos[(size_t)t * k + j];
+            if (p < 0 || p >= S)
+                continue;
+            const uint4 v = *(const uint4 *)(y_perm + (size_t)p * H + c * 8);
+            add8(acc, v, w[(size_t)t * k + j]);
+        }
+        if (shared_out) {
+            const float g = gate_logit ? 1.0f / (1.0f + expf(-gate_logit[t])) : 1.0f;
+            add8(acc, *(const uint4 *)(shared_out + (size_t)t * H + c * 8), g);
+        }
+        uint4 o;
+        uint32_t *ou = &o.x;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t d;
+            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(acc[2 * i + 1]), "f"(acc[2 * i]));
+            ou[i] = d;
+        }
+        *(uint4 *)(y + (size_t)t * H + c * 8) = o;
+    }
+}
+
+cudaError_t launch_combine(const uint16_t *y_perm, const int32_t *dest_pos, const float *w, const uint16_t *shared_out,
+                           const float *gate_logit, int T, int H, int k, uint16_t *y, cudaStream_t st)
+{
+    if (T == 0)
+        return cudaSuccess;
+    const int chunks = H / 8;
+    const int threads = 256;
+    const int per = threads / chunks > 0 ? threads / chunks : 1;
+    combine_kernel<<<(T + per - 1) / per, threads, 0, st>>>(y_perm, dest_pos, w, shared_out, gate_logit, T, H, k, y);
+    return cudaGetLastError();
+}
+
+}  // namespace moeq4

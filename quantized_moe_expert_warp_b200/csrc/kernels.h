@@ -1,0 +1,56 @@
+// Internal launchers shared by the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "moeq4.h"
+
+namespace moeq4 {
+
+struct GemmArgs {
+    const uint8_t *wq;          // codes, kernel layout
+    const uint8_t *wmeta;       // scales / super-block headers, kernel layout
+    const uint16_t *b_src;      // token rows: x [T, H] (gathered) or h [rows, I]
+    int ldb;                    // elements per row of b_src
+    const int32_t *sorted_slot; // permutation (gather pass)
+    int topk;
+    int Tk;                     // T * k: rows at or past Tk belong to the shared expert
+    const int32_t *offsets;     // [E + 1] permutation offsets of the routed experts
+    int E;                      // routed experts
+    int T;                      // tokens (rows of the shared expert)
+    int E_total;                // E (+ 1 with a shared expert)
+    int K;                      // reduction length (H for gate/up, I for down)
+    int F;                      // 128-row tiles per expert matrix
+    int G;                      // int4-sym group size
+    int meta_bytes;             // per (expert, tile) meta block
+    uint16_t *out;              // routed rows: out + p * ldo
+    uint16_t *out_shared;       // shared rows: out_shared + (p - Tk) * ldo
+    int ldo;
+    int *status;                // [code, detail]
+};
+
+cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int num_sms, cudaStream_t st);
+size_t gemm_smem_required(int nmat, int meta_bytes, int E_total);
+
+cudaError_t launch_router_logits(const uint16_t *x, int T, int H, const float *wr, const float *bias, int E,
+                                 const float *gate_w, float *logits, float *gate_logit, cudaStream_t st);
+cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
+                         cudaStream_t st);
+
+size_t permute_scratch_bytes(int T, int E, int k);
+cudaError_t launch_permute(const int32_t *ids, int T, int E, int k, int32_t *counts, int32_t *offsets,
+                           int32_t *sorted_slot, int32_t *dest_pos, void *scratch, int *status, cudaStream_t st);
+
+cudaError_t launch_combine(const uint16_t *y_perm, const int32_t *dest_pos, const float *w, const uint16_t *shared_out,
+                           const float *gate_logit, int T, int H, int k, uint16_t *y, cudaStream_t st);
+
+cudaError_t launch_pack_codes(const moe_config_t &cfg, int which, const uint8_t *canon, uint8_t *out,
+                              cudaStream_t st);
+cudaError_t launch_pack_meta(const moe_config_t &cfg, int which, const uint8_t *canon, const uint16_t *scale,
+                             uint8_t *out, cudaStream_t st);
+cudaError_t launch_dequant_export(const moe_config_t &cfg, int which, int expert, const uint8_t *q,
+                                  const uint8_t *meta, float *out_f32, uint16_t *out_bf16, cudaStream_t st);
+
+}  // namespace moeq4

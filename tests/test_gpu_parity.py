@@ -1,0 +1,283 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Integer work (routing ids on oracle-supplied logits, counts, offsets, the
+permutation, dequantised weights) must match bit for bit; floating-point
+layer outputs must satisfy max|err| <= 2e-2 max|ref| and relative L2 <= 5e-3.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import check_close, compare_layer, run_layer, f32_to_bf16_rne
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import quantized_moe_expert_warp_b200 as mq
+    from quantized_moe_expert_warp_b200 import build
+    build.build()
+    mq.lib()
+    return torch.device("cuda", 0)
+
+
+def small_cfg(name, **kw):
+    d = dict(name=name, T=64, H=256, E=16, k=2, I=128, has_shared=False, wfmt=synth.WFMT_INT4_SYM,
+             G=32, wr_std=0.05, zipf_s=0.0, seed=21)
+    d.update(kw)
+    return synth.LayerConfig(**d)
+
+
+# ------------------------------------------------------------- dequant export
+
+@pytest.mark.parametrize("cfg,experts", [
+    (synth.get_config("tiny_t64"), [0, 7, 15]),
+    (small_cfg("g128", H=512, I=256, E=4, G=128, has_shared=True), [0, 4]),
+    (small_cfg("q4k", H=512, I=256, E=3, G=256, wfmt=synth.WFMT_Q4K, has_shared=True), [0, 2, 3]),
+])
+def test_dequant_export_bitexact(dev, cfg, experts):
+    import quantized_moe_expert_warp_b200 as mq
+    from quantized_moe_expert_warp_b200.host import upload_layer
+    layer = synth.make_layer(cfg)
+    packed = upload_layer(layer, dev)
+    H, I = cfg.H, cfg.I
+    for e in experts:
+        for which, (rows, K) in enumerate([(2 * I, H), (H, I)]):
+            f32 = torch.empty((rows, K), dtype=torch.float32, device=dev)
+            b16 = torch.empty((rows, K), dtype=torch.int16, device=dev)
+            q, meta = (packed.gu_q, packed.gu_meta) if which == 0 else (packed.dn_q, packed.dn_meta)
+            mq.moe_dequant_export(cfg, q, meta, which, e, f32, b16)
+            if cfg.wfmt == synth.WFMT_Q4K:
+                src = layer["gu_q4k"][e] if which == 0 else layer["dn_q4k"][e]
+                ref = oracle.dequant_q4k(src, rows, K)
+            else:
+                nib = layer["gu_nib"][e] if which == 0 else layer["dn_nib"][e]
+                sc = layer["gu_scale"][e] if which == 0 else layer["dn_scale"][e]
+                ref = oracle.dequant_int4sym(nib, sc, rows, K, cfg.G)
+            got = f32.cpu().numpy()
+            assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), (e, which)
+            got16 = b16.cpu().numpy().view(np.uint16)
+            assert np.array_equal(got16, synth.f32_to_bf16_bits(ref)), (e, which)
+
+
+# ------------------------------------------------------------------ routing
+
+def gpu_route(dev, logits, k, renorm=True):
+    import quantized_moe_expert_warp_b200 as mq
+    T, E = logits.shape
+    L = torch.from_numpy(np.ascontiguousarray(logits, np.float32)).to(dev)
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    mq.moe_route(L, T, E, k, renorm, ids, w)
+    return ids.cpu().numpy(), w.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", ["tiny_t64", "a3b_t512", "a3b_t8192_zipf", "a3b_decode_t32"])
+def test_route_bitexact_on_oracle_logits(dev, name):
+    cfg = synth.get_config(name)
+    layer = synth.make_layer(cfg, experts=[])
+    logits = oracle.router_logits(layer["x"], layer["router_w"], layer.get("router_bias"))
+    ids_ref, w_ref, _ = oracle.route(logits, cfg.k, cfg.renorm)
+    ids, w = gpu_route(dev, logits, cfg.k, cfg.renorm)
+    assert np.array_equal(ids, ids_ref)
+    np.testing.assert_allclose(w, w_ref, rtol=2e-6, atol=1e-7)
+
+
+@pytest.mark.parametrize("E,k,renorm", [(16, 2, True), (256, 8, True), (256, 8, False), (33, 7, True),
+                                        (1024, 32, True), (8, 8, True), (1, 1, True)])
+def test_route_bitexact_with_ties(dev, E, k, renorm):
+    rng = np.random.default_rng(E + k)
+    T = 300
+    L = rng.normal(size=(T, E)).astype(np.float32)
+    L[::7] = np.round(L[::7] * 2) / 2       # many exact ties
+    L[3] = 0.0                              # all equal
+    L[4] = -0.0
+    L[5, ::2] = -0.0
+    ids_ref, w_ref, _ = oracle.route(L, k, renorm)
+    ids, w = gpu_route(dev, L, k, renorm)
+    assert np.array_equal(ids, ids_ref)
+    np.testing.assert_allclose(w, w_ref, rtol=2e-6, atol=1e-7)
+
+
+# -------------------------------------------------------------- permutation
+
+def gpu_permute(dev, ids, E):
+    import quantized_moe_expert_warp_b200 as mq
+    T, k = ids.shape
+    d_ids = torch.from_numpy(np.ascontiguousarray(ids, np.int32)).to(dev)
+    counts = torch.full((E,), -7, dtype=torch.int32, device=dev)
+    offsets = torch.full((E + 1,), -7, dtype=torch.int32, device=dev)
+    ss = torch.full((max(1, T * k),), -7, dtype=torch.int32, device=dev)
+    dp = torch.full((max(1, T * k),), -7, dtype=torch.int32, device=dev)
+    n = mq.moe_permute_workspace_size(T, E, k)
+    ws = torch.zeros(n, dtype=torch.uint8, device=dev)
+    mq.moe_permute(d_ids, T, E, k, counts, offsets, ss, dp, ws, n)
+    st, _ = mq.moe_read_status(ws)
+    assert st == 0
+    return counts.cpu().numpy(), offsets.cpu().numpy(), ss.cpu().numpy()[:T * k], dp.cpu().numpy()[:T * k]
+
+
+@pytest.mark.parametrize("T,E,k,skew", [(64, 16, 2, 0), (1, 256, 8, 0), (7, 3, 3, 0), (513, 256, 8, 0),
+                                        (8192, 256, 8, 1), (4096, 1024, 32, 0), (300, 64, 4, 2)])
+def test_permute_bitexact(dev, T, E, k, skew):
+    rng = np.random.default_rng(T * 31 + E)
+    if skew == 0:
+        ids = np.stack([rng.permutation(E)[:k] for _ in range(T)])
+    else:
+        # Zipf-like preference: a few experts take most slots, many stay empty
+        p = 1.0 / np.arange(1, E + 1) ** (1.1 if skew == 1 else 3.0)
+        p /= p.sum()
+        ids = np.stack([rng.choice(E, size=k, replace=False, p=p) for _ in range(T)])
+    ids = ids.astype(np.int32)
+    ref = oracle.permute(ids, E)
+    got = gpu_permute(dev, ids, E)
+    for a, b in zip(got, ref):
+        assert np.array_equal(a, b)
+
+
+# ------------------------------------------------------------------ combine
+
+@pytest.mark.parametrize("T,H,k,shared", [(64, 256, 2, False), (37, 2048, 8, True), (5, 4096, 3, True)])
+def test_combine(dev, T, H, k, shared):
+    import quantized_moe_expert_warp_b200 as mq
+    rng = np.random.default_rng(T + H)
+    Y = synth.f32_to_bf16_bits(rng.normal(size=(T * k, H)))
+    S = synth.f32_to_bf16_bits(rng.normal(size=(T, H))) if shared else None
+    z = rng.normal(size=T).astype(np.float32) if shared else None
+    dp = rng.permutation(T * k).astype(np.int32)
+    w = rng.uniform(0, 1, size=(T, k)).astype(np.float32)
+    to = lambda a, dt=None: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    mq.moe_combine(to(Y.view(np.int16)), to(dp), to(w), to(None if S is None else S.view(np.int16)), to(z),
+                   T, H, k, y)
+    ref = oracle.combine(synth.bf16_bits_to_f32(Y), dp, w,
+                         None if S is None else synth.bf16_bits_to_f32(S), z)
+    got = y.float().cpu().numpy()
+    # fp32 sums then one bf16 rounding: within one bf16 half-ulp plus fp32 noise
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6)
+
+
+# ---------------------------------------------------------- router logits
+
+def test_router_logits_close(dev):
+    import quantized_moe_expert_warp_b200 as mq
+    from quantized_moe_expert_warp_b200.host import upload_layer, x_to_device
+    cfg = synth.get_config("a3b_t512").with_T(200, "router_check").with_(zipf_s=1.1)
+    layer = synth.make_layer(cfg, experts=[])
+    packed = upload_layer(layer, dev)
+    x = x_to_device(layer["x"], dev)
+    logits = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=dev)
+    gl = torch.empty((cfg.T,), dtype=torch.float32, device=dev)
+    mq.moe_router_logits(packed, x, cfg.T, logits, gl)
+    ref = oracle.router_logits(layer["x"], layer["router_w"], layer["router_bias"])
+    np.testing.assert_allclose(logits.cpu().numpy(), ref, rtol=0, atol=2e-5)
+    xs = synth.bf16_bits_to_f32(layer["x"]).astype(np.float64)
+    np.testing.assert_allclose(gl.cpu().numpy(), xs @ layer["shared_gate"].astype(np.float64), atol=2e-5)
+
+
+# -------------------------------------------------------------- whole layer
+
+SMALL_LAYERS = [
+    synth.get_config("tiny_t64"),
+    # several token tiles per expert with a ragged tail, shared expert, G = 64
+    small_cfg("ragged_shared", T=300, H=512, E=8, k=2, I=256, has_shared=True, G=64, wr_std=0.03),
+    # top-1 routing, unrenormalised weights
+    small_cfg("top1_norenorm", T=97, H=256, E=4, k=1, I=128, renorm=False),
+    # Q4K super-blocks, shared expert, K = H = 512 and K = I = 256
+    small_cfg("q4k_small", T=130, H=512, E=6, k=3, I=256, has_shared=True, G=256, wfmt=synth.WFMT_Q4K),
+    # a single token (decode), many experts
+    small_cfg("one_token", T=1, H=512, E=64, k=8, I=128, has_shared=True, G=128),
+    # every expert gets > 128 rows: multi-tile experts without a shared expert
+    small_cfg("big_groups", T=600, H=256, E=4, k=2, I=384, G=128, wr_std=0.02),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL_LAYERS, ids=lambda c: c.name)
+def test_layer_matches_oracle(dev, cfg):
+    layer = synth.make_layer(cfg)
+    got = run_layer(layer, dev)
+    ref, ties, _ = compare_layer(layer, got)
+    # integer intermediates are exact (the oracle's routing, redone where near-ties flipped)
+    assert np.array_equal(got["counts"], ref["counts"])
+    assert np.array_equal(got["offsets"], ref["offsets"])
+    assert np.array_equal(got["sorted_slot"], ref["sorted_slot"])
+    assert np.array_equal(got["dest_pos"], ref["dest_pos"])
+
+
+@pytest.mark.parametrize("cfg", SMALL_LAYERS[:4], ids=lambda c: c.name)
+def test_layer_with_oracle_routing_override(dev, cfg):
+    layer = synth.make_layer(cfg)
+    ref = oracle.layer_forward(layer)
+    got = run_layer(layer, dev, override_ids=ref["ids"], override_w=ref["w"])
+    assert np.array_equal(got["sorted_slot"], ref["sorted_slot"])
+    check_close(got["y"], ref["y"], cfg.name)
+
+
+@pytest.mark.parametrize("cfg", [SMALL_LAYERS[1], SMALL_LAYERS[3]], ids=lambda c: c.name)
+def test_fused_equals_composed_bitwise(dev, cfg):
+    import quantized_moe_expert_warp_b200 as mq
+    from quantized_moe_expert_warp_b200.host import upload_layer, x_to_device
+    layer = synth.make_layer(cfg)
+    packed = upload_layer(layer, dev)
+    fused = run_layer(layer, dev, packed=packed)
+    T, E, k, H = cfg.T, cfg.E, cfg.k, cfg.H
+    x = x_to_device(layer["x"], dev)
+    e32 = lambda *s: torch.empty(s, dtype=torch.float32, device=dev)
+    i32 = lambda *s: torch.empty(s, dtype=torch.int32, device=dev)
+    logits, gl = e32(T, E), e32(T)
+    ids, w = i32(T, k), e32(T, k)
+    counts, offsets, ss, dp = i32(E), i32(E + 1), i32(T * k), i32(T * k)
+    mq.moe_router_logits(packed, x, T, logits, gl)
+    mq.moe_route(logits, T, E, k, cfg.renorm, ids, w)
+    n = mq.moe_permute_workspace_size(T, E, k)
+    pws = torch.zeros(n, dtype=torch.uint8, device=dev)
+    mq.moe_permute(ids, T, E, k, counts, offsets, ss, dp, pws, n)
+    y_perm = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
+    sh = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if cfg.has_shared else None
+    n = mq.moe_expert_ffn_workspace_size(cfg, T)
+    fws = torch.zeros(n, dtype=torch.uint8, device=dev)
+    mq.moe_expert_ffn_q4(packed, x, T, ss, offsets, y_perm, sh, fws, n)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    mq.moe_combine(y_perm, dp, w, sh, gl if cfg.has_shared else None, T, H, k, y)
+    assert mq.moe_read_status(fws)[0] == 0
+    assert torch.equal(y.view(torch.int16), fused["y_bf16"].view(torch.int16))
+
+
+def test_layer_is_deterministic(dev):
+    from quantized_moe_expert_warp_b200.host import upload_layer
+    layer = synth.make_layer(SMALL_LAYERS[1])
+    packed = upload_layer(layer, dev)
+    a = run_layer(layer, dev, packed=packed)["y_bf16"]
+    b = run_layer(layer, dev, packed=packed)["y_bf16"]
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+# --------------------------------------------------------- full-size layers
+
+FULL = [("a3b_t512", 96), ("a3b_t8192_zipf", 48), ("a3b_t4096_q4k", 40),
+        ("a3b_decode_t1", None), ("a3b_decode_t8", None), ("a3b_decode_t32", None)]
+
+
+@pytest.mark.parametrize("name,nsample", FULL, ids=[f[0] for f in FULL])
+def test_full_size_layer_sampled(dev, name, nsample):
+    cfg = synth.get_config(name)
+    layer = synth.make_layer(cfg)
+    got = run_layer(layer, dev)
+    sample = None
+    if nsample is not None:
+        rng = np.random.default_rng(123)
+        sample = np.sort(np.concatenate([[0, cfg.T - 1], rng.choice(np.arange(1, cfg.T - 1), nsample - 2,
+                                                                   replace=False)]))
+    ref, ties, stats = compare_layer(layer, got, sample=sample)
+    # routing, counts and the permutation are exact (up to accepted near-ties)
+    if len(ties) == 0:
+        assert np.array_equal(got["counts"], ref["counts"])
+        assert np.array_equal(got["sorted_slot"], ref["sorted_slot"])
+    assert got["counts"].sum() == cfg.T * cfg.k
+    print(f"{name}: max|err|/max|ref| {stats[0]:.2e} rel L2 {stats[1]:.2e} near-ties {len(ties)}")

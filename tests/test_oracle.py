@@ -233,6 +233,21 @@ def test_permutation_empty_experts():
     assert offsets.tolist() == [0, 4, 4, 4, 4, 4]
 
 
+# ---------------------------------------------------------------- combine
+
+def test_combine_closed_form():
+    # two tokens, k = 2, H = 2; rows placed out of order by dest_pos
+    Y = np.array([[1.0, 2.0], [10.0, 20.0], [100.0, 200.0], [-1.0, 0.5]])
+    dest_pos = np.array([2, 0, 3, 1], np.int32)
+    w = np.array([[0.75, 0.25], [0.5, 0.5]])
+    S = np.array([[4.0, 8.0], [0.0, 2.0]])
+    z = np.array([0.0, math.log(3.0)])          # sigmoid: 1/2 and 3/4
+    y = oracle.combine(Y, dest_pos, w, S, z)
+    assert y[0].tolist() == [0.75 * 100 + 0.25 * 1 + 2.0, 0.75 * 200 + 0.25 * 2 + 4.0]
+    assert np.allclose(y[1], [0.5 * -1 + 0.5 * 10 + 0.0, 0.5 * 0.5 + 0.5 * 20 + 1.5], rtol=1e-15)
+    assert np.array_equal(oracle.combine(Y, dest_pos, w), y - np.array([[2.0, 4.0], [0.0, 1.5]]))
+
+
 # ------------------------------------------------------------- whole layer
 
 def sig(z):
