@@ -176,7 +176,10 @@ def test_router_logits_close(dev):
     gl = torch.empty((cfg.T,), dtype=torch.float32, device=dev)
     mq.moe_router_logits(packed, x, cfg.T, logits, gl)
     ref = oracle.router_logits(layer["x"], layer["router_w"], layer["router_bias"])
-    np.testing.assert_allclose(logits.cpu().numpy(), ref, rtol=0, atol=2e-5)
+    # bf16 x is exact; fp32 weights enter as three bf16 parts with exact products,
+    # summed by the tensor cores' fp32 accumulation (truncating adds over
+    # H / 16 = 128 partial blocks): |err| ~ 1e-5 for |logit| up to ~8
+    np.testing.assert_allclose(logits.cpu().numpy(), ref, rtol=0, atol=1e-4)
     xs = synth.bf16_bits_to_f32(layer["x"]).astype(np.float64)
     np.testing.assert_allclose(gl.cpu().numpy(), xs @ layer["shared_gate"].astype(np.float64), atol=2e-5)
 
