@@ -323,8 +323,8 @@ int moe_router_logits(const moe_layer_t *L, const uint16_t *x, int T, float *log
     const float *g = L->cfg.has_shared && gate_logit ? L->shared_gate : nullptr;
     if (g)
         REQUIRE_PTR(gate_logit);
-    CUDA_TRY(launch_router_logits(x, T, L->cfg.H, L->router_w, L->router_bias, L->cfg.E, g, logits,
-                                  g ? gate_logit : nullptr, (cudaStream_t)stream),
+    CUDA_TRY(launch_router_gemm(x, T, L->cfg.H, L->router_w, L->router_bias, L->cfg.E, g, logits,
+                                g ? gate_logit : nullptr, nullptr, num_sms(), (cudaStream_t)stream),
              "router logits");
     g_launches += 1;
     return ok();
@@ -512,8 +512,8 @@ int moe_layer_forward(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *
         REQUIRE_PTR(dbg->override_w);
     }
     const float *g = c.has_shared ? L->shared_gate : nullptr;
-    CUDA_TRY(launch_router_logits(x, T, c.H, L->router_w, L->router_bias, c.E, g, w.logits, g ? w.gate_logit : nullptr,
-                                  st),
+    CUDA_TRY(launch_router_gemm(x, T, c.H, L->router_w, L->router_bias, c.E, g, w.logits, g ? w.gate_logit : nullptr,
+                                w.status, num_sms(), st),
              "router logits");
     g_launches += 1;
     const int32_t *ids = w.ids;

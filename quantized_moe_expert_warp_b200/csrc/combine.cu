@@ -37,14 +37,25 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict
     if (t >= T)
         return;
     const int S = T * k;
+    const int32_t *dp = dest_pos + (size_t)t * k;
+    const float *wt = w + (size_t)t * k;
     for (int c = threadIdx.x % chunks; c < chunks; c += blockDim.x) {
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < k; ++j) {
-            const int p = dest_pos[(size_t)t * k + j];
-            if (p < 0 || p >= S)
-                continue;
-            const uint4 v = *(const uint4 *)(y_perm + (size_t)p * H + c * 8);
-            add8(acc, v, w[(size_t)t * k + j]);
+        // batches of 8 rows: all loads of a batch are in flight together
+        for (int j0 = 0; j0 < k; j0 += 8) {
+            uint4 v[8];
+            float wj[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int p = j0 + j < k ? dp[j0 + j] : -1;
+                const bool ok = p >= 0 && p < S;
+                wj[j] = ok ? wt[j0 + j] : 0.f;
+                v[j] = ok ? *(const uint4 *)(y_perm + (size_t)p * H + c * 8) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j0 + j < k)
+                    add8(acc, v[j], wj[j]);
         }
         if (shared_out) {
             const float g = gate_logit ? 1.0f / (1.0f + expf(-gate_logit[t])) : 1.0f;

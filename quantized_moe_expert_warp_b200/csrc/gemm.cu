@@ -1,4 +1,4 @@
-// Grouped expert GEMMs on 4-bit weights, tcgen05 tensor cores.
+// Grouped expert GEMMs on 4-bit weights (and the router GEMM), tcgen05 tensor cores.
 //
 // hipfire 0.4.3 benchmarks, "Read this before comparing columns": the MoE
 // prefill route either keeps per-expert buffers or takes the "symmetric
@@ -11,13 +11,19 @@
 // dequant warps write them straight into tensor memory (TMEM), where the
 // MMA reads its A operand, and the tokens are gathered into swizzled
 // shared memory as the B operand.  The accumulator stays in TMEM until the
-// epilogue warps apply SwiGLU (gate/up pass) or round to bf16 (down pass).
+// epilogue warps apply SwiGLU (gate/up pass), round to bf16 (down pass) or
+// add the router bias (router pass).
+//
+// The router pass uses the same engine: its fp32 weights are split into
+// three bf16 parts (hi + mid + lo carry all 24 significand bits), the three
+// products are exact in fp32 and accumulate into one fp32 accumulator.
 //
 // Warp roles of one persistent CTA (one per SM, 512 threads):
 //   warp 0      gathers token rows of B with cp.async (zero rows past the tail)
 //   warp 1      issues tcgen05.mma (one thread) and commits stage releases
 //   warp 2      streams code blocks and per-tile scale blocks with bulk copies
-//   warp 3      owns the TMEM allocation
+//   warp 3      owns the TMEM allocation; in the router pass it also forms
+//               the shared expert's gate logits x . g
 //   warps 4-11  dequantise: row r = 32*(warp%4) + lane, half c = (warp-4)/4
 //   warps 12-15 epilogue (TMEM -> registers -> global)
 // Every wait is bounded; on timeout the CTA records MOE_ERR_TIMEOUT and
@@ -26,26 +32,53 @@
 #include <cuda_runtime.h>
 
 #include "dequant.cuh"
+#include "kernels.h"
 #include "moeq4.h"
 #include "ptx.cuh"
-#include "kernels.h"
 
 namespace moeq4 {
 
-constexpr int kBN = 128;           // max tokens per tile (the MMA's N)
-constexpr int kStages = 4;         // B / TMEM-A pipeline depth
-constexpr int kThreads = 512;
-constexpr int kLag = kStages - 1;  // cp.async groups in flight before a stage is signalled
+// Optional timeline instrumentation: with -DMOEQ4_TRACE the first four CTAs
+// record %globaltimer at pipeline events into g_trace[cta][event][step]
+// (read back with moe_trace_fetch); without it the hooks compile to nothing.
+#if defined(MOEQ4_TRACE) && defined(MOEQ4_TRACE_WARPS)
+#define TRACE_OTHER(ev, step) do { } while (0)
+#else
+#define TRACE_OTHER(ev, step) TRACE_EVENT(ev, step)
+#endif
+#ifdef MOEQ4_TRACE
+constexpr int kTraceSteps = 512;
+__device__ unsigned long long g_trace[4][16][kTraceSteps];
+#define TRACE_EVENT(ev, step)                                                          \
+    do {                                                                               \
+        if (blockIdx.x < 4 && (step) >= 0 && (step) < kTraceSteps)                     \
+            g_trace[blockIdx.x][(ev)][(step)] = globaltimer_ns();                      \
+    } while (0)
+#else
+#define TRACE_EVENT(ev, step) \
+    do {                      \
+    } while (0)
+#endif
 
-template <int NMAT>
-struct GemmSmem {
-    static constexpr int kCodeStages = NMAT == 2 ? 8 : 16;
+constexpr int kBN = 128;     // max tokens per tile (the MMA's N)
+constexpr int kStages = 4;   // B / TMEM-A pipeline depth
+constexpr int kThreads = 512;
+
+enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_ROUTER = 2 };
+
+template <int MODE>
+struct Geo {
+    static constexpr int kNA = MODE == MODE_GATE_UP ? 2 : MODE == MODE_DOWN ? 1 : 3;   // A operands per k-step
+    static constexpr int kNAcc = MODE == MODE_GATE_UP ? 2 : 1;                          // accumulators per unit
+    static constexpr int kAccBufs = MODE == MODE_DOWN ? 2 : 1;                          // accumulator buffers
+    static constexpr int kNCode = MODE == MODE_GATE_UP ? 2 : MODE == MODE_DOWN ? 1 : 0; // code matrices
+    static constexpr int kCodeStages = MODE == MODE_GATE_UP ? 8 : MODE == MODE_DOWN ? 16 : 1;
+    static constexpr int kCodeBytes = kCodeStages * (kNCode ? code_block_bytes(kNCode) : 0);
     static constexpr int kBBytes = kStages * kBN * 128;
-    static constexpr int kCodeBytes = kCodeStages * code_block_bytes(NMAT);
-    static constexpr int kTmemCols = NMAT == 2 ? 512 : 256;
-    static constexpr int kAccCols = NMAT * kBN;
-    // A stages follow the accumulators in TMEM
-    static_assert(kAccCols + kStages * NMAT * 32 <= kTmemCols, "TMEM budget");
+    static constexpr int kAccCols = kAccBufs * kNAcc * kBN;
+    static constexpr int kTmemCols = 512;
+    static_assert(kAccCols + kStages * kNA * 32 <= kTmemCols, "TMEM budget");
+    static constexpr bool kGather = MODE == MODE_GATE_UP;
 };
 
 struct Barriers {
@@ -56,11 +89,12 @@ struct Barriers {
     uint64_t code_empty[16];
     uint64_t meta_full[2];
     uint64_t meta_empty[2];
-    uint64_t acc_full;
-    uint64_t acc_empty;
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
+    int never_abort;   // stays 0: a wait that must not be cut short by an abort
 };
 
 struct Unit {
@@ -97,6 +131,7 @@ __device__ __forceinline__ Unit decode_unit(int u, const GemmArgs &p, const Sche
 // Every CTA derives the tile schedule from the permutation offsets: rows of
 // expert e are [offsets[e], offsets[e+1]); the shared expert (if any) is
 // expert E with rows [T k, T k + T); expert e owns ceil(rows / kBN) tiles.
+// Without offsets (router pass) the T token rows form a single group.
 __device__ void build_schedule(const GemmArgs &p, int *s_tile_start, int *s_row_start, int *s_row_count,
                                int *s_part)
 {
@@ -105,8 +140,17 @@ __device__ void build_schedule(const GemmArgs &p, int *s_tile_start, int *s_row_
     const int e0 = threadIdx.x * per;
     int local = 0;
     for (int e = e0; e < min(n, e0 + per); ++e) {
-        const int start = e < p.E ? p.offsets[e] : p.Tk;
-        const int cnt = e < p.E ? p.offsets[e + 1] - p.offsets[e] : p.T;
+        int start, cnt;
+        if (!p.offsets) {
+            start = 0;
+            cnt = p.T;
+        } else if (e < p.E) {
+            start = p.offsets[e];
+            cnt = p.offsets[e + 1] - p.offsets[e];
+        } else {
+            start = p.Tk;
+            cnt = p.T;
+        }
         s_row_start[e] = start;
         s_row_count[e] = cnt;
         local += (cnt + kBN - 1) / kBN;
@@ -128,18 +172,34 @@ __device__ void build_schedule(const GemmArgs &p, int *s_tile_start, int *s_row_
         s_tile_start[n] = s_part[kThreads - 1];
 }
 
-template <int NMAT, int WFMT, bool GATHER>
-__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_q4_kernel(const GemmArgs p)
+// fp32 -> three bf16 parts (hi, mid, lo): w - hi and (w - hi) - mid are exact
+// in fp32, so hi + mid + lo matches w to about 2^-24 relative.
+__device__ __forceinline__ void split3(float w0, float w1, uint32_t &hi, uint32_t &mid, uint32_t &lo)
 {
-    using L = GemmSmem<NMAT>;
+    hi = pack_bf16x2(w0, w1);
+    const float r0 = w0 - __uint_as_float(hi << 16);
+    const float r1 = w1 - __uint_as_float(hi & 0xFFFF0000u);
+    mid = pack_bf16x2(r0, r1);
+    const float s0 = r0 - __uint_as_float(mid << 16);
+    const float s1 = r1 - __uint_as_float(mid & 0xFFFF0000u);
+    lo = pack_bf16x2(s0, s1);
+}
+
+template <int MODE, int WFMT>
+__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArgs p)
+{
+    using L = Geo<MODE>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled B stages
-    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    // offset arithmetic on the shared array keeps the pointer in the shared
+    // window (a round trip through an integer would make every access generic)
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *sB = smem;
     uint8_t *sCode = sB + L::kBBytes;
     uint8_t *sMeta = sCode + L::kCodeBytes;
     const int meta_bytes = p.meta_bytes;
-    Barriers *bars = (Barriers *)(sMeta + 2 * ((meta_bytes + 127) & ~127));
+    const int meta_al = (meta_bytes + 127) & ~127;
+    Barriers *bars = (Barriers *)(sMeta + 2 * meta_al);
     int *s_tile_start = (int *)(bars + 1);
     int *s_row_start = s_tile_start + p.E_total + 1;
     int *s_row_count = s_row_start + p.E_total;
@@ -151,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_q4_kernel(const Gemm
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&bars->b_full[s], 1);
+            mbar_init(&bars->b_full[s], 32);   // one cp.async completion arrival per lane
             mbar_init(&bars->a_full[s], 8);
             mbar_init(&bars->mma_done[s], 1);
         }
@@ -162,11 +222,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_q4_kernel(const Gemm
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->meta_full[s], 1);
             mbar_init(&bars->meta_empty[s], 8);
+            mbar_init(&bars->acc_full[s], 1);
+            mbar_init(&bars->acc_empty[s], 4);
         }
-        mbar_init(&bars->acc_full, 1);
-        mbar_init(&bars->acc_empty, 4);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
+        bars->never_abort = 0;
         fence_mbar_init();
     }
     build_schedule(p, s_tile_start, s_row_start, s_row_count, s_part);
@@ -197,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_q4_kernel(const Gemm
                 const int prow = un.row0 + r;
                 int srow = 0;
                 if (r < un.nvalid)
-                    srow = GATHER ? (prow < p.Tk ? p.sorted_slot[prow] / p.topk : prow - p.Tk) : prow;
+                    srow = L::kGather ? (prow < p.Tk ? p.sorted_slot[prow] / p.topk : prow - p.Tk) : prow;
                 src[i] = p.b_src + (size_t)srow * p.ldb;
                 bytes[i] = r < un.nvalid ? 16u : 0u;
             }
@@ -219,90 +280,140 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_q4_kernel(const Gemm
                             cp_async_16(rbase + ((j ^ (r & 7)) << 4), g + j * 8, bytes[i]);
                     }
                 }
-                cp_async_commit();
-                if (step >= kLag) {
-                    cp_async_wait_group<kLag>();
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(&bars->b_full[(step - kLag) % kStages]);
-                }
+                // this lane's copies for the stage arrive on b_full[s] when they land
+                cp_async_arrive_noinc(&bars->b_full[s]);
+                if (lane == 0)
+                    TRACE_OTHER(0, step);
             }
         }
-        cp_async_wait_group<0>();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0)
-            for (int s = max(0, step - kLag); s < step; ++s)
-                mbar_arrive(&bars->b_full[s % kStages]);
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            int step = 0, uidx = 0;
-            bool ok = true;
-            for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++uidx) {
-                const Unit un = decode_unit(u, p, sched);
-                const uint32_t idesc = idesc_bf16_f32(128, un.nmma);
-                if (uidx > 0) {
-                    if (!mbar_wait(&bars->acc_empty, (uidx - 1) & 1, wc, 2))
-                        break;
-                    tc_fence_after();
-                }
-                for (int ks = 0; ks < KS; ++ks, ++step) {
-                    const int s = step % kStages;
-                    const uint32_t ph = (step / kStages) & 1;
-                    if (!mbar_wait(&bars->a_full[s], ph, wc, 3) || !mbar_wait(&bars->b_full[s], ph, wc, 4)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t bbase = smem_u32(sB + s * kBN * 128);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t bdesc = sdesc_kmajor_sw128(bbase + kk * 32);
-#pragma unroll
-                        for (int m = 0; m < NMAT; ++m) {
-                            const uint32_t a_t = tmem + L::kAccCols + (s * NMAT + m) * 32 + kk * 8;
-                            mma_ts_f16(tmem + m * kBN, a_t, bdesc, idesc, (ks | kk) != 0);
-                        }
-                    }
-                    mma_commit(&bars->mma_done[s]);
-                }
-                if (ok)
-                    mma_commit(&bars->acc_full);
+        // ------------------------------------------------ MMA issuer (converged warp, one elected lane)
+        int step = 0, uidx = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++uidx) {
+            const Unit un = decode_unit(u, p, sched);
+            const uint32_t idesc = idesc_bf16_f32(128, un.nmma);
+            const int ab = uidx % L::kAccBufs;
+            const uint32_t acc = tmem + ab * L::kNAcc * kBN;
+            if (uidx >= L::kAccBufs) {
+                if (!warp_wait(&bars->acc_empty[ab], ((uidx / L::kAccBufs) & 1) ^ 1, wc, 2))
+                    break;
+                tc_fence_after();
             }
-            // all issued MMAs finish before the CTA may release TMEM
-            mma_commit(&bars->drain);
-            WaitCtx wd{&bars->abort_flag, p.status, globaltimer_ns()};
-            int zero = 0;
-            wd.abort_flag = &zero;   // wait for the drain even after an abort
-            mbar_wait(&bars->drain, 0, wd, 5);
+            for (int ks = 0; ks < KS; ++ks, ++step) {
+                const int s = step % kStages;
+                const uint32_t ph = (step / kStages) & 1;
+                if (!warp_wait(&bars->a_full[s], ph, wc, 3)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0)
+                    TRACE_OTHER(8, step);
+                if (!warp_wait(&bars->b_full[s], ph, wc, 4)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0)
+                    TRACE_OTHER(9, step);
+                // the B stage was written by cp.async (generic proxy); the MMA
+                // reads it through the async proxy
+                fence_proxy_async_smem();
+                tc_fence_after();
+                const uint32_t bbase = smem_u32(sB + s * kBN * 128);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t bdesc = sdesc_kmajor_sw128(bbase + kk * 32);
+#pragma unroll
+                    for (int m = 0; m < L::kNA; ++m) {
+                        const uint32_t a_t = tmem + L::kAccCols + (s * L::kNA + m) * 32 + kk * 8;
+                        if (elect_one()) {
+                            if (MODE == MODE_ROUTER)   // three parts into one accumulator
+                                mma_ts_f16(acc, a_t, bdesc, idesc, (ks | kk | m) != 0);
+                            else
+                                mma_ts_f16(acc + m * kBN, a_t, bdesc, idesc, (ks | kk) != 0);
+                        }
+                        __syncwarp();
+                    }
+                }
+                if (lane == 0)
+                    TRACE_OTHER(10, step);
+                if (elect_one())
+                    mma_commit(&bars->mma_done[s]);
+                __syncwarp();
+                if (lane == 0)
+                    TRACE_OTHER(5, step);
+            }
+            if (ok) {
+                if (elect_one())
+                    mma_commit(&bars->acc_full[ab]);
+                __syncwarp();
+            }
         }
+        // all issued MMAs finish before the CTA may release TMEM
+        if (elect_one())
+            mma_commit(&bars->drain);
+        __syncwarp();
+        WaitCtx wd{&bars->never_abort, p.status, globaltimer_ns()};   // drain even after an abort
+        warp_wait(&bars->drain, 0, wd, 5);
     } else if (warp == 2) {
-        // ------------------------------------------------ code / meta producer
-        if (lane == 0) {
+        // ------------------------------------------------ code / meta producer (converged warp)
+        if (MODE != MODE_ROUTER) {
             int step = 0, munit = 0;
-            const int cbytes = code_block_bytes(NMAT);
+            const int cbytes = code_block_bytes(L::kNCode);
             bool ok = true;
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++munit) {
                 const Unit un = decode_unit(u, p, sched);
                 const size_t tile_id = (size_t)un.e * p.F + un.f;
                 const int mb = munit & 1;
-                if (munit >= 2 && !mbar_wait(&bars->meta_empty[mb], ((munit >> 1) & 1) ^ 1, wc, 6))
+                if (munit >= 2 && !warp_wait(&bars->meta_empty[mb], ((munit >> 1) & 1) ^ 1, wc, 6))
                     break;
-                mbar_arrive_expect_tx(&bars->meta_full[mb], meta_bytes);
-                bulk_g2s(sMeta + mb * ((meta_bytes + 127) & ~127), p.wmeta + tile_id * meta_bytes, meta_bytes,
-                         &bars->meta_full[mb]);
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&bars->meta_full[mb], meta_bytes);
+                    bulk_g2s(sMeta + mb * meta_al, p.wmeta + tile_id * meta_bytes, meta_bytes, &bars->meta_full[mb]);
+                }
+                __syncwarp();
                 for (int ks = 0; ks < KS; ++ks, ++step) {
                     const int s = step % L::kCodeStages;
                     if (step >= L::kCodeStages &&
-                        !mbar_wait(&bars->code_empty[s], ((step / L::kCodeStages) & 1) ^ 1, wc, 7)) {
+                        !warp_wait(&bars->code_empty[s], ((step / L::kCodeStages) & 1) ^ 1, wc, 7)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&bars->code_full[s], cbytes);
-                    bulk_g2s(sCode + s * cbytes, p.wq + (tile_id * KS + ks) * cbytes, cbytes, &bars->code_full[s]);
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(&bars->code_full[s], cbytes);
+                        bulk_g2s(sCode + s * cbytes, p.wq + (tile_id * KS + ks) * cbytes, cbytes,
+                                 &bars->code_full[s]);
+                    }
+                    __syncwarp();
+                    if (lane == 0)
+                        TRACE_OTHER(1, step);
                 }
+            }
+        }
+    } else if (warp == 3) {
+        // ------------------------------------------------ shared-expert gate logits
+        if (MODE == MODE_ROUTER && p.gate_w) {
+            for (int t = blockIdx.x; t < p.T; t += gridDim.x) {
+                const uint16_t *xr = p.b_src + (size_t)t * p.ldb;
+                float acc = 0.f;
+                for (int c0 = lane * 8; c0 < p.K; c0 += 256) {
+                    const uint4 v = *(const uint4 *)(xr + c0);
+                    const float4 g0 = *(const float4 *)(p.gate_w + c0);
+                    const float4 g1 = *(const float4 *)(p.gate_w + c0 + 4);
+                    acc = fmaf(__uint_as_float(v.x << 16), g0.x, acc);
+                    acc = fmaf(__uint_as_float(v.x & 0xFFFF0000u), g0.y, acc);
+                    acc = fmaf(__uint_as_float(v.y << 16), g0.z, acc);
+                    acc = fmaf(__uint_as_float(v.y & 0xFFFF0000u), g0.w, acc);
+                    acc = fmaf(__uint_as_float(v.z << 16), g1.x, acc);
+                    acc = fmaf(__uint_as_float(v.z & 0xFFFF0000u), g1.y, acc);
+                    acc = fmaf(__uint_as_float(v.w << 16), g1.z, acc);
+                    acc = fmaf(__uint_as_float(v.w & 0xFFFF0000u), g1.w, acc);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+                    acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+                if (lane == 0)
+                    p.gate_out[t] = acc;
             }
         }
     } else if (warp >= 4 && warp < 12) {
@@ -310,100 +421,171 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_q4_kernel(const Gemm
         const int c = (warp - 4) >> 2;            // which 32-element half of the k-step
         const int r = (warp & 3) * 32 + lane;     // tile row == TMEM lane
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const int cbytes = code_block_bytes(NMAT);
         int step = 0, munit = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++munit) {
             const int mb = munit & 1;
-            if (!mbar_wait(&bars->meta_full[mb], (munit >> 1) & 1, wc, 8))
-                break;
-            const uint8_t *meta = sMeta + mb * ((meta_bytes + 127) & ~127);
-            const int ngroups = WFMT == MOE_WFMT_Q4K ? p.K / 256 : p.K / p.G;
-            for (int ks = 0; ks < KS; ++ks, ++step) {
-                const int sc = step % L::kCodeStages;
-                if (!mbar_wait(&bars->code_full[sc], (step / L::kCodeStages) & 1, wc, 9)) {
-                    ok = false;
-                    break;
-                }
-                const int kpos = ks * kKStep + c * 32;
-                uint32_t words[NMAT][16];
+            const uint8_t *meta = sMeta + mb * meta_al;
+            float4 pre[8];                        // router: this row's next k-step, prefetched
+            const float *wrow = nullptr;
+            if (MODE == MODE_ROUTER) {
+                const Unit un = decode_unit(u, p, sched);
+                const int e = un.f * kTileRows + r;
+                wrow = e < p.E ? p.a_f32 + (size_t)e * p.K + c * 32 : nullptr;
 #pragma unroll
-                for (int m = 0; m < NMAT; ++m) {
-                    const uint4 codes =
-                        *(const uint4 *)(sCode + sc * cbytes + ((m * 2 + c) * kTileRows + r) * kChunkBytes);
-                    if (WFMT == MOE_WFMT_Q4K) {
-                        const int g = kpos / 256;
-                        const uint4 hdr = *(const uint4 *)(meta + ((m * ngroups + g) * kTileRows + r) * 16);
-                        float dsc, dm;
-                        q4k_subblock_scale(hdr, (kpos % 256) / 32, dsc, dm);
-                        dequant_q4k_chunk(codes, dsc, dm, words[m]);
-                    } else {
-                        const int g = kpos / p.G;
-                        const uint16_t sbits = *(const uint16_t *)(meta + ((m * ngroups + g) * kTileRows + r) * 2);
-                        dequant_int4sym_chunk(codes, sbits, words[m]);
+                for (int i = 0; i < 8; ++i)
+                    pre[i] = wrow ? *(const float4 *)(wrow + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            } else if (!mbar_wait(&bars->meta_full[mb], (munit >> 1) & 1, wc, 8)) {
+                break;
+            }
+            const int ngroups = WFMT == MOE_WFMT_Q4K ? p.K / 256 : p.K / max(p.G, 1);
+            for (int ks = 0; ks < KS; ++ks, ++step) {
+                uint32_t words[L::kNA][16];
+                if (MODE == MODE_ROUTER) {
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        v[4 * i] = pre[i].x;
+                        v[4 * i + 1] = pre[i].y;
+                        v[4 * i + 2] = pre[i].z;
+                        v[4 * i + 3] = pre[i].w;
                     }
+                    if (wrow && ks + 1 < KS) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            pre[i] = *(const float4 *)(wrow + (ks + 1) * kKStep + 4 * i);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        split3(v[2 * j], v[2 * j + 1], words[0][j], words[1 % L::kNA][j], words[2 % L::kNA][j]);
+                } else {
+                    const int sc = step % L::kCodeStages;
+                    if (!mbar_wait(&bars->code_full[sc], (step / L::kCodeStages) & 1, wc, 9)) {
+                        ok = false;
+                        break;
+                    }
+#ifdef MOEQ4_TRACE_WARPS
+                    if (lane == 0)
+                        TRACE_EVENT((warp - 4) * 2, step);
+#else
+                    if (lane == 0 && warp == 4)
+                        TRACE_EVENT(2, step);
+#endif
+                    const int kpos = ks * kKStep + c * 32;
+                    const int cbytes = code_block_bytes(L::kNCode);
+#pragma unroll
+                    for (int m = 0; m < L::kNA; ++m) {
+                        const uint4 codes =
+                            lds128(smem_u32(sCode) + sc * cbytes + ((m * 2 + c) * kTileRows + r) * kChunkBytes);
+                        if (WFMT == MOE_WFMT_Q4K) {
+                            const int g = kpos / 256;
+                            const uint4 hdr = lds128(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 16);
+                            float dsc, dm;
+                            q4k_subblock_scale(hdr, (kpos % 256) / 32, dsc, dm);
+                            dequant_q4k_chunk(codes, dsc, dm, words[m]);
+                        } else {
+                            const int g = kpos / p.G;
+                            const uint16_t sbits = lds16(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 2);
+                            dequant_int4sym_chunk(codes, sbits, words[m]);
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&bars->code_empty[sc]);
                 }
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&bars->code_empty[sc]);
                 const int sa = step % kStages;
+#ifdef MOEQ4_TRACE_WARPS
+                if (lane == 0)
+                    TRACE_EVENT((warp - 4) * 2 + 1, step);
+#else
+                if (lane == 0 && warp == 4)
+                    TRACE_EVENT(11, step);
+#endif
                 if (step >= kStages && !mbar_wait(&bars->mma_done[sa], ((step / kStages) & 1) ^ 1, wc, 10)) {
                     ok = false;
                     break;
                 }
+                if (lane == 0 && warp == 4)
+                    TRACE_OTHER(12, step);
                 tc_fence_after();
 #pragma unroll
-                for (int m = 0; m < NMAT; ++m)
-                    tmem_st16(tmem + lane_off + L::kAccCols + (sa * NMAT + m) * 32 + c * 16, words[m]);
+                for (int m = 0; m < L::kNA; ++m)
+                    tmem_st16(tmem + lane_off + L::kAccCols + (sa * L::kNA + m) * 32 + c * 16, words[m]);
                 tmem_wait_st();
+                if (lane == 0 && warp == 4)
+                    TRACE_OTHER(13, step);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&bars->a_full[sa]);
+                if (lane == 0 && warp == 4)
+                    TRACE_OTHER(3, step);
+                if (lane == 0 && warp == 11)
+                    TRACE_OTHER(4, step);
             }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&bars->meta_empty[mb]);
+            if (MODE != MODE_ROUTER) {
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bars->meta_empty[mb]);
+            }
         }
-    } else if (warp >= 12) {
-        // ------------------------------------------------ epilogue
+    } else {
+        // ------------------------------------------------ epilogue (warps 12-15)
         const int r = (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         int uidx = 0;
         for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++uidx) {
             const Unit un = decode_unit(u, p, sched);
-            if (!mbar_wait(&bars->acc_full, uidx & 1, wc, 11))
+            const int ab = uidx % L::kAccBufs;
+            if (!mbar_wait(&bars->acc_full[ab], (uidx / L::kAccBufs) & 1, wc, 11))
                 break;
             tc_fence_after();
+            if (lane == 0 && warp == 12)
+                TRACE_OTHER(6, uidx);
+            const uint32_t acc = tmem + lane_off + ab * L::kNAcc * kBN;
             const int col = un.f * kTileRows + r;
             for (int n0 = 0; n0 < un.nmma; n0 += 16) {
                 uint32_t g[16], v[16];
-                tmem_ld16(tmem + lane_off + n0, g);
-                if (NMAT == 2)
-                    tmem_ld16(tmem + lane_off + kBN + n0, v);
+                tmem_ld16(acc + n0, g);
+                if (L::kNAcc == 2)
+                    tmem_ld16(acc + kBN + n0, v);
                 tmem_wait_ld();
+                if (MODE == MODE_ROUTER) {
+                    if (col < p.E) {
+                        const float b = p.bias ? p.bias[col] : 0.f;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int n = n0 + j;
-                    if (n < un.nvalid) {
-                        const int prow = un.row0 + n;
-                        float o;
-                        if (NMAT == 2) {
-                            const float a = __uint_as_float(g[j]);
-                            o = a / (1.0f + __expf(-a)) * __uint_as_float(v[j]);
-                        } else {
-                            o = __uint_as_float(g[j]);
+                        for (int j = 0; j < 16; ++j) {
+                            const int n = n0 + j;
+                            if (n < un.nvalid)
+                                p.out_f32[(size_t)(un.row0 + n) * p.E + col] = __uint_as_float(g[j]) + b;
                         }
-                        uint16_t *dst = prow < p.Tk ? p.out + (size_t)prow * p.ldo
-                                                    : p.out_shared + (size_t)(prow - p.Tk) * p.ldo;
-                        dst[col] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int n = n0 + j;
+                        if (n < un.nvalid) {
+                            const int prow = un.row0 + n;
+                            float o;
+                            if (MODE == MODE_GATE_UP) {
+                                const float a = __uint_as_float(g[j]);
+                                o = a / (1.0f + __expf(-a)) * __uint_as_float(v[j]);
+                            } else {
+                                o = __uint_as_float(g[j]);
+                            }
+                            uint16_t *dst = prow < p.Tk ? p.out + (size_t)prow * p.ldo
+                                                        : p.out_shared + (size_t)(prow - p.Tk) * p.ldo;
+                            dst[col] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+                        }
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&bars->acc_empty);
+                mbar_arrive(&bars->acc_empty[ab]);
+            if (lane == 0 && warp == 12)
+                TRACE_OTHER(7, uidx);
         }
     }
 
@@ -414,19 +596,22 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_q4_kernel(const Gemm
     }
 }
 
-template <int NMAT>
+template <int MODE>
 static size_t gemm_smem_bytes(int meta_bytes, int E_total)
 {
-    using L = GemmSmem<NMAT>;
-    return 1024 + L::kBBytes + L::kCodeBytes + 2 * ((meta_bytes + 127) & ~127) + sizeof(Barriers) +
-           sizeof(int) * (3 * E_total + 1 + kThreads) + 16;
+    using L = Geo<MODE>;
+    const size_t need = 1024 + L::kBBytes + L::kCodeBytes + 2 * ((meta_bytes + 127) & ~127) + sizeof(Barriers) +
+                        sizeof(int) * (3 * E_total + 1 + kThreads) + 16;
+    // at least half of the SM's shared memory, so that one CTA (and one TMEM
+    // allocation) runs per SM
+    return need > 116 * 1024 ? need : 116 * 1024;
 }
 
-template <int NMAT, int WFMT, bool GATHER>
+template <int MODE, int WFMT>
 static cudaError_t launch_one(const GemmArgs &a, int num_sms, cudaStream_t st)
 {
-    auto kern = grouped_gemm_q4_kernel<NMAT, WFMT, GATHER>;
-    const size_t smem = gemm_smem_bytes<NMAT>(a.meta_bytes, a.E_total);
+    auto kern = grouped_gemm_kernel<MODE, WFMT>;
+    const size_t smem = gemm_smem_bytes<MODE>(a.meta_bytes, a.E_total);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
@@ -436,17 +621,55 @@ static cudaError_t launch_one(const GemmArgs &a, int num_sms, cudaStream_t st)
 
 size_t gemm_smem_required(int nmat, int meta_bytes, int E_total)
 {
-    return nmat == 2 ? gemm_smem_bytes<2>(meta_bytes, E_total) : gemm_smem_bytes<1>(meta_bytes, E_total);
+    return nmat == 2 ? gemm_smem_bytes<MODE_GATE_UP>(meta_bytes, E_total)
+                     : gemm_smem_bytes<MODE_DOWN>(meta_bytes, E_total);
 }
 
 cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int num_sms, cudaStream_t st)
 {
     if (nmat == 2) {
-        return wfmt == MOE_WFMT_Q4K ? launch_one<2, MOE_WFMT_Q4K, true>(a, num_sms, st)
-                                    : launch_one<2, MOE_WFMT_INT4_SYM, true>(a, num_sms, st);
+        return wfmt == MOE_WFMT_Q4K ? launch_one<MODE_GATE_UP, MOE_WFMT_Q4K>(a, num_sms, st)
+                                    : launch_one<MODE_GATE_UP, MOE_WFMT_INT4_SYM>(a, num_sms, st);
     }
-    return wfmt == MOE_WFMT_Q4K ? launch_one<1, MOE_WFMT_Q4K, false>(a, num_sms, st)
-                                : launch_one<1, MOE_WFMT_INT4_SYM, false>(a, num_sms, st);
+    return wfmt == MOE_WFMT_Q4K ? launch_one<MODE_DOWN, MOE_WFMT_Q4K>(a, num_sms, st)
+                                : launch_one<MODE_DOWN, MOE_WFMT_INT4_SYM>(a, num_sms, st);
+}
+
+// Router logits on tensor cores: logits[t, e] = x[t] . Wr[e] (+ bias[e]),
+// and gate_out[t] = x[t] . g when g is given.
+cudaError_t launch_router_gemm(const uint16_t *x, int T, int H, const float *wr, const float *bias, int E,
+                               const float *gate_w, float *logits, float *gate_out, int *status, int num_sms,
+                               cudaStream_t st)
+{
+    if (T == 0)
+        return cudaSuccess;
+    GemmArgs a{};
+    a.b_src = x;
+    a.ldb = H;
+    a.T = T;
+    a.E = E;
+    a.E_total = 1;
+    a.K = H;
+    a.F = (E + kTileRows - 1) / kTileRows;
+    a.a_f32 = wr;
+    a.bias = bias;
+    a.gate_w = gate_w;
+    a.gate_out = gate_out;
+    a.out_f32 = logits;
+    a.status = status;
+    return launch_one<MODE_ROUTER, 0>(a, num_sms, st);
 }
 
 }  // namespace moeq4
+
+#ifdef MOEQ4_TRACE
+extern "C" int moe_trace_fetch(unsigned long long *host)
+{
+    return (int)cudaMemcpyFromSymbol(host, moeq4::g_trace, sizeof(moeq4::g_trace));
+}
+extern "C" int moe_trace_clear()
+{
+    static unsigned long long zero[4 * 16 * moeq4::kTraceSteps];
+    return (int)cudaMemcpyToSymbol(moeq4::g_trace, zero, sizeof(zero));
+}
+#endif

@@ -25,6 +25,11 @@ struct GemmArgs {
     int F;                      // 128-row tiles per expert matrix
     int G;                      // int4-sym group size
     int meta_bytes;             // per (expert, tile) meta block
+    const float *a_f32;         // router pass: fp32 A rows [E, K]
+    const float *bias;          // router pass: bias [E] or null
+    const float *gate_w;        // router pass: shared-expert gate vector [K] or null
+    float *gate_out;            // router pass: gate logits [T]
+    float *out_f32;             // router pass: logits [T, E]
     uint16_t *out;              // routed rows: out + p * ldo
     uint16_t *out_shared;       // shared rows: out_shared + (p - Tk) * ldo
     int ldo;
@@ -34,8 +39,9 @@ struct GemmArgs {
 cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int num_sms, cudaStream_t st);
 size_t gemm_smem_required(int nmat, int meta_bytes, int E_total);
 
-cudaError_t launch_router_logits(const uint16_t *x, int T, int H, const float *wr, const float *bias, int E,
-                                 const float *gate_w, float *logits, float *gate_logit, cudaStream_t st);
+cudaError_t launch_router_gemm(const uint16_t *x, int T, int H, const float *wr, const float *bias, int E,
+                               const float *gate_w, float *logits, float *gate_out, int *status, int num_sms,
+                               cudaStream_t st);
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
                          cudaStream_t st);
 

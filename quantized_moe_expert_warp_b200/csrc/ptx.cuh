@@ -22,6 +22,28 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+__device__ __forceinline__ uint4 lds128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint16_t lds16(uint32_t addr)
+{
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ int lds_volatile_s32(uint32_t addr)
+{
+    int v;
+    asm volatile("ld.volatile.shared.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
@@ -80,7 +102,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, WaitCt
     while (true) {
         if (mbar_try_wait(bar, parity))
             return true;
-        if (*w.abort_flag)
+        if (lds_volatile_s32(smem_u32((const void *)w.abort_flag)))
             return false;
         if ((++spins & 63u) == 0) {
             if (globaltimer_ns() - w.t0 > kWaitLimitNs) {
@@ -93,6 +115,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, WaitCt
     }
 }
 
+// One lane of a converged warp waits; the whole warp gets the result.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, WaitCtx &w, int where)
+{
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0)
+        ok = mbar_wait(bar, parity, w, where) ? 1 : 0;
+    return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
+
+// True on exactly one lane of a converged warp.  Single-thread tcgen05 and
+// bulk-copy instructions are issued under this predicate from a converged
+// warp: issuing them from a lone divergent lane costs several times longer.
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .b32 %%rx;\n\t.reg .pred %%px;\n\t"
+        "elect.sync %%rx|%%px, %1;\n\t"
+        "@%%px mov.s32 %0, 1;\n\t}"
+        : "+r"(pred)
+        : "r"(0xFFFFFFFFu));
+    return pred != 0;
+}
+
 // ------------------------------------------------------------------ copies
 
 // 16-byte cp.async; src_bytes = 0 writes zeros (the source is not read).
@@ -100,6 +146,13 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint3
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
                  : "memory");
+}
+
+// Arrive on `bar` once all cp.async operations issued so far by this thread
+// have completed (the arrival counts against the barrier's initial count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
