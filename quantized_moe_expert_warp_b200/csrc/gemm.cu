@@ -14,18 +14,20 @@
 // epilogue warps apply SwiGLU (gate/up pass), round to bf16 (down pass) or
 // add the router bias (router pass).
 //
-// The router pass uses the same engine: its fp32 weights are split into
-// three bf16 parts (hi + mid + lo carry all 24 significand bits), the three
-// products are exact in fp32 and accumulate into one fp32 accumulator.
+// The router pass uses the same engine: its fp32 weights are split into two
+// bf16 parts (hi + lo carry 16 significand bits, the rest is below the fp32
+// accumulation error of the tensor cores over K = 2048), both products are
+// exact in fp32 and accumulate into one fp32 accumulator.
 //
-// Warp roles of one persistent CTA (one per SM, 512 threads):
+// Warp roles of one persistent CTA (one per SM, 768 threads):
 //   warp 0      gathers token rows of B with cp.async (zero rows past the tail)
 //   warp 1      issues tcgen05.mma (one thread) and commits stage releases
 //   warp 2      streams code blocks and per-tile scale blocks with bulk copies
 //   warp 3      owns the TMEM allocation; in the router pass it also forms
 //               the shared expert's gate logits x . g
-//   warps 4-11  dequantise: row r = 32*(warp%4) + lane, half c = (warp-4)/4
-//   warps 12-15 epilogue (TMEM -> registers -> global)
+//   warps 4-19  dequantise, in two groups of eight taking alternate k-steps:
+//               row r = 32*(warp%4) + lane, half c of the k-step = ((warp-4)%8)/4
+//   warps 20-23 epilogue (TMEM -> registers -> global)
 // Every wait is bounded; on timeout the CTA records MOE_ERR_TIMEOUT and
 // unwinds.
 #include <cstdint>
@@ -60,30 +62,37 @@ __device__ unsigned long long g_trace[4][16][kTraceSteps];
     } while (0)
 #endif
 
-constexpr int kBN = 128;     // max tokens per tile (the MMA's N)
+constexpr int kBNMax = 128;  // max tokens per tile (the MMA's N); tiles of 64 when groups are small
 constexpr int kStages = 4;   // B / TMEM-A pipeline depth
-constexpr int kThreads = 512;
+constexpr int kEpiTok = 16;  // tokens per epilogue chunk
+constexpr int kEpiStride = 80;                                   // bytes per staged token row (64 + pad)
+constexpr int kEpiBytes = 4 * kEpiTok * kEpiStride;              // staging for the four epilogue warps
+constexpr int kDeqGroups = 2;                  // dequant warp groups, alternating k-steps
+constexpr int kThreads = (8 + 8 * kDeqGroups) * 32;
 
 enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_ROUTER = 2 };
 
-template <int MODE>
+template <int MODE, int BN>
 struct Geo {
-    static constexpr int kNA = MODE == MODE_GATE_UP ? 2 : MODE == MODE_DOWN ? 1 : 3;   // A operands per k-step
+    static constexpr int kBN = BN;
+    static constexpr int kNA = MODE == MODE_DOWN ? 1 : 2;                               // A operands per k-step
     static constexpr int kNAcc = MODE == MODE_GATE_UP ? 2 : 1;                          // accumulators per unit
-    static constexpr int kAccBufs = MODE == MODE_DOWN ? 2 : 1;                          // accumulator buffers
+    static constexpr int kNAcc_ = MODE == MODE_GATE_UP ? 2 : 1;
+    // as many accumulator buffers (up to 2) as TMEM holds next to the A stages:
+    // with two, the epilogue of one tile overlaps the MMAs of the next
+    static constexpr int kAccBufs = (512 - kStages * kNA * 32) / (kNAcc_ * BN) >= 2 ? 2 : 1;
     static constexpr int kNCode = MODE == MODE_GATE_UP ? 2 : MODE == MODE_DOWN ? 1 : 0; // code matrices
     static constexpr int kCodeStages = MODE == MODE_GATE_UP ? 8 : MODE == MODE_DOWN ? 16 : 1;
     static constexpr int kCodeBytes = kCodeStages * (kNCode ? code_block_bytes(kNCode) : 0);
-    static constexpr int kBBytes = kStages * kBN * 128;
-    static constexpr int kAccCols = kAccBufs * kNAcc * kBN;
+    static constexpr int kBBytes = kStages * BN * 128;
+    static constexpr int kAccCols = kAccBufs * kNAcc * BN;
     static constexpr int kTmemCols = 512;
     static_assert(kAccCols + kStages * kNA * 32 <= kTmemCols, "TMEM budget");
     static constexpr bool kGather = MODE == MODE_GATE_UP;
 };
 
 struct Barriers {
-    uint64_t b_full[kStages];
-    uint64_t a_full[kStages];
+    uint64_t full[kStages];       // A dequantised into TMEM and B gathered into shared memory
     uint64_t mma_done[kStages];
     uint64_t code_full[16];
     uint64_t code_empty[16];
@@ -107,6 +116,7 @@ struct Sched {
     const int *row_count;    // [E_total] rows
 };
 
+template <int BN>
 __device__ __forceinline__ Unit decode_unit(int u, const GemmArgs &p, const Sched &sc)
 {
     Unit r;
@@ -122,16 +132,17 @@ __device__ __forceinline__ Unit decode_unit(int u, const GemmArgs &p, const Sche
     }
     r.e = lo;
     const int c = tile - sc.tile_start[lo];
-    r.row0 = sc.row_start[lo] + c * kBN;
-    r.nvalid = min(kBN, sc.row_count[lo] - c * kBN);
+    r.row0 = sc.row_start[lo] + c * BN;
+    r.nvalid = min(BN, sc.row_count[lo] - c * BN);
     r.nmma = max(16, (r.nvalid + 15) & ~15);
     return r;
 }
 
 // Every CTA derives the tile schedule from the permutation offsets: rows of
 // expert e are [offsets[e], offsets[e+1]); the shared expert (if any) is
-// expert E with rows [T k, T k + T); expert e owns ceil(rows / kBN) tiles.
+// expert E with rows [T k, T k + T); expert e owns ceil(rows / BN) tiles.
 // Without offsets (router pass) the T token rows form a single group.
+template <int BN>
 __device__ void build_schedule(const GemmArgs &p, int *s_tile_start, int *s_row_start, int *s_row_count,
                                int *s_part)
 {
@@ -153,7 +164,7 @@ __device__ void build_schedule(const GemmArgs &p, int *s_tile_start, int *s_row_
         }
         s_row_start[e] = start;
         s_row_count[e] = cnt;
-        local += (cnt + kBN - 1) / kBN;
+        local += (cnt + BN - 1) / BN;
     }
     s_part[threadIdx.x] = local;
     __syncthreads();
@@ -166,29 +177,27 @@ __device__ void build_schedule(const GemmArgs &p, int *s_tile_start, int *s_row_
     int run = s_part[threadIdx.x] - local;
     for (int e = e0; e < min(n, e0 + per); ++e) {
         s_tile_start[e] = run;
-        run += (s_row_count[e] + kBN - 1) / kBN;
+        run += (s_row_count[e] + BN - 1) / BN;
     }
     if (threadIdx.x == kThreads - 1)
         s_tile_start[n] = s_part[kThreads - 1];
 }
 
-// fp32 -> three bf16 parts (hi, mid, lo): w - hi and (w - hi) - mid are exact
-// in fp32, so hi + mid + lo matches w to about 2^-24 relative.
-__device__ __forceinline__ void split3(float w0, float w1, uint32_t &hi, uint32_t &mid, uint32_t &lo)
+// fp32 -> two bf16 parts (hi, lo): w - hi is exact in fp32, so hi + lo
+// matches w to about 2^-17 relative.
+__device__ __forceinline__ void split2(float w0, float w1, uint32_t &hi, uint32_t &lo)
 {
     hi = pack_bf16x2(w0, w1);
     const float r0 = w0 - __uint_as_float(hi << 16);
     const float r1 = w1 - __uint_as_float(hi & 0xFFFF0000u);
-    mid = pack_bf16x2(r0, r1);
-    const float s0 = r0 - __uint_as_float(mid << 16);
-    const float s1 = r1 - __uint_as_float(mid & 0xFFFF0000u);
-    lo = pack_bf16x2(s0, s1);
+    lo = pack_bf16x2(r0, r1);
 }
 
-template <int MODE, int WFMT>
+template <int MODE, int WFMT, int BN>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArgs p)
 {
-    using L = Geo<MODE>;
+    using L = Geo<MODE, BN>;
+    constexpr int kBN = BN;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled B stages
     // offset arithmetic on the shared array keeps the pointer in the shared
@@ -204,6 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
     int *s_row_start = s_tile_start + p.E_total + 1;
     int *s_row_count = s_row_start + p.E_total;
     int *s_part = s_row_count + p.E_total;
+    uint8_t *s_epi = (uint8_t *)(s_part + kThreads);
+    s_epi += (16u - (smem_u32(s_epi) & 15u)) & 15u;    // epilogue staging, 16-byte aligned
     const Sched sched{s_tile_start, s_row_start, s_row_count};
 
     const int warp = threadIdx.x / 32;
@@ -211,8 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&bars->b_full[s], 32);   // one cp.async completion arrival per lane
-            mbar_init(&bars->a_full[s], 8);
+            // eight dequant warps + one cp.async completion arrival per lane of the B producer
+            mbar_init(&bars->full[s], 8 + 32);
             mbar_init(&bars->mma_done[s], 1);
         }
         for (int s = 0; s < L::kCodeStages; ++s) {
@@ -221,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->meta_full[s], 1);
-            mbar_init(&bars->meta_empty[s], 8);
+            mbar_init(&bars->meta_empty[s], 8 * kDeqGroups);
             mbar_init(&bars->acc_full[s], 1);
             mbar_init(&bars->acc_empty[s], 4);
         }
@@ -230,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
         bars->never_abort = 0;
         fence_mbar_init();
     }
-    build_schedule(p, s_tile_start, s_row_start, s_row_count, s_part);
+    build_schedule<BN>(p, s_tile_start, s_row_start, s_row_count, s_part);
     if (warp == 3) {
         tmem_alloc(&bars->tmem_base, L::kTmemCols);
         tmem_relinquish();
@@ -249,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
         int step = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
-            const Unit un = decode_unit(u, p, sched);
+            const Unit un = decode_unit<BN>(u, p, sched);
             const uint16_t *src[kBN / 32];
             uint32_t bytes[kBN / 32];
 #pragma unroll
@@ -280,8 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                             cp_async_16(rbase + ((j ^ (r & 7)) << 4), g + j * 8, bytes[i]);
                     }
                 }
-                // this lane's copies for the stage arrive on b_full[s] when they land
-                cp_async_arrive_noinc(&bars->b_full[s]);
+                // this lane's copies for the stage arrive on full[s] when they land
+                cp_async_arrive_noinc(&bars->full[s]);
                 if (lane == 0)
                     TRACE_OTHER(0, step);
             }
@@ -291,25 +302,20 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
         int step = 0, uidx = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++uidx) {
-            const Unit un = decode_unit(u, p, sched);
+            const Unit un = decode_unit<BN>(u, p, sched);
             const uint32_t idesc = idesc_bf16_f32(128, un.nmma);
             const int ab = uidx % L::kAccBufs;
             const uint32_t acc = tmem + ab * L::kNAcc * kBN;
             if (uidx >= L::kAccBufs) {
-                if (!warp_wait(&bars->acc_empty[ab], ((uidx / L::kAccBufs) & 1) ^ 1, wc, 2))
+                if (!mbar_wait(&bars->acc_empty[ab], ((uidx / L::kAccBufs) & 1) ^ 1, wc, 2))
                     break;
                 tc_fence_after();
             }
             for (int ks = 0; ks < KS; ++ks, ++step) {
                 const int s = step % kStages;
                 const uint32_t ph = (step / kStages) & 1;
-                if (!warp_wait(&bars->a_full[s], ph, wc, 3)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0)
-                    TRACE_OTHER(8, step);
-                if (!warp_wait(&bars->b_full[s], ph, wc, 4)) {
+                // every lane polls the same barrier, so the outcome is warp-uniform
+                if (!mbar_wait(&bars->full[s], ph, wc, 3)) {
                     ok = false;
                     break;
                 }
@@ -319,26 +325,23 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                 // reads it through the async proxy
                 fence_proxy_async_smem();
                 tc_fence_after();
-                const uint32_t bbase = smem_u32(sB + s * kBN * 128);
+                const uint64_t bdesc0 = sdesc_kmajor_sw128(smem_u32(sB + s * kBN * 128));
+                const uint32_t a_base = tmem + L::kAccCols + s * L::kNA * 32;
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bdesc = sdesc_kmajor_sw128(bbase + kk * 32);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t bdesc = bdesc0 + (uint64_t)(kk * 2);   // +32 bytes along K
 #pragma unroll
-                    for (int m = 0; m < L::kNA; ++m) {
-                        const uint32_t a_t = tmem + L::kAccCols + (s * L::kNA + m) * 32 + kk * 8;
-                        if (elect_one()) {
-                            if (MODE == MODE_ROUTER)   // three parts into one accumulator
+                        for (int m = 0; m < L::kNA; ++m) {
+                            const uint32_t a_t = a_base + m * 32 + kk * 8;
+                            if (MODE == MODE_ROUTER)   // both parts into one accumulator
                                 mma_ts_f16(acc, a_t, bdesc, idesc, (ks | kk | m) != 0);
                             else
                                 mma_ts_f16(acc + m * kBN, a_t, bdesc, idesc, (ks | kk) != 0);
                         }
-                        __syncwarp();
                     }
-                }
-                if (lane == 0)
-                    TRACE_OTHER(10, step);
-                if (elect_one())
                     mma_commit(&bars->mma_done[s]);
+                }
                 __syncwarp();
                 if (lane == 0)
                     TRACE_OTHER(5, step);
@@ -362,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
             const int cbytes = code_block_bytes(L::kNCode);
             bool ok = true;
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++munit) {
-                const Unit un = decode_unit(u, p, sched);
+                const Unit un = decode_unit<BN>(u, p, sched);
                 const size_t tile_id = (size_t)un.e * p.F + un.f;
                 const int mb = munit & 1;
                 if (munit >= 2 && !warp_wait(&bars->meta_empty[mb], ((munit >> 1) & 1) ^ 1, wc, 6))
@@ -416,9 +419,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                     p.gate_out[t] = acc;
             }
         }
-    } else if (warp >= 4 && warp < 12) {
+    } else if (warp >= 4 && warp < 4 + 8 * kDeqGroups) {
         // ------------------------------------------------ dequant into TMEM
-        const int c = (warp - 4) >> 2;            // which 32-element half of the k-step
+        const int dw = warp - 4;
+        const int grp = dw / 8;                   // this group handles k-steps with step % kDeqGroups == grp
+        const int c = (dw & 7) >> 2;              // which 32-element half of the k-step
         const int r = (warp & 3) * 32 + lane;     // tile row == TMEM lane
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         int step = 0, munit = 0;
@@ -429,17 +434,22 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
             float4 pre[8];                        // router: this row's next k-step, prefetched
             const float *wrow = nullptr;
             if (MODE == MODE_ROUTER) {
-                const Unit un = decode_unit(u, p, sched);
+                const Unit un = decode_unit<BN>(u, p, sched);
                 const int e = un.f * kTileRows + r;
                 wrow = e < p.E ? p.a_f32 + (size_t)e * p.K + c * 32 : nullptr;
+                const int ks0 = ((grp - step) % kDeqGroups + kDeqGroups) % kDeqGroups;   // first k-step of this group
+                if (ks0 >= KS)
+                    wrow = nullptr;
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    pre[i] = wrow ? *(const float4 *)(wrow + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    pre[i] = wrow ? *(const float4 *)(wrow + ks0 * kKStep + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
             } else if (!mbar_wait(&bars->meta_full[mb], (munit >> 1) & 1, wc, 8)) {
                 break;
             }
             const int ngroups = WFMT == MOE_WFMT_Q4K ? p.K / 256 : p.K / max(p.G, 1);
             for (int ks = 0; ks < KS; ++ks, ++step) {
+                if (step % kDeqGroups != grp)
+                    continue;
                 uint32_t words[L::kNA][16];
                 if (MODE == MODE_ROUTER) {
                     float v[32];
@@ -450,14 +460,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                         v[4 * i + 2] = pre[i].z;
                         v[4 * i + 3] = pre[i].w;
                     }
-                    if (wrow && ks + 1 < KS) {
+                    if (wrow && ks + kDeqGroups < KS) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
-                            pre[i] = *(const float4 *)(wrow + (ks + 1) * kKStep + 4 * i);
+                            pre[i] = *(const float4 *)(wrow + (ks + kDeqGroups) * kKStep + 4 * i);
                     }
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        split3(v[2 * j], v[2 * j + 1], words[0][j], words[1 % L::kNA][j], words[2 % L::kNA][j]);
+                        split2(v[2 * j], v[2 * j + 1], words[0][j], words[1 % L::kNA][j]);
                 } else {
                     const int sc = step % L::kCodeStages;
                     if (!mbar_wait(&bars->code_full[sc], (step / L::kCodeStages) & 1, wc, 9)) {
@@ -517,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
-                    mbar_arrive(&bars->a_full[sa]);
+                    mbar_arrive(&bars->full[sa]);
                 if (lane == 0 && warp == 4)
                     TRACE_OTHER(3, step);
                 if (lane == 0 && warp == 11)
@@ -530,26 +540,37 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
             }
         }
     } else {
-        // ------------------------------------------------ epilogue (warps 12-15)
+        // ------------------------------------------------ epilogue (last four warps)
         const int r = (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         int uidx = 0;
         for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++uidx) {
-            const Unit un = decode_unit(u, p, sched);
+            const Unit un = decode_unit<BN>(u, p, sched);
             const int ab = uidx % L::kAccBufs;
             if (!mbar_wait(&bars->acc_full[ab], (uidx / L::kAccBufs) & 1, wc, 11))
                 break;
             tc_fence_after();
-            if (lane == 0 && warp == 12)
+            if (lane == 0 && warp == 4 + 8 * kDeqGroups)
                 TRACE_OTHER(6, uidx);
             const uint32_t acc = tmem + lane_off + ab * L::kNAcc * kBN;
             const int col = un.f * kTileRows + r;
-            for (int n0 = 0; n0 < un.nmma; n0 += 16) {
+            const int q = warp & 3;
+            uint8_t *stage = s_epi + q * kEpiTok * kEpiStride;
+            bool released = false;
+            for (int n0 = 0; n0 < un.nmma; n0 += kEpiTok) {
                 uint32_t g[16], v[16];
                 tmem_ld16(acc + n0, g);
                 if (L::kNAcc == 2)
                     tmem_ld16(acc + kBN + n0, v);
                 tmem_wait_ld();
+                if (n0 + kEpiTok >= un.nmma) {
+                    // every column is in registers: hand the accumulator back to the MMA
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&bars->acc_empty[ab]);
+                    released = true;
+                }
                 if (MODE == MODE_ROUTER) {
                     if (col < p.E) {
                         const float b = p.bias ? p.bias[col] : 0.f;
@@ -561,30 +582,41 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                         }
                     }
                 } else {
+                    // this lane's feature for 16 tokens -> staging [token][feature] (bf16)
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        const int n = n0 + j;
-                        if (n < un.nvalid) {
-                            const int prow = un.row0 + n;
-                            float o;
-                            if (MODE == MODE_GATE_UP) {
-                                const float a = __uint_as_float(g[j]);
-                                o = a / (1.0f + __expf(-a)) * __uint_as_float(v[j]);
-                            } else {
-                                o = __uint_as_float(g[j]);
-                            }
-                            uint16_t *dst = prow < p.Tk ? p.out + (size_t)prow * p.ldo
-                                                        : p.out_shared + (size_t)(prow - p.Tk) * p.ldo;
-                            dst[col] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+                        float o;
+                        if (MODE == MODE_GATE_UP) {
+                            const float a = __uint_as_float(g[j]);
+                            o = __fdividef(a, 1.0f + __expf(-a)) * __uint_as_float(v[j]);   // silu(a) * u
+                        } else {
+                            o = __uint_as_float(g[j]);
                         }
+                        *(__nv_bfloat16 *)(stage + j * kEpiStride + lane * 2) = __float2bfloat16_rn(o);
                     }
+                    __syncwarp();
+                    // lane: token n0 + (lane & 15), 32-byte half (lane >> 4) of the warp's 64-byte row slice
+                    const int t = lane & 15, hh = lane >> 4;
+                    const int n = n0 + t;
+                    if (n < un.nvalid) {
+                        const int prow = un.row0 + n;
+                        uint16_t *dst = prow < p.Tk ? p.out + (size_t)prow * p.ldo
+                                                    : p.out_shared + (size_t)(prow - p.Tk) * p.ldo;
+                        uint4 *d4 = (uint4 *)(dst + un.f * kTileRows + q * 32 + hh * 16);
+                        const uint4 *s4 = (const uint4 *)(stage + t * kEpiStride + hh * 32);
+                        d4[0] = s4[0];
+                        d4[1] = s4[1];
+                    }
+                    __syncwarp();
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&bars->acc_empty[ab]);
-            if (lane == 0 && warp == 12)
+            if (!released) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bars->acc_empty[ab]);
+            }
+            if (lane == 0 && warp == 4 + 8 * kDeqGroups)
                 TRACE_OTHER(7, uidx);
         }
     }
@@ -596,22 +628,22 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
     }
 }
 
-template <int MODE>
+template <int MODE, int BN>
 static size_t gemm_smem_bytes(int meta_bytes, int E_total)
 {
-    using L = Geo<MODE>;
+    using L = Geo<MODE, BN>;
     const size_t need = 1024 + L::kBBytes + L::kCodeBytes + 2 * ((meta_bytes + 127) & ~127) + sizeof(Barriers) +
-                        sizeof(int) * (3 * E_total + 1 + kThreads) + 16;
+                        sizeof(int) * (3 * E_total + 1 + kThreads) + 16 + kEpiBytes;
     // at least half of the SM's shared memory, so that one CTA (and one TMEM
     // allocation) runs per SM
     return need > 116 * 1024 ? need : 116 * 1024;
 }
 
-template <int MODE, int WFMT>
+template <int MODE, int WFMT, int BN>
 static cudaError_t launch_one(const GemmArgs &a, int num_sms, cudaStream_t st)
 {
-    auto kern = grouped_gemm_kernel<MODE, WFMT>;
-    const size_t smem = gemm_smem_bytes<MODE>(a.meta_bytes, a.E_total);
+    auto kern = grouped_gemm_kernel<MODE, WFMT, BN>;
+    const size_t smem = gemm_smem_bytes<MODE, BN>(a.meta_bytes, a.E_total);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
@@ -621,18 +653,27 @@ static cudaError_t launch_one(const GemmArgs &a, int num_sms, cudaStream_t st)
 
 size_t gemm_smem_required(int nmat, int meta_bytes, int E_total)
 {
-    return nmat == 2 ? gemm_smem_bytes<MODE_GATE_UP>(meta_bytes, E_total)
-                     : gemm_smem_bytes<MODE_DOWN>(meta_bytes, E_total);
+    // the 128-token tile is the larger of the two configurations
+    return nmat == 2 ? gemm_smem_bytes<MODE_GATE_UP, 128>(meta_bytes, E_total)
+                     : gemm_smem_bytes<MODE_DOWN, 128>(meta_bytes, E_total);
 }
 
-cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int num_sms, cudaStream_t st)
+int gemm_tile_tokens(int T, int E, int k) { return (long long)T * k <= 64LL * E ? 64 : 128; }
+
+template <int MODE, int BN>
+static cudaError_t launch_fmt(const GemmArgs &a, int wfmt, int num_sms, cudaStream_t st)
 {
-    if (nmat == 2) {
-        return wfmt == MOE_WFMT_Q4K ? launch_one<MODE_GATE_UP, MOE_WFMT_Q4K>(a, num_sms, st)
-                                    : launch_one<MODE_GATE_UP, MOE_WFMT_INT4_SYM>(a, num_sms, st);
-    }
-    return wfmt == MOE_WFMT_Q4K ? launch_one<MODE_DOWN, MOE_WFMT_Q4K>(a, num_sms, st)
-                                : launch_one<MODE_DOWN, MOE_WFMT_INT4_SYM>(a, num_sms, st);
+    return wfmt == MOE_WFMT_Q4K ? launch_one<MODE, MOE_WFMT_Q4K, BN>(a, num_sms, st)
+                                : launch_one<MODE, MOE_WFMT_INT4_SYM, BN>(a, num_sms, st);
+}
+
+cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int tile_tokens, int num_sms, cudaStream_t st)
+{
+    if (nmat == 2)
+        return tile_tokens == 64 ? launch_fmt<MODE_GATE_UP, 64>(a, wfmt, num_sms, st)
+                                 : launch_fmt<MODE_GATE_UP, 128>(a, wfmt, num_sms, st);
+    return tile_tokens == 64 ? launch_fmt<MODE_DOWN, 64>(a, wfmt, num_sms, st)
+                             : launch_fmt<MODE_DOWN, 128>(a, wfmt, num_sms, st);
 }
 
 // Router logits on tensor cores: logits[t, e] = x[t] . Wr[e] (+ bias[e]),
@@ -657,7 +698,7 @@ cudaError_t launch_router_gemm(const uint16_t *x, int T, int H, const float *wr,
     a.gate_out = gate_out;
     a.out_f32 = logits;
     a.status = status;
-    return launch_one<MODE_ROUTER, 0>(a, num_sms, st);
+    return launch_one<MODE_ROUTER, 0, 128>(a, num_sms, st);
 }
 
 }  // namespace moeq4

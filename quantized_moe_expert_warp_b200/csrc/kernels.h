@@ -36,7 +36,10 @@ struct GemmArgs {
     int *status;                // [code, detail]
 };
 
-cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int num_sms, cudaStream_t st);
+// Token-tile width of the grouped GEMMs: 64 when experts average at most 64
+// rows (T k <= 64 E), else 128.  Both passes of one FFN must use the same.
+int gemm_tile_tokens(int T, int E, int k);
+cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int tile_tokens, int num_sms, cudaStream_t st);
 size_t gemm_smem_required(int nmat, int meta_bytes, int E_total);
 
 cudaError_t launch_router_gemm(const uint16_t *x, int T, int H, const float *wr, const float *bias, int E,

@@ -176,7 +176,7 @@ def test_router_logits_close(dev):
     gl = torch.empty((cfg.T,), dtype=torch.float32, device=dev)
     mq.moe_router_logits(packed, x, cfg.T, logits, gl)
     ref = oracle.router_logits(layer["x"], layer["router_w"], layer["router_bias"])
-    # bf16 x is exact; fp32 weights enter as three bf16 parts with exact products,
+    # bf16 x is exact; fp32 weights enter as two bf16 parts (16 significand bits) with exact products,
     # summed by the tensor cores' fp32 accumulation (truncating adds over
     # H / 16 = 128 partial blocks): |err| ~ 1e-5 for |logit| up to ~8
     np.testing.assert_allclose(logits.cpu().numpy(), ref, rtol=0, atol=1e-4)
@@ -198,6 +198,8 @@ SMALL_LAYERS = [
     small_cfg("one_token", T=1, H=512, E=64, k=8, I=128, has_shared=True, G=128),
     # every expert gets > 128 rows: multi-tile experts without a shared expert
     small_cfg("big_groups", T=600, H=256, E=4, k=2, I=384, G=128, wr_std=0.02),
+    # 64-token tiles (T k <= 64 E): ragged multi-tile shared expert, some routed experts over 64 rows
+    small_cfg("small_tiles_shared", T=200, H=512, E=8, k=2, I=256, has_shared=True, G=128, wr_std=0.04),
 ]
 
 
