@@ -173,6 +173,29 @@ size_t moe_permute_workspace_size(int T, int E, int k);
 int moe_permute(const int32_t *topk_ids, int T, int E, int k, int32_t *counts, int32_t *offsets,
                 int32_t *sorted_slot, int32_t *dest_pos, void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * moe_permute without a workspace, for callers that cannot allocate device
+ * memory when they route (for instance code that runs under another
+ * allocator's lock, or a host framework that forbids cudaMalloc after
+ * start-up and hands out no scratch).  The pages have no counterpart of
+ * this call; it exists for such integrations.
+ *  - Same inputs, outputs and results as moe_permute (bit for bit).
+ *  - Scratch: one fixed array inside the library, in device global memory,
+ *    sized for E <= 1024 experts (any T); each GPU that loads the library
+ *    keeps it (128 KB) until the process exits.  E > 1024 returns
+ *    MOE_ERR_UNSUPPORTED.  The call allocates nothing.
+ *  - The first call on a device looks up the array's device address (a
+ *    runtime call, no stream work); make that first call before any stream
+ *    capture.
+ *  - All calls on a device share the array: calls that may overlap on the GPU
+ *    (unordered streams) race and must be serialised by the caller.  Nothing
+ *    needs clearing between calls.
+ *  - Ids outside [0, E) are not reported through a status word (there is no
+ *    workspace); their dest_pos entries come back as -1.
+ */
+int moe_permute_noalloc(const int32_t *topk_ids, int T, int E, int k, int32_t *counts, int32_t *offsets,
+                        int32_t *sorted_slot, int32_t *dest_pos, void *stream);
+
 /* Workspace bytes of moe_expert_ffn_q4 for T tokens. */
 size_t moe_expert_ffn_workspace_size(const moe_config_t *cfg, int T);
 

@@ -16,7 +16,8 @@ __all__ = [
     "MoeError", "Config", "lib", "moe_version", "moe_last_error", "moe_packed_sizes", "moe_pack_weights",
     "moe_dequant_export", "moe_router_logits", "moe_route", "moe_permute_workspace_size", "moe_permute",
     "moe_expert_ffn_workspace_size", "moe_expert_ffn_q4", "moe_combine", "moe_layer_workspace_size",
-    "moe_layer_forward", "moe_read_status", "moe_kernel_launches", "moe_expert_gate_up_q4", "moe_expert_down_q4", "PackedLayer", "WFMT_INT4_SYM", "WFMT_Q4K", "LIB_PATH",
+    "moe_layer_forward", "moe_read_status", "moe_kernel_launches", "moe_expert_gate_up_q4", "moe_expert_down_q4",
+    "moe_permute_noalloc", "PackedLayer", "WFMT_INT4_SYM", "WFMT_Q4K", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoeq4.so")
@@ -87,6 +88,7 @@ def lib():
             "moe_route": (i32, [vp, i32, i32, i32, i32, vp, vp, vp]),
             "moe_permute_workspace_size": (sz, [i32, i32, i32]),
             "moe_permute": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]),
+            "moe_permute_noalloc": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp]),
             "moe_expert_ffn_workspace_size": (sz, [vp, i32]),
             "moe_expert_ffn_q4": (i32, [vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]),
             "moe_combine": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, vp, vp]),
@@ -184,6 +186,12 @@ def moe_permute_workspace_size(T, E, k) -> int:
 def moe_permute(topk_ids, T, E, k, counts, offsets, sorted_slot, dest_pos, ws, ws_bytes, stream=None):
     _call("moe_permute", _ptr(topk_ids), T, E, k, _ptr(counts), _ptr(offsets), _ptr(sorted_slot),
           _ptr(dest_pos), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def moe_permute_noalloc(topk_ids, T, E, k, counts, offsets, sorted_slot, dest_pos, stream=None):
+    """moe_permute with the library's built-in scratch array (no workspace; E <= 1024)."""
+    _call("moe_permute_noalloc", _ptr(topk_ids), T, E, k, _ptr(counts), _ptr(offsets), _ptr(sorted_slot),
+          _ptr(dest_pos), _stream(stream))
 
 
 def moe_expert_ffn_workspace_size(cfg, T) -> int:

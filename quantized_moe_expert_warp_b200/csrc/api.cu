@@ -377,6 +377,29 @@ int moe_permute(const int32_t *topk_ids, int T, int E, int k, int32_t *counts, i
     return ok();
 }
 
+int moe_permute_noalloc(const int32_t *topk_ids, int T, int E, int k, int32_t *counts, int32_t *offsets,
+                        int32_t *sorted_slot, int32_t *dest_pos, void *stream)
+{
+    REQUIRE(T >= 0, "T must be >= 0");
+    if (E < 1 || E > noalloc_max_experts())
+        return fail(MOE_ERR_UNSUPPORTED,
+                    "moe_permute_noalloc: E = %d is outside [1, %d], the size of its built-in scratch array", E,
+                    noalloc_max_experts());
+    REQUIRE(k >= 1 && k <= E, "k must be in [1, E]");
+    REQUIRE((size_t)T * k < (1u << 30), "T*k too large");
+    REQUIRE_PTR(counts);
+    REQUIRE_PTR(offsets);
+    if (T > 0) {
+        REQUIRE_PTR(topk_ids);
+        REQUIRE_PTR(sorted_slot);
+        REQUIRE_PTR(dest_pos);
+    }
+    CUDA_TRY(launch_permute_noalloc(topk_ids, T, E, k, counts, offsets, sorted_slot, dest_pos, (cudaStream_t)stream),
+             "moe_permute_noalloc");
+    g_launches += T > 0 ? 2 : 0;
+    return ok();
+}
+
 size_t moe_expert_ffn_workspace_size(const moe_config_t *cfg, int T)
 {
     if (check_config(cfg) || T < 0)

@@ -52,6 +52,10 @@ size_t permute_scratch_bytes(int T, int E, int k);
 cudaError_t launch_permute(const int32_t *ids, int T, int E, int k, int32_t *counts, int32_t *offsets,
                            int32_t *sorted_slot, int32_t *dest_pos, void *scratch, int *status, cudaStream_t st);
 
+int noalloc_max_experts();
+cudaError_t launch_permute_noalloc(const int32_t *ids, int T, int E, int k, int32_t *counts, int32_t *offsets,
+                                   int32_t *sorted_slot, int32_t *dest_pos, cudaStream_t st);
+
 cudaError_t launch_combine(const uint16_t *y_perm, const int32_t *dest_pos, const float *w, const uint16_t *shared_out,
                            const float *gate_logit, int T, int H, int k, uint16_t *y, cudaStream_t st);
 

@@ -10,6 +10,7 @@
 //           per-warp counts) and scatters.  CTA 0 writes counts and offsets.
 // No floating point and no atomics on the outputs: the result is unique.
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "kernels.h"
@@ -148,6 +149,89 @@ cudaError_t launch_permute(const int32_t *ids, int T, int E, int k, int32_t *cou
     int32_t *hist = (int32_t *)scratch;
     permute_hist_kernel<<<nblk, kPermThreads, E * sizeof(int32_t), st>>>(ids, S, E, chunk, hist, status);
     cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess)
+        return err;
+    const size_t smem = (E + kPermThreads) * sizeof(int32_t) + 32 * E * sizeof(uint16_t);
+    if (smem > 48 * 1024) {
+        err = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess)
+            return err;
+    }
+    permute_scatter_kernel<<<nblk, kPermThreads, smem, st>>>(ids, S, E, chunk, hist, counts, offsets, sorted_slot,
+                                                              dest_pos);
+    return cudaGetLastError();
+}
+
+
+// ------------------------------------------------------------------------
+// Allocation-free variant of moe_permute.
+//
+// Some callers cannot allocate device memory at the point where they need a
+// permutation: code running inside another allocator's critical section, a
+// plugin host that forbids cudaMalloc after start-up, or a caller that has no
+// workspace to hand over.  For them the chunk histograms live in one
+// fixed-size array in device global memory that belongs to this library.
+// Its size bounds the expert count (E <= kNoAllocMaxExperts); the token count
+// is not bounded by it, because the slots are always cut into at most 32
+// chunks.  Every GPU that loads the library keeps the array until the process
+// exits.
+//
+// The array is shared by all calls on a device: two calls that overlap on the
+// GPU (different streams without ordering between them) race on it.  Each
+// call rewrites every histogram entry it later reads, so nothing has to be
+// cleared between calls.
+// ------------------------------------------------------------------------
+
+constexpr int kNoAllocMaxExperts = 1024;
+static __device__ __align__(256) int32_t g_noalloc_hist[kPermMaxChunks * kNoAllocMaxExperts];
+
+// Device address of g_noalloc_hist, looked up once per device (the name
+// alone is a host-side stand-in, not a device address).
+static int32_t *noalloc_hist_ptr(cudaError_t *err)
+{
+    static std::mutex mu;
+    static int32_t *ptrs[64] = {nullptr};
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess)
+        return nullptr;
+    if (dev < 0 || dev >= 64) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        *err = cudaGetSymbolAddress(&p, g_noalloc_hist);
+        if (*err != cudaSuccess)
+            return nullptr;
+        ptrs[dev] = (int32_t *)p;
+    }
+    return ptrs[dev];
+}
+
+int noalloc_max_experts() { return kNoAllocMaxExperts; }
+
+cudaError_t launch_permute_noalloc(const int32_t *ids, int T, int E, int k, int32_t *counts, int32_t *offsets,
+                                   int32_t *sorted_slot, int32_t *dest_pos, cudaStream_t st)
+{
+    const int S = T * k;
+    if (S == 0) {
+        cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st);
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st);
+        return e;
+    }
+    cudaError_t err = cudaSuccess;
+    int32_t *hist = noalloc_hist_ptr(&err);
+    if (!hist)
+        return err;
+    const int chunk = perm_chunk(S);
+    const int nblk = perm_blocks(S);
+    // ids outside [0, E) are not reported through a status word here; their
+    // dest_pos entries come back as -1
+    permute_hist_kernel<<<nblk, kPermThreads, E * sizeof(int32_t), st>>>(ids, S, E, chunk, hist, nullptr);
+    err = cudaGetLastError();
     if (err != cudaSuccess)
         return err;
     const size_t smem = (E + kPermThreads) * sizeof(int32_t) + 32 * E * sizeof(uint16_t);
