@@ -57,7 +57,7 @@ extern "C" {
 #define MOE_WFMT_Q4K 1      /* Q4_K-style 256-weight super-blocks (see moe_pack_weights)   */
 
 /* Shapes of one layer.  Admitted: H % 128 == 0, I % 128 == 0, 1 <= k <= E <= 1024,
- * int4-sym: G % 32 == 0 and G divides H and I; Q4K: H % 256 == 0, I % 256 == 0. */
+ * int4-sym: G a power of two, G >= 32, G divides H and I; Q4K: H % 256 == 0, I % 256 == 0. */
 typedef struct moe_config {
     int32_t H;          /* hidden size                                   */
     int32_t I;          /* expert intermediate size (shared expert too)  */

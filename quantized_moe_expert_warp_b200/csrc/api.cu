@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <cuda_runtime.h>
 
@@ -63,6 +64,9 @@ bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// CTAs of the persistent kernels: one per SM.  MOEQ4_GRID_CTAS (1 .. SM
+// count) launches fewer, so that tests can give each CTA many work units
+// and wrap its shared-memory rings on small problems.
 int num_sms()
 {
     static int cache[64] = {0};
@@ -74,6 +78,12 @@ int num_sms()
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             n = 148;
         cache[dev] = n;
+    }
+    const char *env = getenv("MOEQ4_GRID_CTAS");
+    if (env) {
+        const int g = atoi(env);
+        if (g >= 1 && g < cache[dev])
+            return g;
     }
     return cache[dev];
 }
@@ -91,8 +101,9 @@ int check_config(const moe_config_t *c)
     if (c->E > 1024 || c->k > 32 || c->k > c->E)
         return fail(MOE_ERR_UNSUPPORTED, "cfg: need k <= min(E, 32) and E <= 1024 (E=%d k=%d)", c->E, c->k);
     if (c->wfmt == MOE_WFMT_INT4_SYM) {
-        if (c->G <= 0 || c->G % 32 || c->H % c->G || c->I % c->G)
-            return fail(MOE_ERR_UNSUPPORTED, "cfg: int4 group G=%d must be a multiple of 32 dividing H and I", c->G);
+        if (c->G < 32 || (c->G & (c->G - 1)) || c->H % c->G || c->I % c->G)
+            return fail(MOE_ERR_UNSUPPORTED, "cfg: int4 group G=%d must be a power of two >= 32 dividing H and I",
+                        c->G);
     } else if (c->H % 256 || c->I % 256) {
         return fail(MOE_ERR_UNSUPPORTED, "cfg: Q4K needs H and I multiples of 256");
     }
@@ -210,6 +221,7 @@ int run_expert_ffn(const moe_layer_t *L, const uint16_t *x, int T, const int32_t
         a.wmeta = (const uint8_t *)L->gu_meta;
         a.b_src = x;
         a.ldb = c.H;
+        a.b_rows = T;
         a.K = c.H;
         a.F = c.I / kTileRows;
         a.meta_bytes = meta_block_bytes(2, c.wfmt, c.H, c.G);
@@ -225,6 +237,7 @@ int run_expert_ffn(const moe_layer_t *L, const uint16_t *x, int T, const int32_t
         a.wmeta = (const uint8_t *)L->dn_meta;
         a.b_src = h;
         a.ldb = c.I;
+        a.b_rows = Tk + (c.has_shared ? T : 0);
         a.K = c.I;
         a.F = c.H / kTileRows;
         a.meta_bytes = meta_block_bytes(1, c.wfmt, c.I, c.G);

@@ -33,6 +33,11 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#ifdef MOEQ4_TRACE
+// per wait site, summed over warps: [0] waits that polled more than once, [1] failed polls
+__device__ unsigned long long g_wait_stats[16][2];
+#endif
+
 #include "dequant.cuh"
 #include "kernels.h"
 #include "moeq4.h"
@@ -53,7 +58,7 @@ constexpr int kTraceSteps = 512;
 __device__ unsigned long long g_trace[4][16][kTraceSteps];
 #define TRACE_EVENT(ev, step)                                                          \
     do {                                                                               \
-        if (blockIdx.x < 4 && (step) >= 0 && (step) < kTraceSteps)                     \
+        if (blockIdx.x < 4 && (ev) >= 0 && (ev) < 16 && (step) >= 0 && (step) < kTraceSteps) \
             g_trace[blockIdx.x][(ev)][(step)] = globaltimer_ns();                      \
     } while (0)
 #else
@@ -62,13 +67,14 @@ __device__ unsigned long long g_trace[4][16][kTraceSteps];
     } while (0)
 #endif
 
-constexpr int kBNMax = 128;  // max tokens per tile (the MMA's N); tiles of 64 when groups are small
-constexpr int kStages = 4;   // B / TMEM-A pipeline depth
+constexpr int kAStages = 4;  // TMEM A-operand ring depth (dequantised k-steps)
+constexpr int kMaxCodeChunks = 8;   // code ring: chunks of several k-steps, one bulk copy each
+constexpr int kMaxMetaBufs = 4;
 constexpr int kEpiTok = 16;  // tokens per epilogue chunk
 constexpr int kEpiStride = 80;                                   // bytes per staged token row (64 + pad)
 constexpr int kEpiBytes = 4 * kEpiTok * kEpiStride;              // staging for the four epilogue warps
-constexpr int kDeqGroups = 2;                  // dequant warp groups, alternating k-steps
-constexpr int kThreads = (8 + 8 * kDeqGroups) * 32;
+constexpr int kDeqWarps = 16;                  // dequant warps (warps 4 .. 19)
+constexpr int kThreads = (8 + kDeqWarps) * 32;
 
 enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_ROUTER = 2 };
 
@@ -80,24 +86,33 @@ struct Geo {
     static constexpr int kNAcc_ = MODE == MODE_GATE_UP ? 2 : 1;
     // as many accumulator buffers (up to 2) as TMEM holds next to the A stages:
     // with two, the epilogue of one tile overlaps the MMAs of the next
-    static constexpr int kAccBufs = (512 - kStages * kNA * 32) / (kNAcc_ * BN) >= 2 ? 2 : 1;
+    static constexpr int kAccBufs = (512 - kAStages * kNA * 32) / (kNAcc_ * BN) >= 2 ? 2 : 1;
     static constexpr int kNCode = MODE == MODE_GATE_UP ? 2 : MODE == MODE_DOWN ? 1 : 0; // code matrices
-    static constexpr int kCodeStages = MODE == MODE_GATE_UP ? 8 : MODE == MODE_DOWN ? 16 : 1;
-    static constexpr int kCodeBytes = kCodeStages * (kNCode ? code_block_bytes(kNCode) : 0);
-    static constexpr int kBBytes = kStages * BN * 128;
+    // dequant warp groups: four groups of four warps, each warp a full k-step
+    // of its 32 rows (router: two groups of eight, one half each)
+    static constexpr int kGroups = MODE == MODE_ROUTER ? 2 : 4;
+    static constexpr int kGroupWarps = kDeqWarps / kGroups;
+    static constexpr int kHalves = kGroupWarps == 8 ? 1 : 2;
+    static constexpr int kCodeBlock = kNCode ? code_block_bytes(kNCode) : 0;
+    // the gathered token rows wait on L2 / HBM latency, so their shared-memory
+    // ring is deeper than the TMEM ring
+    static constexpr int kBStages = BN == 64 ? 8 : 4;
+    static constexpr int kBBytes = kBStages * BN * 128;
     static constexpr int kAccCols = kAccBufs * kNAcc * BN;
     static constexpr int kTmemCols = 512;
-    static_assert(kAccCols + kStages * kNA * 32 <= kTmemCols, "TMEM budget");
+    static_assert(kAccCols + kAStages * kNA * 32 <= kTmemCols, "TMEM budget");
     static constexpr bool kGather = MODE == MODE_GATE_UP;
 };
 
 struct Barriers {
-    uint64_t full[kStages];       // A dequantised into TMEM and B gathered into shared memory
-    uint64_t mma_done[kStages];
-    uint64_t code_full[16];
-    uint64_t code_empty[16];
-    uint64_t meta_full[2];
-    uint64_t meta_empty[2];
+    uint64_t a_full[kAStages];    // k-step dequantised into TMEM (8 dequant warps)
+    uint64_t a_empty[kAStages];   // MMAs reading that TMEM stage completed
+    uint64_t b_full[8];           // token rows landed in shared memory (32 cp.async arrivals)
+    uint64_t b_empty[8];
+    uint64_t code_full[kMaxCodeChunks];
+    uint64_t code_empty[kMaxCodeChunks];
+    uint64_t meta_full[kMaxMetaBufs];
+    uint64_t meta_empty[kMaxMetaBufs];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
@@ -205,10 +220,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *sB = smem;
     uint8_t *sCode = sB + L::kBBytes;
-    uint8_t *sMeta = sCode + L::kCodeBytes;
+    // code ring: NCS chunks of CK k-steps; meta ring: NMETA per-tile blocks
+    const int CK = 1 << p.ck_log2, NCS = 1 << p.ncs_log2, NMETA = 1 << p.nmeta_log2;
+    const int chunk_bytes = CK * L::kCodeBlock;
+    uint8_t *sMeta = sCode + NCS * chunk_bytes;
     const int meta_bytes = p.meta_bytes;
     const int meta_al = (meta_bytes + 127) & ~127;
-    Barriers *bars = (Barriers *)(sMeta + 2 * meta_al);
+    Barriers *bars = (Barriers *)(sMeta + NMETA * meta_al);
     int *s_tile_start = (int *)(bars + 1);
     int *s_row_start = s_tile_start + p.E_total + 1;
     int *s_row_count = s_row_start + p.E_total;
@@ -221,18 +239,23 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
     const int lane = threadIdx.x % 32;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            // eight dequant warps + one cp.async completion arrival per lane of the B producer
-            mbar_init(&bars->full[s], 8 + 32);
-            mbar_init(&bars->mma_done[s], 1);
+        for (int s = 0; s < kAStages; ++s) {
+            mbar_init(&bars->a_full[s], L::kGroupWarps);
+            mbar_init(&bars->a_empty[s], 1);
         }
-        for (int s = 0; s < L::kCodeStages; ++s) {
+        for (int s = 0; s < L::kBStages; ++s) {
+            mbar_init(&bars->b_full[s], 32);   // one cp.async completion arrival per lane of the B producer
+            mbar_init(&bars->b_empty[s], 1);
+        }
+        for (int s = 0; s < NCS; ++s) {
             mbar_init(&bars->code_full[s], 1);
-            mbar_init(&bars->code_empty[s], 8);
+            mbar_init(&bars->code_empty[s], kDeqWarps);   // every dequant warp reads every chunk
+        }
+        for (int s = 0; s < NMETA; ++s) {
+            mbar_init(&bars->meta_full[s], 1);
+            mbar_init(&bars->meta_empty[s], kDeqWarps);
         }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars->meta_full[s], 1);
-            mbar_init(&bars->meta_empty[s], 8 * kDeqGroups);
             mbar_init(&bars->acc_full[s], 1);
             mbar_init(&bars->acc_empty[s], 4);
         }
@@ -256,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
     WaitCtx wc{&bars->abort_flag, p.status, globaltimer_ns()};
 
     if (warp == 0) {
-        // ------------------------------------------------ B producer (gather)
+        // ------------------------------------------------ B producer (cp.async row gather)
         int step = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
@@ -274,8 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                 bytes[i] = r < un.nvalid ? 16u : 0u;
             }
             for (int ks = 0; ks < KS; ++ks, ++step) {
-                const int s = step % kStages;
-                if (step >= kStages && !mbar_wait(&bars->mma_done[s], ((step / kStages) & 1) ^ 1, wc, 1)) {
+                const int s = step % L::kBStages;
+                if (step >= L::kBStages && !mbar_wait(&bars->b_empty[s], ((step / L::kBStages) & 1) ^ 1, wc, 1)) {
                     ok = false;
                     break;
                 }
@@ -291,8 +314,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                             cp_async_16(rbase + ((j ^ (r & 7)) << 4), g + j * 8, bytes[i]);
                     }
                 }
-                // this lane's copies for the stage arrive on full[s] when they land
-                cp_async_arrive_noinc(&bars->full[s]);
+                // this lane's copies for the stage arrive on b_full[s] when they land
+                cp_async_arrive_noinc(&bars->b_full[s]);
                 if (lane == 0)
                     TRACE_OTHER(0, step);
             }
@@ -312,21 +335,21 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                 tc_fence_after();
             }
             for (int ks = 0; ks < KS; ++ks, ++step) {
-                const int s = step % kStages;
-                const uint32_t ph = (step / kStages) & 1;
-                // every lane polls the same barrier, so the outcome is warp-uniform
-                if (!mbar_wait(&bars->full[s], ph, wc, 3)) {
+                const int sa = step % kAStages, sb = step % L::kBStages;
+                // every lane polls the same barriers, so the outcome is warp-uniform
+                if (!mbar_wait(&bars->a_full[sa], (step / kAStages) & 1, wc, 3) ||
+                    !mbar_wait(&bars->b_full[sb], (step / L::kBStages) & 1, wc, 4)) {
                     ok = false;
                     break;
                 }
                 if (lane == 0)
                     TRACE_OTHER(9, step);
+                tc_fence_after();
                 // the B stage was written by cp.async (generic proxy); the MMA
                 // reads it through the async proxy
                 fence_proxy_async_smem();
-                tc_fence_after();
-                const uint64_t bdesc0 = sdesc_kmajor_sw128(smem_u32(sB + s * kBN * 128));
-                const uint32_t a_base = tmem + L::kAccCols + s * L::kNA * 32;
+                const uint64_t bdesc0 = sdesc_kmajor_sw128(smem_u32(sB + sb * kBN * 128));
+                const uint32_t a_base = tmem + L::kAccCols + sa * L::kNA * 32;
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
@@ -340,7 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                                 mma_ts_f16(acc + m * kBN, a_t, bdesc, idesc, (ks | kk) != 0);
                         }
                     }
-                    mma_commit(&bars->mma_done[s]);
+                    mma_commit(&bars->a_empty[sa]);
+                    mma_commit(&bars->b_empty[sb]);
                 }
                 __syncwarp();
                 if (lane == 0)
@@ -360,40 +384,81 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
         warp_wait(&bars->drain, 0, wd, 5);
     } else if (warp == 2) {
         // ------------------------------------------------ code / meta producer (converged warp)
+        // A unit's code blocks are contiguous in the kernel layout, so one bulk
+        // copy moves CK k-steps: the copy engine's throughput is set by the
+        // number of copies more than by their size.
         if (MODE != MODE_ROUTER) {
-            int step = 0, munit = 0;
-            const int cbytes = code_block_bytes(L::kNCode);
+            int cidx = 0, munit = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++munit) {
                 const Unit un = decode_unit<BN>(u, p, sched);
                 const size_t tile_id = (size_t)un.e * p.F + un.f;
-                const int mb = munit & 1;
-                if (munit >= 2 && !warp_wait(&bars->meta_empty[mb], ((munit >> 1) & 1) ^ 1, wc, 6))
+                const int mb = munit & (NMETA - 1);
+                if (munit >= NMETA &&
+                    !warp_wait(&bars->meta_empty[mb], ((munit >> p.nmeta_log2) & 1) ^ 1, wc, 6))
                     break;
                 if (elect_one()) {
                     mbar_arrive_expect_tx(&bars->meta_full[mb], meta_bytes);
                     bulk_g2s(sMeta + mb * meta_al, p.wmeta + tile_id * meta_bytes, meta_bytes, &bars->meta_full[mb]);
                 }
                 __syncwarp();
-                for (int ks = 0; ks < KS; ++ks, ++step) {
-                    const int s = step % L::kCodeStages;
-                    if (step >= L::kCodeStages &&
-                        !warp_wait(&bars->code_empty[s], ((step / L::kCodeStages) & 1) ^ 1, wc, 7)) {
+                for (int c0 = 0; c0 < KS; c0 += CK, ++cidx) {
+                    const int s = cidx & (NCS - 1);
+                    if (cidx >= NCS && !warp_wait(&bars->code_empty[s], ((cidx >> p.ncs_log2) & 1) ^ 1, wc, 7)) {
                         ok = false;
                         break;
                     }
+                    const uint32_t bytes = (uint32_t)(min(CK, KS - c0) * L::kCodeBlock);
                     if (elect_one()) {
-                        mbar_arrive_expect_tx(&bars->code_full[s], cbytes);
-                        bulk_g2s(sCode + s * cbytes, p.wq + (tile_id * KS + ks) * cbytes, cbytes,
+                        mbar_arrive_expect_tx(&bars->code_full[s], bytes);
+                        bulk_g2s(sCode + s * chunk_bytes, p.wq + (tile_id * KS + c0) * L::kCodeBlock, bytes,
                                  &bars->code_full[s]);
                     }
                     __syncwarp();
                     if (lane == 0)
-                        TRACE_OTHER(1, step);
+                        TRACE_OTHER(1, cidx);
                 }
             }
         }
     } else if (warp == 3) {
+#ifdef MOEQ4_TRACE
+        // instrumented builds, first CTAs: record when each code chunk lands
+        // (event 14, by chunk), each B stage lands (event 8, by step) and each
+        // A stage is complete in TMEM (event 10, by step)
+        if (MODE != MODE_ROUTER && blockIdx.x < 4 && lane == 0) {
+            int n_units = 0;
+            for (int u = blockIdx.x; u < total_units; u += gridDim.x)
+                ++n_units;
+            const int n_chunks = n_units * ((KS + CK - 1) / CK), n_steps = n_units * KS;
+            int ci = 0, bi = 0, ai = 0;
+            uint64_t t_last = globaltimer_ns();
+            auto test = [](uint32_t bar, uint32_t par) {
+                uint32_t done;
+                asm volatile("{\n\t.reg .pred q;\n\t"
+                             "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 q, [%1], %2;\n\t"
+                             "selp.u32 %0, 1, 0, q;\n\t}"
+                             : "=r"(done) : "r"(bar), "r"(par) : "memory");
+                return done != 0;
+            };
+            while ((ci < n_chunks || bi < n_steps || ai < n_steps) && globaltimer_ns() - t_last < 200000) {
+                if (ci < n_chunks && test(smem_u32(&bars->code_full[ci & (NCS - 1)]), (ci >> p.ncs_log2) & 1)) {
+                    TRACE_EVENT(14, ci);
+                    ++ci;
+                    t_last = globaltimer_ns();
+                }
+                if (bi < n_steps && test(smem_u32(&bars->b_full[bi % L::kBStages]), (bi / L::kBStages) & 1)) {
+                    TRACE_EVENT(8, bi);
+                    ++bi;
+                    t_last = globaltimer_ns();
+                }
+                if (ai < n_steps && test(smem_u32(&bars->a_full[ai % kAStages]), (ai / kAStages) & 1)) {
+                    TRACE_EVENT(10, ai);
+                    ++ai;
+                    t_last = globaltimer_ns();
+                }
+            }
+        }
+#endif
         // ------------------------------------------------ shared-expert gate logits
         if (MODE == MODE_ROUTER && p.gate_w) {
             for (int t = blockIdx.x; t < p.T; t += gridDim.x) {
@@ -419,39 +484,54 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                     p.gate_out[t] = acc;
             }
         }
-    } else if (warp >= 4 && warp < 4 + 8 * kDeqGroups) {
+    } else if (warp >= 4 && warp < 4 + kDeqWarps) {
         // ------------------------------------------------ dequant into TMEM
+        // Groups of L::kGroupWarps warps take k-steps round-robin; a warp owns
+        // TMEM lane quadrant warp % 4 (32 weight rows) and L::kHalves of the
+        // two 32-element halves of each of its k-steps.
         const int dw = warp - 4;
-        const int grp = dw / 8;                   // this group handles k-steps with step % kDeqGroups == grp
-        const int c = (dw & 7) >> 2;              // which 32-element half of the k-step
-        const int r = (warp & 3) * 32 + lane;     // tile row == TMEM lane
+        const int grp = dw / L::kGroupWarps;              // k-steps with step % kGroups == grp
+        const int c0 = L::kHalves == 1 ? (dw & 7) >> 2 : 0;
+        const int r = (warp & 3) * 32 + lane;             // tile row == TMEM lane
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        int step = 0, munit = 0;
+        const int gshift = __ffs(max(p.G, 1)) - 1;        // int4-sym groups are a power of two
+        int step = 0, munit = 0, cbase = 0;               // cbase: code chunk index of the unit's first k-step
         bool ok = true;
         for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++munit) {
-            const int mb = munit & 1;
+            const int mb = munit & (NMETA - 1);
             const uint8_t *meta = sMeta + mb * meta_al;
-            float4 pre[8];                        // router: this row's next k-step, prefetched
+            float4 pre[8];                                // router: this row's next k-step, prefetched
             const float *wrow = nullptr;
             if (MODE == MODE_ROUTER) {
                 const Unit un = decode_unit<BN>(u, p, sched);
                 const int e = un.f * kTileRows + r;
-                wrow = e < p.E ? p.a_f32 + (size_t)e * p.K + c * 32 : nullptr;
-                const int ks0 = ((grp - step) % kDeqGroups + kDeqGroups) % kDeqGroups;   // first k-step of this group
+                wrow = e < p.E ? p.a_f32 + (size_t)e * p.K + c0 * 32 : nullptr;
+                const int ks0 = ((grp - step) % L::kGroups + L::kGroups) % L::kGroups;   // first k-step of this group
                 if (ks0 >= KS)
                     wrow = nullptr;
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     pre[i] = wrow ? *(const float4 *)(wrow + ks0 * kKStep + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
-            } else if (!mbar_wait(&bars->meta_full[mb], (munit >> 1) & 1, wc, 8)) {
+            } else if (!mbar_wait(&bars->meta_full[mb], (munit >> p.nmeta_log2) & 1, wc, 8)) {
                 break;
             }
-            const int ngroups = WFMT == MOE_WFMT_Q4K ? p.K / 256 : p.K / max(p.G, 1);
+            const int ngroups = WFMT == MOE_WFMT_Q4K ? p.K / 256 : p.K >> gshift;
             for (int ks = 0; ks < KS; ++ks, ++step) {
-                if (step % kDeqGroups != grp)
+                // every dequant warp frees every code chunk once, after its own
+                // k-steps in the chunk (it may have none)
+                const bool chunk_last = MODE != MODE_ROUTER && (((ks + 1) & (CK - 1)) == 0 || ks + 1 == KS);
+                if (step % L::kGroups != grp) {
+                    if (chunk_last) {
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(&bars->code_empty[(cbase + (ks >> p.ck_log2)) & (NCS - 1)]);
+                    }
                     continue;
-                uint32_t words[L::kNA][16];
+                }
+                const int sa = step % kAStages;
+                const uint32_t a_col = tmem + lane_off + L::kAccCols + sa * L::kNA * 32;
                 if (MODE == MODE_ROUTER) {
+                    uint32_t words[L::kNA][16];
                     float v[32];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
@@ -460,17 +540,28 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                         v[4 * i + 2] = pre[i].z;
                         v[4 * i + 3] = pre[i].w;
                     }
-                    if (wrow && ks + kDeqGroups < KS) {
+                    if (wrow && ks + L::kGroups < KS) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
-                            pre[i] = *(const float4 *)(wrow + (ks + kDeqGroups) * kKStep + 4 * i);
+                            pre[i] = *(const float4 *)(wrow + (ks + L::kGroups) * kKStep + 4 * i);
                     }
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        split2(v[2 * j], v[2 * j + 1], words[0][j], words[1 % L::kNA][j]);
+                    for (int jj = 0; jj < 16; ++jj)
+                        split2(v[2 * jj], v[2 * jj + 1], words[0][jj], words[1 % L::kNA][jj]);
+                    if (step >= kAStages && !mbar_wait(&bars->a_empty[sa], ((step / kAStages) & 1) ^ 1, wc, 10)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int m = 0; m < L::kNA; ++m)
+                        tmem_st16(a_col + m * 32 + c0 * 16, words[m]);
                 } else {
-                    const int sc = step % L::kCodeStages;
-                    if (!mbar_wait(&bars->code_full[sc], (step / L::kCodeStages) & 1, wc, 9)) {
+                    const int cidx = cbase + (ks >> p.ck_log2);
+                    const int sc = cidx & (NCS - 1);
+                    if (lane == 0 && warp == 4)
+                        TRACE_OTHER(15, step);
+                    if (!mbar_wait(&bars->code_full[sc], (cidx >> p.ncs_log2) & 1, wc, 9)) {
                         ok = false;
                         break;
                     }
@@ -481,56 +572,62 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                     if (lane == 0 && warp == 4)
                         TRACE_EVENT(2, step);
 #endif
-                    const int kpos = ks * kKStep + c * 32;
-                    const int cbytes = code_block_bytes(L::kNCode);
+                    const uint32_t cblk = smem_u32(sCode) + sc * chunk_bytes + (ks & (CK - 1)) * L::kCodeBlock;
+#pragma unroll 1
+                    for (int h = 0; h < L::kHalves; ++h) {
+                        const int c = c0 + h;
+                        const int kpos = ks * kKStep + c * 32;
+                        uint32_t words[L::kNA][16];
 #pragma unroll
-                    for (int m = 0; m < L::kNA; ++m) {
-                        const uint4 codes =
-                            lds128(smem_u32(sCode) + sc * cbytes + ((m * 2 + c) * kTileRows + r) * kChunkBytes);
-                        if (WFMT == MOE_WFMT_Q4K) {
-                            const int g = kpos / 256;
-                            const uint4 hdr = lds128(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 16);
-                            float dsc, dm;
-                            q4k_subblock_scale(hdr, (kpos % 256) / 32, dsc, dm);
-                            dequant_q4k_chunk(codes, dsc, dm, words[m]);
-                        } else {
-                            const int g = kpos / p.G;
-                            const uint16_t sbits = lds16(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 2);
-                            dequant_int4sym_chunk(codes, sbits, words[m]);
+                        for (int m = 0; m < L::kNA; ++m) {
+                            const uint4 codes = lds128(cblk + ((m * 2 + c) * kTileRows + r) * kChunkBytes);
+                            if (WFMT == MOE_WFMT_Q4K) {
+                                const int g = kpos / 256;
+                                const uint4 hdr = lds128(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 16);
+                                float dsc, dm;
+                                q4k_subblock_scale(hdr, (kpos % 256) / 32, dsc, dm);
+                                dequant_q4k_chunk(codes, dsc, dm, words[m]);
+                            } else {
+                                const int g = kpos >> gshift;
+                                const uint16_t sbits = lds16(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 2);
+                                dequant_int4sym_chunk(codes, sbits, words[m]);
+                            }
                         }
-                    }
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(&bars->code_empty[sc]);
-                }
-                const int sa = step % kStages;
-#ifdef MOEQ4_TRACE_WARPS
-                if (lane == 0)
-                    TRACE_EVENT((warp - 4) * 2 + 1, step);
-#else
-                if (lane == 0 && warp == 4)
-                    TRACE_EVENT(11, step);
-#endif
-                if (step >= kStages && !mbar_wait(&bars->mma_done[sa], ((step / kStages) & 1) ^ 1, wc, 10)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0 && warp == 4)
-                    TRACE_OTHER(12, step);
-                tc_fence_after();
+                        if (h == 0) {
+                            if (lane == 0 && warp == 4)
+                                TRACE_EVENT(11, step);
+                            // the MMAs that read this TMEM stage kAStages k-steps ago have finished
+                            if (step >= kAStages &&
+                                !mbar_wait(&bars->a_empty[sa], ((step / kAStages) & 1) ^ 1, wc, 10)) {
+                                ok = false;
+                                break;
+                            }
+                            if (lane == 0 && warp == 4)
+                                TRACE_OTHER(12, step);
+                            tc_fence_after();
+                        }
 #pragma unroll
-                for (int m = 0; m < L::kNA; ++m)
-                    tmem_st16(tmem + lane_off + L::kAccCols + (sa * L::kNA + m) * 32 + c * 16, words[m]);
+                        for (int m = 0; m < L::kNA; ++m)
+                            tmem_st16(a_col + m * 32 + c * 16, words[m]);
+                    }
+                    if (!ok)
+                        break;
+                    if (chunk_last) {
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(&bars->code_empty[sc]);
+                    }
+                }
                 tmem_wait_st();
                 if (lane == 0 && warp == 4)
                     TRACE_OTHER(13, step);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
-                    mbar_arrive(&bars->full[sa]);
+                    mbar_arrive(&bars->a_full[sa]);
                 if (lane == 0 && warp == 4)
                     TRACE_OTHER(3, step);
-                if (lane == 0 && warp == 11)
+                if (lane == 0 && warp == 7)
                     TRACE_OTHER(4, step);
             }
             if (MODE != MODE_ROUTER) {
@@ -538,6 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                 if (lane == 0)
                     mbar_arrive(&bars->meta_empty[mb]);
             }
+            cbase += (KS + CK - 1) >> p.ck_log2;
         }
     } else {
         // ------------------------------------------------ epilogue (last four warps)
@@ -550,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
             if (!mbar_wait(&bars->acc_full[ab], (uidx / L::kAccBufs) & 1, wc, 11))
                 break;
             tc_fence_after();
-            if (lane == 0 && warp == 4 + 8 * kDeqGroups)
+            if (lane == 0 && warp == 4 + kDeqWarps)
                 TRACE_OTHER(6, uidx);
             const uint32_t acc = tmem + lane_off + ab * L::kNAcc * kBN;
             const int col = un.f * kTileRows + r;
@@ -616,11 +714,22 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                 if (lane == 0)
                     mbar_arrive(&bars->acc_empty[ab]);
             }
-            if (lane == 0 && warp == 4 + 8 * kDeqGroups)
+            if (lane == 0 && warp == 4 + kDeqWarps)
                 TRACE_OTHER(7, uidx);
         }
     }
 
+#ifdef MOEQ4_TRACE
+    if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (wc.waits[i]) {
+                atomicAdd(&g_wait_stats[i][0], (unsigned long long)wc.waits[i]);
+                atomicAdd(&g_wait_stats[i][1], (unsigned long long)wc.polls[i]);
+            }
+        }
+    }
+#endif
     __syncthreads();
     if (warp == 3) {
         tc_fence_after();
@@ -628,22 +737,62 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
     }
 }
 
+constexpr size_t kSmemLimit = 227 * 1024;
+
+// Shared-memory ring configuration of one launch (all counts are powers of two).
+struct Rings {
+    int ck_log2, ncs_log2, nmeta_log2;
+};
+
 template <int MODE, int BN>
-static size_t gemm_smem_bytes(int meta_bytes, int E_total)
+static size_t gemm_smem_bytes(int meta_bytes, int E_total, const Rings &r)
 {
     using L = Geo<MODE, BN>;
-    const size_t need = 1024 + L::kBBytes + L::kCodeBytes + 2 * ((meta_bytes + 127) & ~127) + sizeof(Barriers) +
-                        sizeof(int) * (3 * E_total + 1 + kThreads) + 16 + kEpiBytes;
+    const size_t code = ((size_t)L::kCodeBlock << r.ck_log2) << r.ncs_log2;
+    const size_t need = 1024 + L::kBBytes + code + ((size_t)((meta_bytes + 127) & ~127) << r.nmeta_log2) +
+                        sizeof(Barriers) + sizeof(int) * (3 * E_total + 1 + kThreads) + 16 + kEpiBytes;
     // at least half of the SM's shared memory, so that one CTA (and one TMEM
     // allocation) runs per SM
     return need > 116 * 1024 ? need : 116 * 1024;
 }
 
+// Code chunks of up to 32 KB (CK k-steps per bulk copy) and as many chunks in
+// flight (up to 8, at least 4 where possible) as shared memory holds; four
+// meta blocks in flight when they are small.
+template <int MODE, int BN>
+static Rings gemm_rings(int meta_bytes, int E_total, int KS)
+{
+    using L = Geo<MODE, BN>;
+    Rings r{0, 0, 1};
+    if (MODE == MODE_ROUTER)
+        return r;
+    r.nmeta_log2 = meta_bytes <= 4096 ? 2 : 1;
+    r.ck_log2 = 1;
+    while ((L::kCodeBlock << (r.ck_log2 + 1)) <= 32768 && (1 << (r.ck_log2 + 1)) <= KS)
+        ++r.ck_log2;
+    for (;;) {
+        r.ncs_log2 = 3;
+        while (r.ncs_log2 > 1 && gemm_smem_bytes<MODE, BN>(meta_bytes, E_total, r) > kSmemLimit)
+            --r.ncs_log2;
+        if (r.ncs_log2 >= 2 || r.ck_log2 == 1)
+            break;
+        --r.ck_log2;
+    }
+    return r;
+}
+
 template <int MODE, int WFMT, int BN>
-static cudaError_t launch_one(const GemmArgs &a, int num_sms, cudaStream_t st)
+static cudaError_t launch_one(const GemmArgs &a_in, int num_sms, cudaStream_t st)
 {
     auto kern = grouped_gemm_kernel<MODE, WFMT, BN>;
-    const size_t smem = gemm_smem_bytes<MODE, BN>(a.meta_bytes, a.E_total);
+    GemmArgs a = a_in;
+    const Rings r = gemm_rings<MODE, BN>(a.meta_bytes, a.E_total, a.K / kKStep);
+    a.ck_log2 = r.ck_log2;
+    a.ncs_log2 = r.ncs_log2;
+    a.nmeta_log2 = r.nmeta_log2;
+    const size_t smem = gemm_smem_bytes<MODE, BN>(a.meta_bytes, a.E_total, r);
+    if (smem > kSmemLimit)
+        return cudaErrorInvalidConfiguration;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
@@ -653,9 +802,13 @@ static cudaError_t launch_one(const GemmArgs &a, int num_sms, cudaStream_t st)
 
 size_t gemm_smem_required(int nmat, int meta_bytes, int E_total)
 {
-    // the 128-token tile is the larger of the two configurations
-    return nmat == 2 ? gemm_smem_bytes<MODE_GATE_UP, 128>(meta_bytes, E_total)
-                     : gemm_smem_bytes<MODE_DOWN, 128>(meta_bytes, E_total);
+    // the smallest rings (two chunks of two k-steps, two meta blocks) of the larger tile
+    const Rings r{1, 1, 1};
+    const size_t a = nmat == 2 ? gemm_smem_bytes<MODE_GATE_UP, 64>(meta_bytes, E_total, r)
+                               : gemm_smem_bytes<MODE_DOWN, 64>(meta_bytes, E_total, r);
+    const size_t b = nmat == 2 ? gemm_smem_bytes<MODE_GATE_UP, 128>(meta_bytes, E_total, r)
+                               : gemm_smem_bytes<MODE_DOWN, 128>(meta_bytes, E_total, r);
+    return a > b ? a : b;
 }
 
 int gemm_tile_tokens(int T, int E, int k) { return (long long)T * k <= 64LL * E ? 64 : 128; }
@@ -687,6 +840,7 @@ cudaError_t launch_router_gemm(const uint16_t *x, int T, int H, const float *wr,
     GemmArgs a{};
     a.b_src = x;
     a.ldb = H;
+    a.b_rows = T;
     a.T = T;
     a.E = E;
     a.E_total = 1;
@@ -711,6 +865,14 @@ extern "C" int moe_trace_fetch(unsigned long long *host)
 extern "C" int moe_trace_clear()
 {
     static unsigned long long zero[4 * 16 * moeq4::kTraceSteps];
-    return (int)cudaMemcpyToSymbol(moeq4::g_trace, zero, sizeof(zero));
+    static unsigned long long zero_w[16 * 2];
+    cudaError_t e = cudaMemcpyToSymbol(g_wait_stats, zero_w, sizeof(zero_w));
+    if (e == cudaSuccess)
+        e = cudaMemcpyToSymbol(moeq4::g_trace, zero, sizeof(zero));
+    return (int)e;
+}
+extern "C" int moe_wait_stats_fetch(unsigned long long *host)
+{
+    return (int)cudaMemcpyFromSymbol(host, g_wait_stats, sizeof(g_wait_stats));
 }
 #endif

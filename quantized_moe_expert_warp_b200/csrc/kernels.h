@@ -14,6 +14,7 @@ struct GemmArgs {
     const uint8_t *wmeta;       // scales / super-block headers, kernel layout
     const uint16_t *b_src;      // token rows: x [T, H] (gathered) or h [rows, I]
     int ldb;                    // elements per row of b_src
+    int b_rows;                 // rows of b_src
     const int32_t *sorted_slot; // permutation (gather pass)
     int topk;
     int Tk;                     // T * k: rows at or past Tk belong to the shared expert
@@ -25,6 +26,9 @@ struct GemmArgs {
     int F;                      // 128-row tiles per expert matrix
     int G;                      // int4-sym group size
     int meta_bytes;             // per (expert, tile) meta block
+    int ck_log2;                // k-steps per code chunk (set by the launcher)
+    int ncs_log2;               // code chunks in the ring (set by the launcher)
+    int nmeta_log2;             // meta blocks in the ring (set by the launcher)
     const float *a_f32;         // router pass: fp32 A rows [E, K]
     const float *bias;          // router pass: bias [E] or null
     const float *gate_w;        // router pass: shared-expert gate vector [K] or null

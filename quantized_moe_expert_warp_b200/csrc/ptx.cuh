@@ -68,10 +68,27 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+// A waiting thread sleeps inside try_wait until the phase completes or the
+// suspend-time hint (ns) runs out, so idle warps do not take issue slots from
+// the warps doing work.  0 selects the form without a hint.
+#ifndef MOEQ4_WAIT_HINT_NS
+#define MOEQ4_WAIT_HINT_NS 10000000
+#endif
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity, bool sleep = true)
 {
     uint32_t ok;
-#ifdef MOEQ4_WAIT_HINT_NS
+#if MOEQ4_WAIT_HINT_NS > 0
+    if (!sleep) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        return ok != 0;
+    }
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
@@ -97,24 +114,64 @@ struct WaitCtx {
     volatile int *abort_flag;   // shared memory
     int *status;                // global status words [code, detail] (may be null)
     uint64_t t0;
+#ifdef MOEQ4_TRACE
+    uint32_t polls[16] = {};    // failed polls per call site (instrumented builds)
+    uint32_t waits[16] = {};    // waits per call site that polled more than once
+#endif
 };
 
+// Instrumentation hook: called once per wait that did not complete at the
+// first try, with the call site and the number of further failed polls.
+#ifdef MOEQ4_TRACE
+#define MOEQ4_WAIT_HOOK(where, spins) \
+    do {                              \
+        if (spins) {                  \
+            w.waits[where] += 1;      \
+            w.polls[where] += spins;  \
+        }                             \
+    } while (0)
+#else
+#define MOEQ4_WAIT_HOOK(where, spins) \
+    do {                              \
+    } while (0)
+#endif
+
+// Call sites (bit `where`) that poll without the suspend-time hint.
+#ifndef MOEQ4_NOHINT_SITES
+#define MOEQ4_NOHINT_SITES 0u
+#endif
+
+// Call sites (bit `where`) whose failed polls back off with __nanosleep.
+#ifndef MOEQ4_BACKOFF_SITES
+#define MOEQ4_BACKOFF_SITES 0u
+#endif
+#ifndef MOEQ4_BACKOFF_NS
+#define MOEQ4_BACKOFF_NS 128
+#endif
+
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: kernels here take well under 10 ms
+// failed try_waits between clock reads: each one may already have slept up to the hint
+constexpr uint32_t kClockEvery = MOEQ4_WAIT_HINT_NS > 0 ? 1u : 64u;
 
 // Wait for the phase of `bar` with parity `parity` to complete.  Returns
 // false (after recording MOE_ERR_TIMEOUT) if the wait budget runs out or
 // another role of this CTA already gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, WaitCtx &w, int where)
 {
-    if (mbar_try_wait(bar, parity))
+    const bool sleep = !((MOEQ4_NOHINT_SITES >> where) & 1u);
+    if (mbar_try_wait(bar, parity, sleep))
         return true;
     uint32_t spins = 0;
     while (true) {
-        if (mbar_try_wait(bar, parity))
+        if (mbar_try_wait(bar, parity, sleep)) {
+            MOEQ4_WAIT_HOOK(where, spins);
             return true;
+        }
         if (lds_volatile_s32(smem_u32((const void *)w.abort_flag)))
             return false;
-        if ((++spins & 63u) == 0) {
+        if ((MOEQ4_BACKOFF_SITES >> where) & 1u)
+            __nanosleep(MOEQ4_BACKOFF_NS);
+        if (++spins % kClockEvery == 0) {
             if (globaltimer_ns() - w.t0 > kWaitLimitNs) {
                 *w.abort_flag = 1;
                 if (w.status && atomicCAS(w.status, 0, MOE_ERR_TIMEOUT) == 0)

@@ -78,6 +78,7 @@ def test_packed_sizes_q4k(L):
     (dict(k=40), mq.MOE_ERR_UNSUPPORTED),
     (dict(E=4, k=5), mq.MOE_ERR_UNSUPPORTED),
     (dict(G=48), mq.MOE_ERR_UNSUPPORTED),
+    (dict(G=96), mq.MOE_ERR_UNSUPPORTED),
     (dict(G=16), mq.MOE_ERR_UNSUPPORTED),
     (dict(wfmt=7), mq.MOE_ERR_UNSUPPORTED),
     (dict(wfmt=mq.WFMT_Q4K, I=384), mq.MOE_ERR_UNSUPPORTED),

@@ -254,6 +254,22 @@ def test_fused_equals_composed_bitwise(dev, cfg):
     assert torch.equal(y.view(torch.int16), fused["y_bf16"].view(torch.int16))
 
 
+@pytest.mark.parametrize("cfg", [SMALL_LAYERS[5], SMALL_LAYERS[3], SMALL_LAYERS[1]], ids=lambda c: c.name)
+@pytest.mark.parametrize("ctas", [1, 3])
+def test_layer_on_few_ctas_is_bitwise_equal(dev, cfg, ctas, monkeypatch):
+    """Each work unit is computed the same way whichever CTA takes it, so a
+    launch on 1 or 3 CTAs (every shared-memory ring wraps many times, and
+    k-step counts that do not divide the ring's chunks meet unit ends) gives
+    the full-grid result bit for bit."""
+    from quantized_moe_expert_warp_b200.host import upload_layer
+    layer = synth.make_layer(cfg)
+    packed = upload_layer(layer, dev)
+    full = run_layer(layer, dev, packed=packed)
+    monkeypatch.setenv("MOEQ4_GRID_CTAS", str(ctas))
+    few = run_layer(layer, dev, packed=packed)
+    assert torch.equal(few["y_bf16"].view(torch.int16), full["y_bf16"].view(torch.int16))
+
+
 def test_layer_is_deterministic(dev):
     from quantized_moe_expert_warp_b200.host import upload_layer
     layer = synth.make_layer(SMALL_LAYERS[1])
