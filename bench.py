@@ -308,6 +308,8 @@ def main():
     counts, offsets, ss, dp = i32(E), i32(E + 1), i32(T * k), i32(T * k)
     pn = mq.moe_permute_workspace_size(T, E, k)
     pws = torch.zeros(pn, dtype=torch.uint8, device=dev)
+    rn = mq.moe_router_workspace_size(cfg, T)
+    rws = torch.zeros(rn, dtype=torch.uint8, device=dev)
     fn = mq.moe_expert_ffn_workspace_size(cfg, T)
     fws = torch.zeros(fn, dtype=torch.uint8, device=dev)
     h = torch.empty((T * k + T, cfg.I), dtype=torch.bfloat16, device=dev)
@@ -315,7 +317,7 @@ def main():
     sh = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     names = ["router_logits", "route", "permute", "gate_up_gemm", "down_gemm", "combine"]
     calls = [
-        lambda: mq.moe_router_logits(packed, x, T, logits, gl, stream),
+        lambda: mq.moe_router_logits(packed, x, T, logits, gl, rws, rn, stream),
         lambda: mq.moe_route(logits, T, E, k, cfg.renorm, ids, tw, stream),
         lambda: mq.moe_permute(ids, T, E, k, counts, offsets, ss, dp, pws, pn, stream),
         lambda: mq.moe_expert_gate_up_q4(packed, x, T, ss, offsets, h, fws, fn, stream),

@@ -144,14 +144,21 @@ int moe_dequant_export(const moe_config_t *cfg, const void *q, const void *meta,
 
 /* ------------------------------------------------------------ the steps */
 
+/* Workspace bytes of moe_router_logits for up to T tokens. */
+size_t moe_router_workspace_size(const moe_config_t *cfg, int T);
+
 /*
  * Router logits and the shared expert's gate logit.
  *   x [T, H] bf16, logits [T, E] fp32 (bias added when L->router_bias),
  *   gate_logit [T] fp32 = x . shared_gate (may be NULL; ignored without a
- *   shared expert).  fp32 accumulation.
+ *   shared expert).  fp32 accumulation.  For small T the reduction over H
+ *   is cut into slices that run on separate SMs; their partial logits live
+ *   in the caller's workspace ws (at least moe_router_workspace_size bytes,
+ *   256-byte aligned; MOE_ERR_WORKSPACE if smaller) and are summed in slice
+ *   order.
  */
-int moe_router_logits(const moe_layer_t *L, const uint16_t *x, int T, float *logits, float *gate_logit,
-                      void *stream);
+int moe_router_logits(const moe_layer_t *L, const uint16_t *x, int T, float *logits, float *gate_logit, void *ws,
+                      size_t ws_bytes, void *stream);
 
 /*
  * Top-k routing, one warp per token.  logits [T, E] fp32 (finite),

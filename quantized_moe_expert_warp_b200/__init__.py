@@ -14,7 +14,7 @@ import os
 
 __all__ = [
     "MoeError", "Config", "lib", "moe_version", "moe_last_error", "moe_packed_sizes", "moe_pack_weights",
-    "moe_dequant_export", "moe_router_logits", "moe_route", "moe_permute_workspace_size", "moe_permute",
+    "moe_dequant_export", "moe_router_workspace_size", "moe_router_logits", "moe_route", "moe_permute_workspace_size", "moe_permute",
     "moe_expert_ffn_workspace_size", "moe_expert_ffn_q4", "moe_combine", "moe_layer_workspace_size",
     "moe_layer_forward", "moe_read_status", "moe_kernel_launches", "moe_expert_gate_up_q4", "moe_expert_down_q4",
     "moe_permute_noalloc", "PackedLayer", "WFMT_INT4_SYM", "WFMT_Q4K", "LIB_PATH",
@@ -84,7 +84,8 @@ def lib():
             "moe_packed_sizes": (i32, [vp, vp, vp, vp, vp]),
             "moe_pack_weights": (i32, [vp] * 10),
             "moe_dequant_export": (i32, [vp, vp, vp, i32, i32, vp, vp, vp]),
-            "moe_router_logits": (i32, [vp, vp, i32, vp, vp, vp]),
+            "moe_router_workspace_size": (C.c_size_t, [vp, i32]),
+            "moe_router_logits": (i32, [vp, vp, i32, vp, vp, vp, C.c_size_t, vp]),
             "moe_route": (i32, [vp, i32, i32, i32, i32, vp, vp, vp]),
             "moe_permute_workspace_size": (sz, [i32, i32, i32]),
             "moe_permute": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]),
@@ -170,9 +171,14 @@ def moe_dequant_export(cfg, q, meta, which, expert, out_f32, out_bf16=None, stre
           _stream(stream))
 
 
-def moe_router_logits(layer: "PackedLayer", x, T, logits, gate_logit=None, stream=None):
-    _call("moe_router_logits", C.byref(layer.c_layer), _ptr(x), T, _ptr(logits), _ptr(gate_logit),
-          _stream(stream))
+def moe_router_workspace_size(cfg, T) -> int:
+    c = Config.of(cfg)
+    return lib().moe_router_workspace_size(C.byref(c), T)
+
+
+def moe_router_logits(layer: "PackedLayer", x, T, logits, gate_logit=None, ws=None, ws_bytes=0, stream=None):
+    _call("moe_router_logits", C.byref(layer.c_layer), _ptr(x), T, _ptr(logits), _ptr(gate_logit), _ptr(ws),
+          ws_bytes, _stream(stream))
 
 
 def moe_route(logits, T, E, k, renorm, topk_ids, topk_w, stream=None):

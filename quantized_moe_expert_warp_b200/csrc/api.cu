@@ -64,10 +64,8 @@ bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// CTAs of the persistent kernels: one per SM.  MOEQ4_GRID_CTAS (1 .. SM
-// count) launches fewer, so that tests can give each CTA many work units
-// and wrap its shared-memory rings on small problems.
-int num_sms()
+// SMs of the current device (148 when it cannot be queried).
+int device_sms()
 {
     static int cache[64] = {0};
     int dev = 0;
@@ -79,13 +77,41 @@ int num_sms()
             n = 148;
         cache[dev] = n;
     }
+    return cache[dev];
+}
+
+// CTAs of the persistent kernels: one per SM.  MOEQ4_GRID_CTAS (1 .. SM
+// count) launches fewer, so that tests can give each CTA many work units
+// and wrap its shared-memory rings on small problems.  Work decomposition
+// (tile sizes, router K slices) never depends on it.
+int num_sms()
+{
+    const int n = device_sms();
     const char *env = getenv("MOEQ4_GRID_CTAS");
     if (env) {
         const int g = atoi(env);
-        if (g >= 1 && g < cache[dev])
+        if (g >= 1 && g < n)
             return g;
     }
-    return cache[dev];
+    return n;
+}
+
+// Router K slices and the bytes of their partial logits (0 without a split).
+int router_slices(const moe_config_t *c, int T) { return router_ksplit(T, c->E, c->H, device_sms()); }
+
+// Bytes of the partial logits for any token count up to T (the slice count
+// falls as T grows, so the largest need can come before T; it is taken at
+// the ends of the 128-token steps where the slice count changes).
+size_t router_part_bytes(const moe_config_t *c, int T)
+{
+    size_t best = 0;
+    for (int t = 128; t < T + 128; t += 128) {
+        const int tt = t < T ? t : T;
+        const int s = router_slices(c, tt);
+        const size_t b = s > 1 ? sizeof(float) * (size_t)s * tt * c->E : 0;
+        best = b > best ? b : best;
+    }
+    return best;
 }
 
 int check_config(const moe_config_t *c)
@@ -138,7 +164,7 @@ FfnWs ffn_layout(const moe_config_t *c, int T, uint8_t *base)
 
 struct LayerWs {
     int *status;
-    float *logits, *gate_logit, *w;
+    float *logits, *gate_logit, *w, *router_part;
     int32_t *ids, *counts, *offsets, *sorted_slot, *dest_pos;
     void *perm_scratch;
     uint8_t *ffn;
@@ -158,6 +184,7 @@ LayerWs layer_layout(const moe_config_t *c, int T, uint8_t *base)
     };
     w.status = (int *)take(256);
     w.logits = (float *)take(sizeof(float) * (size_t)T * c->E);
+    w.router_part = (float *)take(router_part_bytes(c, T));
     w.gate_logit = (float *)take(sizeof(float) * (size_t)T);
     w.ids = (int32_t *)take(sizeof(int32_t) * Tk);
     w.w = (float *)take(sizeof(float) * Tk);
@@ -323,12 +350,24 @@ int moe_dequant_export(const moe_config_t *cfg, const void *q, const void *meta,
     return ok();
 }
 
-int moe_router_logits(const moe_layer_t *L, const uint16_t *x, int T, float *logits, float *gate_logit, void *stream)
+size_t moe_router_workspace_size(const moe_config_t *cfg, int T)
+{
+    if (!cfg || T < 0 || check_config(cfg))
+        return 0;
+    return align256(router_part_bytes(cfg, T)) + 256;
+}
+
+int moe_router_logits(const moe_layer_t *L, const uint16_t *x, int T, float *logits, float *gate_logit, void *ws,
+                      size_t ws_bytes, void *stream)
 {
     int rc = check_layer(L);
     if (rc)
         return rc;
     REQUIRE(T >= 0, "T must be >= 0");
+    const size_t need = moe_router_workspace_size(&L->cfg, T);
+    if (!ws || ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "router workspace: need %zu bytes, got %zu", need, ws ? ws_bytes : (size_t)0);
+    REQUIRE_PTR(ws);
     if (T == 0)
         return ok();
     REQUIRE_PTR(x);
@@ -336,10 +375,17 @@ int moe_router_logits(const moe_layer_t *L, const uint16_t *x, int T, float *log
     const float *g = L->cfg.has_shared && gate_logit ? L->shared_gate : nullptr;
     if (g)
         REQUIRE_PTR(gate_logit);
-    CUDA_TRY(launch_router_gemm(x, T, L->cfg.H, L->router_w, L->router_bias, L->cfg.E, g, logits,
-                                g ? gate_logit : nullptr, nullptr, num_sms(), (cudaStream_t)stream),
+    cudaStream_t st = (cudaStream_t)stream;
+    const int S = router_slices(&L->cfg, T);
+    float *part = S > 1 ? (float *)ws : logits;
+    CUDA_TRY(launch_router_gemm(x, T, L->cfg.H, L->router_w, L->router_bias, L->cfg.E, g, part,
+                                g ? gate_logit : nullptr, S, nullptr, num_sms(), st),
              "router logits");
     g_launches += 1;
+    if (S > 1) {
+        CUDA_TRY(launch_router_reduce(part, S, T, L->cfg.E, L->router_bias, logits, st), "router reduce");
+        g_launches += 1;
+    }
     return ok();
 }
 
@@ -548,8 +594,9 @@ int moe_layer_forward(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *
         REQUIRE_PTR(dbg->override_w);
     }
     const float *g = c.has_shared ? L->shared_gate : nullptr;
-    CUDA_TRY(launch_router_gemm(x, T, c.H, L->router_w, L->router_bias, c.E, g, w.logits, g ? w.gate_logit : nullptr,
-                                w.status, num_sms(), st),
+    const int S = router_slices(&c, T);
+    CUDA_TRY(launch_router_gemm(x, T, c.H, L->router_w, L->router_bias, c.E, g, S > 1 ? w.router_part : w.logits,
+                                g ? w.gate_logit : nullptr, S, w.status, num_sms(), st),
              "router logits");
     g_launches += 1;
     const int32_t *ids = w.ids;
@@ -557,8 +604,15 @@ int moe_layer_forward(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *
     if (override_route) {
         ids = dbg->override_ids;
         tw = dbg->override_w;
+        if (S > 1) {
+            CUDA_TRY(launch_router_reduce(w.router_part, S, T, c.E, L->router_bias, w.logits, st), "router reduce");
+            g_launches += 1;
+        }
     } else {
-        CUDA_TRY(launch_route(w.logits, T, c.E, c.k, c.renorm, w.ids, w.w, st), "route");
+        // with split-K partials the route kernel sums them (and writes the logits)
+        CUDA_TRY(launch_route(w.logits, T, c.E, c.k, c.renorm, w.ids, w.w, st, S > 1 ? w.router_part : nullptr, S,
+                              L->router_bias, w.logits),
+                 "route");
         g_launches += 1;
     }
     CUDA_TRY(launch_permute(ids, T, c.E, c.k, w.counts, w.offsets, w.sorted_slot, w.dest_pos, w.perm_scratch,

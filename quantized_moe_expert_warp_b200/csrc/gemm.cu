@@ -123,6 +123,7 @@ struct Barriers {
 
 struct Unit {
     int e, f, row0, nvalid, nmma;
+    int split, ks0, nks;   // K slice of the unit (router split-K; otherwise the whole K)
 };
 
 struct Sched {
@@ -135,6 +136,14 @@ template <int BN>
 __device__ __forceinline__ Unit decode_unit(int u, const GemmArgs &p, const Sched &sc)
 {
     Unit r;
+    const int ks_all = p.K / kKStep;
+    r.split = 0;
+    if (p.ksplit > 1) {
+        r.split = u % p.ksplit;
+        u /= p.ksplit;
+    }
+    r.nks = ks_all / p.ksplit;
+    r.ks0 = r.split * r.nks;
     const int tile = u / p.F;
     r.f = u - tile * p.F;
     int lo = 0, hi = p.E_total - 1;   // largest e with tile_start[e] <= tile (a non-empty expert)
@@ -274,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    const int total_units = s_tile_start[p.E_total] * p.F;
+    const int total_units = s_tile_start[p.E_total] * p.F * p.ksplit;
     const int KS = p.K / kKStep;
     WaitCtx wc{&bars->abort_flag, p.status, globaltimer_ns()};
 
@@ -296,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                 src[i] = p.b_src + (size_t)srow * p.ldb;
                 bytes[i] = r < un.nvalid ? 16u : 0u;
             }
-            for (int ks = 0; ks < KS; ++ks, ++step) {
+            for (int ks = un.ks0; ks < un.ks0 + un.nks; ++ks, ++step) {
                 const int s = step % L::kBStages;
                 if (step >= L::kBStages && !mbar_wait(&bars->b_empty[s], ((step / L::kBStages) & 1) ^ 1, wc, 1)) {
                     ok = false;
@@ -334,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                     break;
                 tc_fence_after();
             }
-            for (int ks = 0; ks < KS; ++ks, ++step) {
+            for (int ks = 0; ks < un.nks; ++ks, ++step) {
                 const int sa = step % kAStages, sb = step % L::kBStages;
                 // every lane polls the same barriers, so the outcome is warp-uniform
                 if (!mbar_wait(&bars->a_full[sa], (step / kAStages) & 1, wc, 3) ||
@@ -502,21 +511,25 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
             const uint8_t *meta = sMeta + mb * meta_al;
             float4 pre[8];                                // router: this row's next k-step, prefetched
             const float *wrow = nullptr;
+            int kbeg = 0, kend = KS;                      // k-steps of the unit
             if (MODE == MODE_ROUTER) {
                 const Unit un = decode_unit<BN>(u, p, sched);
+                kbeg = un.ks0;
+                kend = un.ks0 + un.nks;
                 const int e = un.f * kTileRows + r;
                 wrow = e < p.E ? p.a_f32 + (size_t)e * p.K + c0 * 32 : nullptr;
-                const int ks0 = ((grp - step) % L::kGroups + L::kGroups) % L::kGroups;   // first k-step of this group
-                if (ks0 >= KS)
+                // first k-step of this group in the unit
+                const int kfirst = kbeg + ((grp - step) % L::kGroups + L::kGroups) % L::kGroups;
+                if (kfirst >= kend)
                     wrow = nullptr;
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    pre[i] = wrow ? *(const float4 *)(wrow + ks0 * kKStep + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    pre[i] = wrow ? *(const float4 *)(wrow + kfirst * kKStep + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
             } else if (!mbar_wait(&bars->meta_full[mb], (munit >> p.nmeta_log2) & 1, wc, 8)) {
                 break;
             }
             const int ngroups = WFMT == MOE_WFMT_Q4K ? p.K / 256 : p.K >> gshift;
-            for (int ks = 0; ks < KS; ++ks, ++step) {
+            for (int ks = kbeg; ks < kend; ++ks, ++step) {
                 // every dequant warp frees every code chunk once, after its own
                 // k-steps in the chunk (it may have none)
                 const bool chunk_last = MODE != MODE_ROUTER && (((ks + 1) & (CK - 1)) == 0 || ks + 1 == KS);
@@ -540,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                         v[4 * i + 2] = pre[i].z;
                         v[4 * i + 3] = pre[i].w;
                     }
-                    if (wrow && ks + L::kGroups < KS) {
+                    if (wrow && ks + L::kGroups < kend) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             pre[i] = *(const float4 *)(wrow + (ks + L::kGroups) * kKStep + 4 * i);
@@ -670,13 +683,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                     released = true;
                 }
                 if (MODE == MODE_ROUTER) {
+                    // split-K: one partial [T, E] per K slice, the bias is added when they are summed
                     if (col < p.E) {
-                        const float b = p.bias ? p.bias[col] : 0.f;
+                        const float b = p.ksplit == 1 && p.bias ? p.bias[col] : 0.f;
+                        float *out = p.out_f32 + (size_t)un.split * p.T * p.E;
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int n = n0 + j;
                             if (n < un.nvalid)
-                                p.out_f32[(size_t)(un.row0 + n) * p.E + col] = __uint_as_float(g[j]) + b;
+                                out[(size_t)(un.row0 + n) * p.E + col] = __uint_as_float(g[j]) + b;
                         }
                     }
                 } else {
@@ -786,6 +801,8 @@ static cudaError_t launch_one(const GemmArgs &a_in, int num_sms, cudaStream_t st
 {
     auto kern = grouped_gemm_kernel<MODE, WFMT, BN>;
     GemmArgs a = a_in;
+    if (a.ksplit < 1)
+        a.ksplit = 1;
     const Rings r = gemm_rings<MODE, BN>(a.meta_bytes, a.E_total, a.K / kKStep);
     a.ck_log2 = r.ck_log2;
     a.ncs_log2 = r.ncs_log2;
@@ -811,6 +828,18 @@ size_t gemm_smem_required(int nmat, int meta_bytes, int E_total)
     return a > b ? a : b;
 }
 
+// K slices of the router GEMM: enough work units (128 experts x 128 tokens x
+// K slice) to cover the SMs, at most 32 slices, each a whole number of k-steps.
+int router_ksplit(int T, int E, int H, int sms)
+{
+    const int units = ((E + kTileRows - 1) / kTileRows) * ((T + 127) / 128);
+    const int ks = H / kKStep;
+    int s = 1;
+    while (2 * s <= 32 && ks % (2 * s) == 0 && units * 2 * s <= sms)
+        s *= 2;
+    return s;
+}
+
 int gemm_tile_tokens(int T, int E, int k) { return (long long)T * k <= 64LL * E ? 64 : 128; }
 
 template <int MODE, int BN>
@@ -832,8 +861,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int tile_
 // Router logits on tensor cores: logits[t, e] = x[t] . Wr[e] (+ bias[e]),
 // and gate_out[t] = x[t] . g when g is given.
 cudaError_t launch_router_gemm(const uint16_t *x, int T, int H, const float *wr, const float *bias, int E,
-                               const float *gate_w, float *logits, float *gate_out, int *status, int num_sms,
-                               cudaStream_t st)
+                               const float *gate_w, float *logits, float *gate_out, int ksplit, int *status,
+                               int num_sms, cudaStream_t st)
 {
     if (T == 0)
         return cudaSuccess;
@@ -851,6 +880,7 @@ cudaError_t launch_router_gemm(const uint16_t *x, int T, int H, const float *wr,
     a.gate_w = gate_w;
     a.gate_out = gate_out;
     a.out_f32 = logits;
+    a.ksplit = ksplit;
     a.status = status;
     return launch_one<MODE_ROUTER, 0, 128>(a, num_sms, st);
 }

@@ -23,6 +23,7 @@ struct GemmArgs {
     int T;                      // tokens (rows of the shared expert)
     int E_total;                // E (+ 1 with a shared expert)
     int K;                      // reduction length (H for gate/up, I for down)
+    int ksplit;                 // router: K slices (partials out_f32 + slice * T * E); 1 otherwise
     int F;                      // 128-row tiles per expert matrix
     int G;                      // int4-sym group size
     int meta_bytes;             // per (expert, tile) meta block
@@ -47,10 +48,18 @@ cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int tile_
 size_t gemm_smem_required(int nmat, int meta_bytes, int E_total);
 
 cudaError_t launch_router_gemm(const uint16_t *x, int T, int H, const float *wr, const float *bias, int E,
-                               const float *gate_w, float *logits, float *gate_out, int *status, int num_sms,
-                               cudaStream_t st);
+                               const float *gate_w, float *logits, float *gate_out, int ksplit, int *status,
+                               int num_sms, cudaStream_t st);
+int router_ksplit(int T, int E, int H, int sms);
+// Top-k routing on logits [T, E], or on the sum of `nsplit` partials
+// part[s][T][E] (summed in slice order, bias added last); with partials the
+// summed logits are also written to `logits` when it is not null.
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
-                         cudaStream_t st);
+                         cudaStream_t st, const float *part = nullptr, int nsplit = 1, const float *bias = nullptr,
+                         float *logits_out = nullptr);
+// logits = sum of the partials in slice order + bias (same order as launch_route)
+cudaError_t launch_router_reduce(const float *part, int nsplit, int T, int E, const float *bias, float *logits,
+                                 cudaStream_t st);
 
 size_t permute_scratch_bytes(int T, int E, int k);
 cudaError_t launch_permute(const int32_t *ids, int T, int E, int k, int32_t *counts, int32_t *offsets,

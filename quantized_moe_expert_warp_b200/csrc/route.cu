@@ -21,20 +21,48 @@ __device__ __forceinline__ bool better(float v, int id, float bv, int bid)
     return v > bv || (v == bv && id < bid);
 }
 
+// Router logit of (t, e) from split-K partials: slices summed in order,
+// then the bias.  Shared by the route and reduce kernels so that both give
+// the same bits.
+__device__ __forceinline__ float sum_partials(const float *__restrict__ part, int nsplit, size_t TE, size_t idx,
+                                              const float *__restrict__ bias, int e)
+{
+    float acc = part[idx];
+    for (int s = 1; s < nsplit; ++s)
+        acc += part[(size_t)s * TE + idx];
+    return bias ? acc + bias[e] : acc;
+}
+
 template <int NPL>
 __global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ logits, int T, int E, int k,
-                                                    int renorm, int32_t *ids, float *w)
+                                                    int renorm, int32_t *ids, float *w,
+                                                    const float *__restrict__ part, int nsplit,
+                                                    const float *__restrict__ bias, float *logits_out)
 {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
     const int lane = threadIdx.x % 32;
     if (warp >= T)
         return;
-    const float *L = logits + (size_t)warp * E;
     float v[NPL];
+    if (part) {
+        const size_t TE = (size_t)T * E;
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-        const int e = i * 32 + lane;
-        v[i] = e < E ? L[e] : -CUDART_INF_F;
+        for (int i = 0; i < NPL; ++i) {
+            const int e = i * 32 + lane;
+            v[i] = -CUDART_INF_F;
+            if (e < E) {
+                v[i] = sum_partials(part, nsplit, TE, (size_t)warp * E + e, bias, e);
+                if (logits_out)
+                    logits_out[(size_t)warp * E + e] = v[i];
+            }
+        }
+    } else {
+        const float *L = logits + (size_t)warp * E;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = i * 32 + lane;
+            v[i] = e < E ? L[e] : -CUDART_INF_F;
+        }
     }
     uint32_t taken = 0;
     float top = 0.f, my_val = 0.f;
@@ -93,24 +121,45 @@ __global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ lo
 }
 
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
-                         cudaStream_t st)
+                         cudaStream_t st, const float *part, int nsplit, const float *bias, float *logits_out)
 {
     if (T == 0)
         return cudaSuccess;
     const int blocks = (T + 7) / 8;
     const int npl = (E + 31) / 32;
+#define ROUTE_ARGS logits, T, E, k, renorm, ids, w, part, nsplit, bias, logits_out
     if (npl <= 1)
-        route_kernel<1><<<blocks, 256, 0, st>>>(logits, T, E, k, renorm, ids, w);
+        route_kernel<1><<<blocks, 256, 0, st>>>(ROUTE_ARGS);
     else if (npl <= 2)
-        route_kernel<2><<<blocks, 256, 0, st>>>(logits, T, E, k, renorm, ids, w);
+        route_kernel<2><<<blocks, 256, 0, st>>>(ROUTE_ARGS);
     else if (npl <= 4)
-        route_kernel<4><<<blocks, 256, 0, st>>>(logits, T, E, k, renorm, ids, w);
+        route_kernel<4><<<blocks, 256, 0, st>>>(ROUTE_ARGS);
     else if (npl <= 8)
-        route_kernel<8><<<blocks, 256, 0, st>>>(logits, T, E, k, renorm, ids, w);
+        route_kernel<8><<<blocks, 256, 0, st>>>(ROUTE_ARGS);
     else if (npl <= 16)
-        route_kernel<16><<<blocks, 256, 0, st>>>(logits, T, E, k, renorm, ids, w);
+        route_kernel<16><<<blocks, 256, 0, st>>>(ROUTE_ARGS);
     else
-        route_kernel<32><<<blocks, 256, 0, st>>>(logits, T, E, k, renorm, ids, w);
+        route_kernel<32><<<blocks, 256, 0, st>>>(ROUTE_ARGS);
+#undef ROUTE_ARGS
+    return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(256) router_reduce_kernel(const float *__restrict__ part, int nsplit, int T, int E,
+                                                            const float *__restrict__ bias, float *logits)
+{
+    const size_t TE = (size_t)T * E;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < TE; i += (size_t)gridDim.x * blockDim.x)
+        logits[i] = sum_partials(part, nsplit, TE, i, bias, (int)(i % E));
+}
+
+cudaError_t launch_router_reduce(const float *part, int nsplit, int T, int E, const float *bias, float *logits,
+                                 cudaStream_t st)
+{
+    const size_t TE = (size_t)T * E;
+    if (TE == 0)
+        return cudaSuccess;
+    const int blocks = (int)((TE + 255) / 256 < 4096 ? (TE + 255) / 256 : 4096);
+    router_reduce_kernel<<<blocks, 256, 0, st>>>(part, nsplit, T, E, bias, logits);
     return cudaGetLastError();
 }
 

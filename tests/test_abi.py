@@ -28,7 +28,7 @@ def declared_functions():
 def test_header_declares_the_path():
     names = declared_functions()
     for n in ["moe_route", "moe_permute", "moe_expert_ffn_q4", "moe_combine", "moe_layer_forward",
-              "moe_router_logits", "moe_pack_weights", "moe_layer_workspace_size", "moe_read_status"]:
+              "moe_router_logits", "moe_router_workspace_size", "moe_pack_weights", "moe_layer_workspace_size", "moe_read_status"]:
         assert n in names
 
 
@@ -118,6 +118,11 @@ def test_workspace_too_small_is_reported(L):
     assert rc == mq.MOE_ERR_WORKSPACE
     layer = mq.Layer(cfg(), 0x1000, None, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000)
     rc = L.moe_layer_forward(C.byref(layer), 0x1000, 512, 0x1000, 0x1000, 1024, None, None)
+    assert rc == mq.MOE_ERR_WORKSPACE
+    # the router's split-K partials: several MB at T = 512
+    rneed = L.moe_router_workspace_size(C.byref(cfg()), 512)
+    assert rneed >= 8 * 512 * 256 * 4
+    rc = L.moe_router_logits(C.byref(layer), 0x1000, 512, 0x1000, None, 0x1000, rneed - 16, None)
     assert rc == mq.MOE_ERR_WORKSPACE
 
 

@@ -165,16 +165,20 @@ def test_combine(dev, T, H, k, shared):
 
 # ---------------------------------------------------------- router logits
 
-def test_router_logits_close(dev):
+@pytest.mark.parametrize("T", [1, 200, 600])
+def test_router_logits_close(dev, T):
+    """T = 1 and 200 split the reduction over H into 32 slices, T = 600 into 8."""
     import quantized_moe_expert_warp_b200 as mq
     from quantized_moe_expert_warp_b200.host import upload_layer, x_to_device
-    cfg = synth.get_config("a3b_t512").with_T(200, "router_check").with_(zipf_s=1.1)
+    cfg = synth.get_config("a3b_t512").with_T(T, "router_check").with_(zipf_s=1.1)
     layer = synth.make_layer(cfg, experts=[])
     packed = upload_layer(layer, dev)
     x = x_to_device(layer["x"], dev)
     logits = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=dev)
     gl = torch.empty((cfg.T,), dtype=torch.float32, device=dev)
-    mq.moe_router_logits(packed, x, cfg.T, logits, gl)
+    rn = mq.moe_router_workspace_size(cfg, cfg.T)
+    rws = torch.zeros(rn, dtype=torch.uint8, device=dev)
+    mq.moe_router_logits(packed, x, cfg.T, logits, gl, rws, rn)
     ref = oracle.router_logits(layer["x"], layer["router_w"], layer["router_bias"])
     # bf16 x is exact; fp32 weights enter as two bf16 parts (16 significand bits) with exact products,
     # summed by the tensor cores' fp32 accumulation (truncating adds over
@@ -238,7 +242,9 @@ def test_fused_equals_composed_bitwise(dev, cfg):
     logits, gl = e32(T, E), e32(T)
     ids, w = i32(T, k), e32(T, k)
     counts, offsets, ss, dp = i32(E), i32(E + 1), i32(T * k), i32(T * k)
-    mq.moe_router_logits(packed, x, T, logits, gl)
+    rn = mq.moe_router_workspace_size(cfg, T)
+    rws = torch.zeros(rn, dtype=torch.uint8, device=dev)
+    mq.moe_router_logits(packed, x, T, logits, gl, rws, rn)
     mq.moe_route(logits, T, E, k, cfg.renorm, ids, w)
     n = mq.moe_permute_workspace_size(T, E, k)
     pws = torch.zeros(n, dtype=torch.uint8, device=dev)
