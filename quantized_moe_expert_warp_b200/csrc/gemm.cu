@@ -36,6 +36,31 @@
 #ifdef MOEQ4_TRACE
 // per wait site, summed over warps: [0] waits that polled more than once, [1] failed polls
 __device__ unsigned long long g_wait_stats[16][2];
+// cycle accounting of the first CTAs: per warp, clock cycles by pipeline phase
+__device__ unsigned long long g_cyc[4][24][8];
+#define CYC_DECL                                   \
+    unsigned long long cyc_[8] = {0, 0, 0, 0, 0, 0, 0, 0}; \
+    long long cyc_t_ = clock64();
+#define CYC(b)                                     \
+    do {                                           \
+        const long long n_ = clock64();            \
+        cyc_[(b)] += (unsigned long long)(n_ - cyc_t_); \
+        cyc_t_ = n_;                               \
+    } while (0)
+#define CYC_FLUSH                                                       \
+    do {                                                                \
+        if (blockIdx.x < 4 && lane == 0)                                \
+            for (int i_ = 0; i_ < 8; ++i_)                              \
+                g_cyc[blockIdx.x][warp][i_] = cyc_[i_];                 \
+    } while (0)
+#else
+#define CYC_DECL
+#define CYC(b) \
+    do {       \
+    } while (0)
+#define CYC_FLUSH \
+    do {          \
+    } while (0)
 #endif
 
 #include "dequant.cuh"
@@ -286,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
     const int total_units = s_tile_start[p.E_total] * p.F * p.ksplit;
     const int KS = p.K / kKStep;
     WaitCtx wc{&bars->abort_flag, p.status, globaltimer_ns()};
+    CYC_DECL
 
     if (warp == 0) {
         // ------------------------------------------------ B producer (cp.async row gather)
@@ -305,12 +331,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                 src[i] = p.b_src + (size_t)srow * p.ldb;
                 bytes[i] = r < un.nvalid ? 16u : 0u;
             }
+            CYC(2);
             for (int ks = un.ks0; ks < un.ks0 + un.nks; ++ks, ++step) {
                 const int s = step % L::kBStages;
                 if (step >= L::kBStages && !mbar_wait(&bars->b_empty[s], ((step / L::kBStages) & 1) ^ 1, wc, 1)) {
                     ok = false;
                     break;
                 }
+                CYC(0);
                 const uint32_t base = smem_u32(sB + s * kBN * 128);
 #pragma unroll
                 for (int i = 0; i < kBN / 32; ++i) {
@@ -325,6 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                 }
                 // this lane's copies for the stage arrive on b_full[s] when they land
                 cp_async_arrive_noinc(&bars->b_full[s]);
+                CYC(1);
                 if (lane == 0)
                     TRACE_OTHER(0, step);
             }
@@ -338,19 +367,26 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
             const uint32_t idesc = idesc_bf16_f32(128, un.nmma);
             const int ab = uidx % L::kAccBufs;
             const uint32_t acc = tmem + ab * L::kNAcc * kBN;
+            CYC(4);
             if (uidx >= L::kAccBufs) {
                 if (!mbar_wait(&bars->acc_empty[ab], ((uidx / L::kAccBufs) & 1) ^ 1, wc, 2))
                     break;
                 tc_fence_after();
             }
+            CYC(0);
             for (int ks = 0; ks < un.nks; ++ks, ++step) {
                 const int sa = step % kAStages, sb = step % L::kBStages;
                 // every lane polls the same barriers, so the outcome is warp-uniform
-                if (!mbar_wait(&bars->a_full[sa], (step / kAStages) & 1, wc, 3) ||
-                    !mbar_wait(&bars->b_full[sb], (step / L::kBStages) & 1, wc, 4)) {
+                if (!mbar_wait(&bars->a_full[sa], (step / kAStages) & 1, wc, 3)) {
                     ok = false;
                     break;
                 }
+                CYC(1);
+                if (!mbar_wait(&bars->b_full[sb], (step / L::kBStages) & 1, wc, 4)) {
+                    ok = false;
+                    break;
+                }
+                CYC(2);
                 if (lane == 0)
                     TRACE_OTHER(9, step);
                 tc_fence_after();
@@ -376,6 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                     mma_commit(&bars->b_empty[sb]);
                 }
                 __syncwarp();
+                CYC(3);
                 if (lane == 0)
                     TRACE_OTHER(5, step);
             }
@@ -528,6 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
             } else if (!mbar_wait(&bars->meta_full[mb], (munit >> p.nmeta_log2) & 1, wc, 8)) {
                 break;
             }
+            CYC(7);
             const int ngroups = WFMT == MOE_WFMT_Q4K ? p.K / 256 : p.K >> gshift;
             for (int ks = kbeg; ks < kend; ++ks, ++step) {
                 // every dequant warp frees every code chunk once, after its own
@@ -543,6 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                 }
                 const int sa = step % kAStages;
                 const uint32_t a_col = tmem + lane_off + L::kAccCols + sa * L::kNA * 32;
+                CYC(6);
                 if (MODE == MODE_ROUTER) {
                     uint32_t words[L::kNA][16];
                     float v[32];
@@ -578,6 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                         ok = false;
                         break;
                     }
+                    CYC(0);
 #ifdef MOEQ4_TRACE_WARPS
                     if (lane == 0)
                         TRACE_EVENT((warp - 4) * 2, step);
@@ -607,6 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                             }
                         }
                         if (h == 0) {
+                            CYC(1);
                             if (lane == 0 && warp == 4)
                                 TRACE_EVENT(11, step);
                             // the MMAs that read this TMEM stage kAStages k-steps ago have finished
@@ -618,10 +659,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                             if (lane == 0 && warp == 4)
                                 TRACE_OTHER(12, step);
                             tc_fence_after();
+                            CYC(2);
                         }
 #pragma unroll
                         for (int m = 0; m < L::kNA; ++m)
                             tmem_st16(a_col + m * 32 + c * 16, words[m]);
+                        CYC(h == 0 ? 3 : 4);
                     }
                     if (!ok)
                         break;
@@ -632,6 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                     }
                 }
                 tmem_wait_st();
+                CYC(5);
                 if (lane == 0 && warp == 4)
                     TRACE_OTHER(13, step);
                 tc_fence_before();
@@ -658,8 +702,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
         for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++uidx) {
             const Unit un = decode_unit<BN>(u, p, sched);
             const int ab = uidx % L::kAccBufs;
+            CYC(1);
             if (!mbar_wait(&bars->acc_full[ab], (uidx / L::kAccBufs) & 1, wc, 11))
                 break;
+            CYC(0);
             tc_fence_after();
             if (lane == 0 && warp == 4 + kDeqWarps)
                 TRACE_OTHER(6, uidx);
@@ -734,6 +780,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
         }
     }
 
+    CYC(7);
+    CYC_FLUSH;
 #ifdef MOEQ4_TRACE
     if (lane == 0) {
 #pragma unroll
@@ -900,6 +948,10 @@ extern "C" int moe_trace_clear()
     if (e == cudaSuccess)
         e = cudaMemcpyToSymbol(moeq4::g_trace, zero, sizeof(zero));
     return (int)e;
+}
+extern "C" int moe_cyc_fetch(unsigned long long *host)
+{
+    return (int)cudaMemcpyFromSymbol(host, g_cyc, sizeof(g_cyc));
 }
 extern "C" int moe_wait_stats_fetch(unsigned long long *host)
 {

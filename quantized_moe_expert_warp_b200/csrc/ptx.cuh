@@ -156,8 +156,72 @@ constexpr uint32_t kClockEvery = MOEQ4_WAIT_HINT_NS > 0 ? 1u : 64u;
 // Wait for the phase of `bar` with parity `parity` to complete.  Returns
 // false (after recording MOE_ERR_TIMEOUT) if the wait budget runs out or
 // another role of this CTA already gave up.
+// Non-blocking probe of a phase.
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Polling policy.  Mode 0 (default) polls with try_wait and its suspend-time
+// hint.  Mode 1 probes with test_wait and sleeps between probes for a time
+// that doubles up to a cap (short on the critical path of a k-step, call
+// sites 3, 4, 9, 10; longer elsewhere); it frees issue slots but wakes
+// later, and measured slower on these kernels.
+#ifndef MOEQ4_WAIT_MODE
+#define MOEQ4_WAIT_MODE 0   // 0: try_wait loop (suspend-time hint); 1: test_wait with sleeping back-off
+#endif
+#ifndef MOEQ4_NS_CRIT
+#define MOEQ4_NS_CRIT 32
+#endif
+#ifndef MOEQ4_NS_CRIT_MAX
+#define MOEQ4_NS_CRIT_MAX 128
+#endif
+#ifndef MOEQ4_NS_BG
+#define MOEQ4_NS_BG 128
+#endif
+#ifndef MOEQ4_NS_BG_MAX
+#define MOEQ4_NS_BG_MAX 1024
+#endif
+
+__device__ __forceinline__ constexpr bool wait_site_critical(int where)
+{
+    return where == 3 || where == 4 || where == 9 || where == 10;
+}
+
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, WaitCtx &w, int where)
 {
+#if MOEQ4_WAIT_MODE == 1
+    if (mbar_test(bar, parity))
+        return true;
+    const bool crit = wait_site_critical(where);
+    uint32_t ns = crit ? MOEQ4_NS_CRIT : MOEQ4_NS_BG;
+    const uint32_t ns_max = crit ? MOEQ4_NS_CRIT_MAX : MOEQ4_NS_BG_MAX;
+    uint32_t spins = 0;
+    while (true) {
+        __nanosleep(ns);
+        if (mbar_test(bar, parity)) {
+            MOEQ4_WAIT_HOOK(where, spins);
+            return true;
+        }
+        if (lds_volatile_s32(smem_u32((const void *)w.abort_flag)))
+            return false;
+        ns = ns * 2 < ns_max ? ns * 2 : ns_max;
+        if ((++spins & 15u) == 0 && globaltimer_ns() - w.t0 > kWaitLimitNs) {
+            *w.abort_flag = 1;
+            if (w.status && atomicCAS(w.status, 0, MOE_ERR_TIMEOUT) == 0)
+                w.status[1] = where;
+            return false;
+        }
+    }
+#else
     const bool sleep = !((MOEQ4_NOHINT_SITES >> where) & 1u);
     if (mbar_try_wait(bar, parity, sleep))
         return true;
@@ -180,6 +244,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, WaitCt
             }
         }
     }
+#endif
 }
 
 // One lane of a converged warp waits; the whole warp gets the result.
