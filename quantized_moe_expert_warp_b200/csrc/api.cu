@@ -432,7 +432,7 @@ int moe_permute(const int32_t *topk_ids, int T, int E, int k, int32_t *counts, i
     CUDA_TRY(launch_permute(topk_ids, T, E, k, counts, offsets, sorted_slot, dest_pos, (uint8_t *)ws + 256,
                             (int *)ws, (cudaStream_t)stream),
              "permute");
-    g_launches += T > 0 ? 2 : 0;
+    g_launches += permute_launch_count(T, k);
     return ok();
 }
 
@@ -455,7 +455,7 @@ int moe_permute_noalloc(const int32_t *topk_ids, int T, int E, int k, int32_t *c
     }
     CUDA_TRY(launch_permute_noalloc(topk_ids, T, E, k, counts, offsets, sorted_slot, dest_pos, (cudaStream_t)stream),
              "moe_permute_noalloc");
-    g_launches += T > 0 ? 2 : 0;
+    g_launches += permute_launch_count(T, k);
     return ok();
 }
 
@@ -618,7 +618,7 @@ int moe_layer_forward(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *
     CUDA_TRY(launch_permute(ids, T, c.E, c.k, w.counts, w.offsets, w.sorted_slot, w.dest_pos, w.perm_scratch,
                             w.status, st),
              "permute");
-    g_launches += 2;
+    g_launches += permute_launch_count(T, c.k);
     rc = run_expert_ffn(L, x, T, w.sorted_slot, w.offsets, w.y_perm, c.has_shared ? w.shared_out : nullptr, w.ffn,
                         w.status, st);
     if (rc)

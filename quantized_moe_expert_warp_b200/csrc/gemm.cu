@@ -877,13 +877,17 @@ size_t gemm_smem_required(int nmat, int meta_bytes, int E_total)
 }
 
 // K slices of the router GEMM: enough work units (128 experts x 128 tokens x
-// K slice) to cover the SMs, at most 32 slices, each a whole number of k-steps.
+// K slice) to cover the SMs, at most 32 slices, each a whole number of
+// k-steps, and at most 4 MB of partial logits (they are written and read
+// back once more).
 int router_ksplit(int T, int E, int H, int sms)
 {
     const int units = ((E + kTileRows - 1) / kTileRows) * ((T + 127) / 128);
     const int ks = H / kKStep;
+    const size_t part_cap = (size_t)4 << 20;
     int s = 1;
-    while (2 * s <= 32 && ks % (2 * s) == 0 && units * 2 * s <= sms)
+    while (2 * s <= 32 && ks % (2 * s) == 0 && units * 2 * s <= sms &&
+           (size_t)2 * s * T * E * sizeof(float) <= part_cap)
         s *= 2;
     return s;
 }

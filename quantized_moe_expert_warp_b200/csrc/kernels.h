@@ -62,6 +62,7 @@ cudaError_t launch_router_reduce(const float *part, int nsplit, int T, int E, co
                                  cudaStream_t st);
 
 size_t permute_scratch_bytes(int T, int E, int k);
+int permute_launch_count(int T, int k);   // kernels launch_permute runs
 cudaError_t launch_permute(const int32_t *ids, int T, int E, int k, int32_t *counts, int32_t *offsets,
                            int32_t *sorted_slot, int32_t *dest_pos, void *scratch, int *status, cudaStream_t st);
 

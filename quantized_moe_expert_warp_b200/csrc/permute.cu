@@ -54,26 +54,25 @@ __global__ void __launch_bounds__(kPermThreads) permute_hist_kernel(const int32_
         hist[(size_t)blockIdx.x * E + e] = s_hist[e];
 }
 
-__global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(const int32_t *__restrict__ ids, int S, int E,
-                                                                       int chunk, const int32_t *__restrict__ hist,
-                                                                       int32_t *counts, int32_t *offsets,
-                                                                       int32_t *sorted_slot, int32_t *dest_pos)
+// Ranks and scatters slots [c_begin, c_end) (one CTA's chunk).  tot_e / pre_e
+// give expert e's total count and the count in earlier chunks (thread e < E
+// calls them); CTA `writer` also writes counts and offsets.
+template <typename Tot, typename Pre>
+__device__ __forceinline__ void permute_rank_scatter(const int32_t *__restrict__ ids, int c_begin, int c_end, int E,
+                                                     Tot tot_e, Pre pre_e, bool writer, int32_t *counts,
+                                                     int32_t *offsets, int32_t *sorted_slot, int32_t *dest_pos,
+                                                     int32_t *s_mem)
 {
-    extern __shared__ int32_t s_mem[];
     int32_t *s_base = s_mem;                                  // [E] next position of each expert in this chunk
     int32_t *s_scan = s_mem + E;                              // [kPermThreads] scan scratch
     uint16_t *s_wcnt = (uint16_t *)(s_scan + kPermThreads);   // [32 warps][E]
-    const int nblk = gridDim.x, b = blockIdx.x;
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
 
     // expert totals, this chunk's prefix, and the exclusive scan over experts
     int tot = 0, pre = 0;
     if (tid < E) {
-        for (int bb = 0; bb < nblk; ++bb) {
-            const int h = hist[(size_t)bb * E + tid];
-            tot += h;
-            pre += bb < b ? h : 0;
-        }
+        tot = tot_e(tid);
+        pre = pre_e(tid);
     }
     s_scan[tid] = tot;
     __syncthreads();
@@ -86,22 +85,21 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(const int
     if (tid < E) {
         const int off_e = s_scan[tid] - tot;
         s_base[tid] = off_e + pre;
-        if (b == 0) {
+        if (writer) {
             counts[tid] = tot;
             offsets[tid] = off_e;
         }
     }
-    if (b == 0 && tid == 0)
+    if (writer && tid == 0)
         offsets[E] = s_scan[kPermThreads - 1];
     for (int i = tid; i < 32 * E; i += kPermThreads)
         s_wcnt[i] = 0;
     __syncthreads();
 
-    const int c1 = min(S, (b + 1) * chunk);
-    for (int c0 = b * chunk; c0 < c1; c0 += kPermThreads) {
+    for (int c0 = c_begin; c0 < c_end; c0 += kPermThreads) {
         const int s = c0 + tid;
         int e = -1;
-        if (s < c1) {
+        if (s < c_end) {
             e = ids[s];
             if (e < 0 || e >= E)
                 e = -1;
@@ -117,7 +115,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(const int
                 rank += s_wcnt[w * E + e];
             sorted_slot[rank] = s;
             dest_pos[s] = rank;
-        } else if (s < c1) {
+        } else if (s < c_end) {
             dest_pos[s] = -1;
         }
         __syncthreads();
@@ -134,6 +132,57 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(const int
     }
 }
 
+__global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(const int32_t *__restrict__ ids, int S, int E,
+                                                                       int chunk, const int32_t *__restrict__ hist,
+                                                                       int32_t *counts, int32_t *offsets,
+                                                                       int32_t *sorted_slot, int32_t *dest_pos)
+{
+    extern __shared__ int32_t s_mem[];
+    const int nblk = gridDim.x, b = blockIdx.x;
+    auto tot_e = [&](int e) {
+        int t = 0;
+        for (int bb = 0; bb < nblk; ++bb)
+            t += hist[(size_t)bb * E + e];
+        return t;
+    };
+    auto pre_e = [&](int e) {
+        int t = 0;
+        for (int bb = 0; bb < b; ++bb)
+            t += hist[(size_t)bb * E + e];
+        return t;
+    };
+    permute_rank_scatter(ids, b * chunk, min(S, (b + 1) * chunk), E, tot_e, pre_e, b == 0, counts, offsets,
+                         sorted_slot, dest_pos, s_mem);
+}
+
+// Small problems (up to two 1024-slot passes): histogram, scan and scatter in
+// one CTA and one launch.  Larger ones spread the slots over several CTAs.
+constexpr int kPermSingleMax = 2048;
+
+__global__ void __launch_bounds__(kPermThreads) permute_single_kernel(const int32_t *__restrict__ ids, int S, int E,
+                                                                      int32_t *counts, int32_t *offsets,
+                                                                      int32_t *sorted_slot, int32_t *dest_pos,
+                                                                      int *status)
+{
+    extern __shared__ int32_t s_mem[];
+    int32_t *s_hist = s_mem + E + kPermThreads + (32 * E + 1) / 2;   // [E], after the scatter's scratch
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        s_hist[e] = 0;
+    __syncthreads();
+    for (int s = threadIdx.x; s < S; s += blockDim.x) {
+        const int e = ids[s];
+        if (e >= 0 && e < E)
+            atomicAdd(&s_hist[e], 1);
+        else
+            record_error(status, MOE_ERR_INVALID_ARG, s);
+    }
+    __syncthreads();
+    permute_rank_scatter(ids, 0, S, E, [&](int e) { return s_hist[e]; }, [](int) { return 0; }, true, counts,
+                         offsets, sorted_slot, dest_pos, s_mem);
+}
+
+int permute_launch_count(int T, int k) { return T * k == 0 ? 0 : (T * k <= kPermSingleMax ? 1 : 2); }
+
 cudaError_t launch_permute(const int32_t *ids, int T, int E, int k, int32_t *counts, int32_t *offsets,
                            int32_t *sorted_slot, int32_t *dest_pos, void *scratch, int *status, cudaStream_t st)
 {
@@ -143,6 +192,19 @@ cudaError_t launch_permute(const int32_t *ids, int T, int E, int k, int32_t *cou
         if (e == cudaSuccess)
             e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st);
         return e;
+    }
+    if (S <= kPermSingleMax) {
+        const size_t smem1 = (E + kPermThreads) * sizeof(int32_t) + ((32 * E + 1) / 2) * sizeof(int32_t) +
+                             E * sizeof(int32_t);
+        if (smem1 > 48 * 1024) {
+            const cudaError_t e1 =
+                cudaFuncSetAttribute(permute_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+            if (e1 != cudaSuccess)
+                return e1;
+        }
+        permute_single_kernel<<<1, kPermThreads, smem1, st>>>(ids, S, E, counts, offsets, sorted_slot, dest_pos,
+                                                               status);
+        return cudaGetLastError();
     }
     const int chunk = perm_chunk(S);
     const int nblk = perm_blocks(S);

@@ -34,7 +34,7 @@ __device__ __forceinline__ float sum_partials(const float *__restrict__ part, in
 }
 
 template <int NPL>
-__global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ logits, int T, int E, int k,
+__global__ void __launch_bounds__(128) route_kernel(const float *__restrict__ logits, int T, int E, int k,
                                                     int renorm, int32_t *ids, float *w,
                                                     const float *__restrict__ part, int nsplit,
                                                     const float *__restrict__ bias, float *logits_out)
@@ -45,15 +45,35 @@ __global__ void __launch_bounds__(256) route_kernel(const float *__restrict__ lo
         return;
     float v[NPL];
     if (part) {
+        // the same order as sum_partials: slice 0, 1, ..., then the bias;
+        // all of a slice's loads are issued together
         const size_t TE = (size_t)T * E;
+        const float *row = part + (size_t)warp * E;
 #pragma unroll
         for (int i = 0; i < NPL; ++i) {
             const int e = i * 32 + lane;
-            v[i] = -CUDART_INF_F;
+            v[i] = e < E ? row[e] : 0.f;
+        }
+#pragma unroll 2
+        for (int sl = 1; sl < nsplit; ++sl) {
+            const float *r = row + (size_t)sl * TE;
+#pragma unroll
+            for (int i = 0; i < NPL; ++i) {
+                const int e = i * 32 + lane;
+                if (e < E)
+                    v[i] += r[e];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = i * 32 + lane;
             if (e < E) {
-                v[i] = sum_partials(part, nsplit, TE, (size_t)warp * E + e, bias, e);
+                if (bias)
+                    v[i] += bias[e];
                 if (logits_out)
                     logits_out[(size_t)warp * E + e] = v[i];
+            } else {
+                v[i] = -CUDART_INF_F;
             }
         }
     } else {
@@ -125,21 +145,21 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
 {
     if (T == 0)
         return cudaSuccess;
-    const int blocks = (T + 7) / 8;
+    const int blocks = (T + 3) / 4;   // four tokens (warps) per block: more SMs share the partial reads
     const int npl = (E + 31) / 32;
 #define ROUTE_ARGS logits, T, E, k, renorm, ids, w, part, nsplit, bias, logits_out
     if (npl <= 1)
-        route_kernel<1><<<blocks, 256, 0, st>>>(ROUTE_ARGS);
+        route_kernel<1><<<blocks, 128, 0, st>>>(ROUTE_ARGS);
     else if (npl <= 2)
-        route_kernel<2><<<blocks, 256, 0, st>>>(ROUTE_ARGS);
+        route_kernel<2><<<blocks, 128, 0, st>>>(ROUTE_ARGS);
     else if (npl <= 4)
-        route_kernel<4><<<blocks, 256, 0, st>>>(ROUTE_ARGS);
+        route_kernel<4><<<blocks, 128, 0, st>>>(ROUTE_ARGS);
     else if (npl <= 8)
-        route_kernel<8><<<blocks, 256, 0, st>>>(ROUTE_ARGS);
+        route_kernel<8><<<blocks, 128, 0, st>>>(ROUTE_ARGS);
     else if (npl <= 16)
-        route_kernel<16><<<blocks, 256, 0, st>>>(ROUTE_ARGS);
+        route_kernel<16><<<blocks, 128, 0, st>>>(ROUTE_ARGS);
     else
-        route_kernel<32><<<blocks, 256, 0, st>>>(ROUTE_ARGS);
+        route_kernel<32><<<blocks, 128, 0, st>>>(ROUTE_ARGS);
 #undef ROUTE_ARGS
     return cudaGetLastError();
 }
