@@ -37,9 +37,9 @@
 // per wait site, summed over warps: [0] waits that polled more than once, [1] failed polls
 __device__ unsigned long long g_wait_stats[16][2];
 // cycle accounting of the first CTAs: per warp, clock cycles by pipeline phase
-__device__ unsigned long long g_cyc[4][24][8];
+__device__ unsigned long long g_cyc[4][24][12];
 #define CYC_DECL                                   \
-    unsigned long long cyc_[8] = {0, 0, 0, 0, 0, 0, 0, 0}; \
+    unsigned long long cyc_[12] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0}; \
     long long cyc_t_ = clock64();
 #define CYC(b)                                     \
     do {                                           \
@@ -50,7 +50,7 @@ __device__ unsigned long long g_cyc[4][24][8];
 #define CYC_FLUSH                                                       \
     do {                                                                \
         if (blockIdx.x < 4 && lane == 0)                                \
-            for (int i_ = 0; i_ < 8; ++i_)                              \
+            for (int i_ = 0; i_ < 12; ++i_)                             \
                 g_cyc[blockIdx.x][warp][i_] = cyc_[i_];                 \
     } while (0)
 #else
@@ -567,18 +567,16 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
             }
             CYC(7);
             const int ngroups = WFMT == MOE_WFMT_Q4K ? p.K / 256 : p.K >> gshift;
-            for (int ks = kbeg; ks < kend; ++ks, ++step) {
-                // every dequant warp frees every code chunk once, after its own
-                // k-steps in the chunk (it may have none)
-                const bool chunk_last = MODE != MODE_ROUTER && (((ks + 1) & (CK - 1)) == 0 || ks + 1 == KS);
-                if (step % L::kGroups != grp) {
-                    if (chunk_last) {
-                        __syncwarp();
-                        if (lane == 0)
-                            mbar_arrive(&bars->code_empty[(cbase + (ks >> p.ck_log2)) & (NCS - 1)]);
-                    }
-                    continue;
-                }
+            // This warp's k-steps of the unit: those with step % kGroups == grp.
+            // Every dequant warp frees every code chunk of the unit exactly
+            // once: right after its last k-step in the chunk, or, for chunks
+            // where it has none, as it passes them.
+            const int step0 = step;                       // global step of k-step kbeg
+            const int nchunks = MODE == MODE_ROUTER ? 0 : (KS + CK - 1) >> p.ck_log2;
+            int released = 0;                             // chunks of this unit already freed
+            for (int ks = kbeg + ((grp - step0) % L::kGroups + L::kGroups) % L::kGroups; ks < kend;
+                 ks += L::kGroups) {
+                step = step0 + (ks - kbeg);
                 const int sa = step % kAStages;
                 const uint32_t a_col = tmem + lane_off + L::kAccCols + sa * L::kNA * 32;
                 CYC(6);
@@ -609,8 +607,19 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                     for (int m = 0; m < L::kNA; ++m)
                         tmem_st16(a_col + m * 32 + c0 * 16, words[m]);
                 } else {
-                    const int cidx = cbase + (ks >> p.ck_log2);
+                    const int my_chunk = ks >> p.ck_log2;
+                    const int cidx = cbase + my_chunk;
                     const int sc = cidx & (NCS - 1);
+                    // chunks passed without a k-step of this warp are freed before it
+                    // waits for a later one (a warp never holds one chunk while
+                    // waiting for another)
+                    if (my_chunk > released) {
+                        __syncwarp();
+                        if (lane == 0)
+                            for (int cc = released; cc < my_chunk; ++cc)
+                                mbar_arrive(&bars->code_empty[(cbase + cc) & (NCS - 1)]);
+                        released = my_chunk;
+                    }
                     if (lane == 0 && warp == 4)
                         TRACE_OTHER(15, step);
                     if (!mbar_wait(&bars->code_full[sc], (cidx >> p.ncs_log2) & 1, wc, 9)) {
@@ -668,11 +677,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                     }
                     if (!ok)
                         break;
-                    if (chunk_last) {
+                    // after its last k-step in the chunk the warp frees it
+                    const int chunk_end = min((my_chunk + 1) << p.ck_log2, KS);
+                    if (ks + L::kGroups >= chunk_end) {
                         __syncwarp();
                         if (lane == 0)
                             mbar_arrive(&bars->code_empty[sc]);
+                        released = my_chunk + 1;
                     }
+                    CYC(11);
                 }
                 tmem_wait_st();
                 CYC(5);
@@ -680,17 +693,26 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                     TRACE_OTHER(13, step);
                 tc_fence_before();
                 __syncwarp();
+                CYC(9);
                 if (lane == 0)
                     mbar_arrive(&bars->a_full[sa]);
+                __syncwarp();
+                CYC(10);
                 if (lane == 0 && warp == 4)
                     TRACE_OTHER(3, step);
                 if (lane == 0 && warp == 7)
                     TRACE_OTHER(4, step);
             }
+            if (!ok)
+                break;
+            step = step0 + (kend - kbeg);
             if (MODE != MODE_ROUTER) {
                 __syncwarp();
-                if (lane == 0)
+                if (lane == 0) {
+                    for (int cc = released; cc < nchunks; ++cc)
+                        mbar_arrive(&bars->code_empty[(cbase + cc) & (NCS - 1)]);
                     mbar_arrive(&bars->meta_empty[mb]);
+                }
             }
             cbase += (KS + CK - 1) >> p.ck_log2;
         }
