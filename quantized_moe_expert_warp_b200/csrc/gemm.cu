@@ -98,7 +98,10 @@ constexpr int kMaxMetaBufs = 4;
 constexpr int kEpiTok = 16;  // tokens per epilogue chunk
 constexpr int kEpiStride = 80;                                   // bytes per staged token row (64 + pad)
 constexpr int kEpiBytes = 4 * kEpiTok * kEpiStride;              // staging for the four epilogue warps
-constexpr int kDeqWarps = 16;                  // dequant warps (warps 4 .. 19)
+#ifndef MOEQ4_DEQ_WARPS
+#define MOEQ4_DEQ_WARPS 16
+#endif
+constexpr int kDeqWarps = MOEQ4_DEQ_WARPS;     // dequant warps (warps 4 .. 3 + kDeqWarps), a multiple of 8
 constexpr int kThreads = (8 + kDeqWarps) * 32;
 
 enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_ROUTER = 2 };
@@ -113,10 +116,14 @@ struct Geo {
     // with two, the epilogue of one tile overlaps the MMAs of the next
     static constexpr int kAccBufs = (512 - kAStages * kNA * 32) / (kNAcc_ * BN) >= 2 ? 2 : 1;
     static constexpr int kNCode = MODE == MODE_GATE_UP ? 2 : MODE == MODE_DOWN ? 1 : 0; // code matrices
-    // dequant warp groups: four groups of four warps, each warp a full k-step
-    // of its 32 rows (router: two groups of eight, one half each)
-    static constexpr int kGroups = MODE == MODE_ROUTER ? 2 : 4;
-    static constexpr int kGroupWarps = kDeqWarps / kGroups;
+    // dequant warp groups: groups of four warps, each warp a full k-step of
+    // its 32 rows, or groups of eight, each warp one half of a k-step (the
+    // router, and any warp count that would give more groups than TMEM A
+    // stages: a group must not reuse a stage whose previous MMAs it has not
+    // waited for, so that no mbarrier waiter runs two phases ahead)
+    static constexpr int kGroupWarps = MODE == MODE_ROUTER || kDeqWarps / 4 > kAStages ? 8 : 4;
+    static constexpr int kGroups = kDeqWarps / kGroupWarps;
+    static_assert(kGroups <= kAStages, "dequant groups must not outnumber the TMEM A stages");
     static constexpr int kHalves = kGroupWarps == 8 ? 1 : 2;
     static constexpr int kCodeBlock = kNCode ? code_block_bytes(kNCode) : 0;
     // the gathered token rows wait on L2 / HBM latency, so their shared-memory
