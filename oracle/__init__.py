@@ -26,6 +26,7 @@ _lib = None
 
 WFMT_INT4_SYM = 0
 WFMT_Q4K = 1
+WFMT_INT4_ASYM = 2
 
 
 def build(force: bool = False) -> str:
@@ -60,6 +61,7 @@ def lib():
             i64, vp = C.c_int64, C.c_void_p
             L.oracle_dequant_int4sym.argtypes = [vp, vp, i64, i64, i64, vp]
             L.oracle_dequant_q4k.argtypes = [vp, i64, i64, vp]
+            L.oracle_dequant_int4asym.argtypes = [vp, vp, i64, i64, i64, vp]
             L.oracle_router_logits.argtypes = [vp, i64, i64, vp, vp, i64, vp]
             L.oracle_route.argtypes = [vp, i64, i64, i64, C.c_int, vp, vp, vp]
             L.oracle_permute.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp]
@@ -88,6 +90,14 @@ def dequant_int4sym(nib, scale, N, K, G) -> np.ndarray:
     nib, scale = _c(nib, np.uint8), _c(scale, np.uint16)
     out = np.empty((N, K), np.float32)
     _check(lib().oracle_dequant_int4sym(_p(nib), _p(scale), N, K, G, _p(out)), "dequant_int4sym")
+    return out
+
+
+def dequant_int4asym(nib, sm, N, K, G) -> np.ndarray:
+    """sm: uint16 [N, K/G, 2] bf16 (scale, min) pairs."""
+    nib, sm = _c(nib, np.uint8), _c(sm, np.uint16)
+    out = np.empty((N, K), np.float32)
+    _check(lib().oracle_dequant_int4asym(_p(nib), _p(sm), N, K, G, _p(out)), "dequant_int4asym")
     return out
 
 
@@ -170,7 +180,7 @@ def layer_forward(layer: dict, sample=None, override_ids=None, override_w=None):
     A.router_w = arr("wr", layer["router_w"], np.float32)
     A.router_bias = arr("rb", layer.get("router_bias"), np.float32)
     A.shared_gate = arr("sg", layer.get("shared_gate"), np.float32)
-    if cfg.wfmt == WFMT_INT4_SYM:
+    if cfg.wfmt in (WFMT_INT4_SYM, WFMT_INT4_ASYM):
         A.gu_q = arr("guq", layer["gu_nib"], np.uint8)
         A.gu_scale = arr("gus", layer["gu_scale"], np.uint16)
         A.dn_q = arr("dnq", layer["dn_nib"], np.uint8)

@@ -37,7 +37,7 @@
 #define ORACLE_EINVAL (-1)
 #define ORACLE_ENOMEM (-2)
 
-enum { WFMT_INT4_SYM = 0, WFMT_Q4K = 1 };
+enum { WFMT_INT4_SYM = 0, WFMT_Q4K = 1, WFMT_INT4_ASYM = 2 };
 
 /* ---------------------------------------------------------------- scalars */
 
@@ -84,6 +84,29 @@ int oracle_dequant_int4sym(const uint8_t *nib, const uint16_t *scale, int64_t N,
             int q = u >= 8 ? u - 16 : u;
             double s = bf16_value(scale[n * (K / G) + k / G]);
             out[n * K + k] = (float)(q * s);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * Asymmetric int4 (the mq4r file's experts, hipfire 0.4.3 benchmarks,
+ * "Read this before comparing columns"; reading: one bf16 scale s and one
+ * bf16 minimum m per G weights along K, unsigned 4-bit q, as in the GGUF
+ * Q4_1 family).  sm holds the pairs (s, m) per group: [N, K/G, 2].
+ * w[n][k] = q * s + m, formed exactly in fp64 and rounded once to fp32.
+ */
+int oracle_dequant_int4asym(const uint8_t *nib, const uint16_t *sm, int64_t N, int64_t K, int64_t G,
+                            float *out)
+{
+    if (!nib || !sm || !out || N < 0 || K <= 0 || G <= 0 || K % G || K % 2)
+        return ORACLE_EINVAL;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t byte = nib[n * (K / 2) + k / 2];
+            int q = (k & 1) ? (byte >> 4) : (byte & 0xF);
+            const uint16_t *p = sm + (n * (K / G) + k / G) * 2;
+            out[n * K + k] = (float)(q * bf16_value(p[0]) + bf16_value(p[1]));
         }
     }
     return ORACLE_OK;
@@ -315,9 +338,9 @@ typedef struct {
     const float *router_bias;    /* [E] or NULL */
     const float *shared_gate;    /* [H] (has_shared) */
     const uint8_t *gu_q;         /* int4: nib [Et, 2I, H/2]; Q4K: [Et, 2I, H/256*144] */
-    const uint16_t *gu_scale;    /* int4: [Et, 2I, H/G]; Q4K: NULL */
+    const uint16_t *gu_scale;    /* int4-sym: [Et, 2I, H/G]; int4-asym: [Et, 2I, H/G, 2]; Q4K: NULL */
     const uint8_t *dn_q;         /* int4: nib [Et, H, I/2]; Q4K: [Et, H, I/256*144] */
-    const uint16_t *dn_scale;    /* int4: [Et, H, I/G]; Q4K: NULL */
+    const uint16_t *dn_scale;    /* int4-sym: [Et, H, I/G]; int4-asym: [Et, H, I/G, 2]; Q4K: NULL */
     const int32_t *override_ids; /* optional [T, k]: routing to use instead of the oracle's */
     const float *override_w;     /* optional [T, k] (with override_ids) */
     const int32_t *sample;       /* tokens whose output rows are computed; NULL = all */
@@ -345,6 +368,14 @@ static int dequant_expert(const oracle_layer_args *A, int64_t e, float *wgu, flo
         return oracle_dequant_int4sym(A->dn_q + e * H * (I / 2), A->dn_scale + e * H * (I / A->G), H,
                                       I, A->G, wdn);
     }
+    if (A->wfmt == WFMT_INT4_ASYM) {
+        int rc = oracle_dequant_int4asym(A->gu_q + e * (2 * I) * (H / 2),
+                                         A->gu_scale + e * (2 * I) * (H / A->G) * 2, 2 * I, H, A->G, wgu);
+        if (rc)
+            return rc;
+        return oracle_dequant_int4asym(A->dn_q + e * H * (I / 2), A->dn_scale + e * H * (I / A->G) * 2, H,
+                                       I, A->G, wdn);
+    }
     if (A->wfmt == WFMT_Q4K) {
         int rc = oracle_dequant_q4k(A->gu_q + e * (2 * I) * (H / 256 * 144), 2 * I, H, wgu);
         if (rc)
@@ -369,7 +400,7 @@ int oracle_layer_forward(const oracle_layer_args *A)
     const int64_t T = A->T, H = A->H, E = A->E, k = A->k, I = A->I;
     if (T < 0 || H <= 0 || E <= 0 || k <= 0 || k > E || I <= 0)
         return ORACLE_EINVAL;
-    if (A->wfmt == WFMT_INT4_SYM && (!A->gu_scale || !A->dn_scale || A->G <= 0))
+    if ((A->wfmt == WFMT_INT4_SYM || A->wfmt == WFMT_INT4_ASYM) && (!A->gu_scale || !A->dn_scale || A->G <= 0))
         return ORACLE_EINVAL;
     if (A->has_shared && !A->shared_gate)
         return ORACLE_EINVAL;

@@ -50,6 +50,7 @@ GENERATOR_VERSION = 3
 
 WFMT_INT4_SYM = 0
 WFMT_Q4K = 1
+WFMT_INT4_ASYM = 2
 
 
 @dataclass(frozen=True)
@@ -61,7 +62,7 @@ class LayerConfig:
     k: int            # experts per token
     I: int            # expert intermediate size
     has_shared: bool  # one always-on shared expert of intermediate I
-    wfmt: int         # WFMT_INT4_SYM or WFMT_Q4K
+    wfmt: int         # WFMT_INT4_SYM, WFMT_Q4K or WFMT_INT4_ASYM
     G: int            # int4-sym group size along K (256 for Q4K: super-block)
     wr_std: float     # router weight std
     zipf_s: float     # 0: no router bias; else Zipf exponent of the bias
@@ -101,6 +102,8 @@ CONFIGS = {
     "a3b_t8192_zipf": _a3b("a3b_t8192_zipf", 8192, seed=2, zipf_s=1.1),
     # 4096 tokens, Q4_K-style super-block weights
     "a3b_t4096_q4k": _a3b("a3b_t4096_q4k", 4096, seed=3, wfmt=WFMT_Q4K, G=256),
+    # asymmetric int4 (scale and minimum per group of 128), 512 tokens
+    "a3b_t512_asym": _a3b("a3b_t512_asym", 512, seed=5, wfmt=WFMT_INT4_ASYM),
     # decode-shaped batches
     "a3b_decode_t1": _a3b("a3b_decode_t1", 1, seed=4, x_stream=1),
     "a3b_decode_t8": _a3b("a3b_decode_t8", 8, seed=4, x_stream=8),
@@ -172,6 +175,28 @@ def quantize_int4_sym(w: np.ndarray, G: int):
     u = (q.astype(np.uint8) & 0xF)
     nib = (u[:, 0::2] | (u[:, 1::2] << 4)).astype(np.uint8)
     return nib, s_bits
+
+
+def quantize_int4_asym(w: np.ndarray, G: int):
+    """Asymmetric int4 with one bf16 scale and one bf16 minimum per G weights.
+
+    m = bf16(min w); s = bf16((max w - m) / 15); q = clamp(rint((w - m) / s),
+    0, 15) (q = 0 where s = 0).  Returns (nib uint8 [N, K/2] with unsigned
+    codes, element 2i in the low nibble; sm uint16 [N, K/G, 2] = (s, m)).
+    """
+    N, K = w.shape
+    assert K % G == 0 and K % 2 == 0
+    wg = w.reshape(N, K // G, G).astype(np.float32)
+    m_bits = f32_to_bf16_bits(wg.min(axis=2))
+    m = bf16_bits_to_f32(m_bits)
+    s_bits = f32_to_bf16_bits((wg.max(axis=2) - m) / np.float32(15.0))
+    s = bf16_bits_to_f32(s_bits)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.where(s[:, :, None] > 0, np.rint((wg - m[:, :, None]) / s[:, :, None]), 0.0)
+    u = np.clip(q, 0, 15).astype(np.uint8).reshape(N, K)
+    nib = (u[:, 0::2] | (u[:, 1::2] << 4)).astype(np.uint8)
+    sm = np.stack([s_bits, m_bits], axis=-1).astype(np.uint16)
+    return nib, sm
 
 
 def _pack_6bit_fields(fields: np.ndarray) -> np.ndarray:
@@ -295,6 +320,8 @@ def make_expert(cfg: LayerConfig, e: int):
     wdn = _normal(cfg.seed, _T_DN, e, (H, I), 0.02)
     if cfg.wfmt == WFMT_INT4_SYM:
         return quantize_int4_sym(wgu, cfg.G) + quantize_int4_sym(wdn, cfg.G)
+    if cfg.wfmt == WFMT_INT4_ASYM:
+        return quantize_int4_asym(wgu, cfg.G) + quantize_int4_asym(wdn, cfg.G)
     return (quantize_q4k(wgu), quantize_q4k(wdn))
 
 
@@ -341,6 +368,14 @@ def make_layer(cfg: LayerConfig, experts: Optional[list] = None) -> dict:
         for e, (a, b, c, d) in zip(sel, drawn):
             gu_nib[e], gu_sc[e], dn_nib[e], dn_sc[e] = a, b, c, d
         out.update(gu_nib=gu_nib, gu_scale=gu_sc, dn_nib=dn_nib, dn_scale=dn_sc)
+    elif cfg.wfmt == WFMT_INT4_ASYM:
+        gu_nib = np.zeros((Et, 2 * I, H // 2), np.uint8)
+        gu_sm = np.zeros((Et, 2 * I, H // cfg.G, 2), np.uint16)
+        dn_nib = np.zeros((Et, H, I // 2), np.uint8)
+        dn_sm = np.zeros((Et, H, I // cfg.G, 2), np.uint16)
+        for e, (a, b, c, d) in zip(sel, drawn):
+            gu_nib[e], gu_sm[e], dn_nib[e], dn_sm[e] = a, b, c, d
+        out.update(gu_nib=gu_nib, gu_scale=gu_sm, dn_nib=dn_nib, dn_scale=dn_sm)
     else:
         gu = np.zeros((Et, 2 * I, H // 256 * 144), np.uint8)
         dn = np.zeros((Et, H, I // 256 * 144), np.uint8)

@@ -67,6 +67,57 @@ def test_int4_roundtrip_of_representable_weights():
     assert np.array_equal(oracle.dequant_int4sym(nib, sc, N, K, G), w)
 
 
+def test_int4asym_dequant_hand_built_block():
+    # unsigned codes; per group of 2: (scale, min) = (0.5, -2), (0.25, 1) | (0, 3), (2, -0.5)
+    q = [[0, 15, 1, 7], [3, 0, 8, 2]]
+    nib = pack_nibbles(q)
+    assert nib.tolist() == [[0xF0, 0x71], [0x03, 0x28]]
+    sm = np.array([[[0x3F00, 0xC000], [0x3E80, 0x3F80]],
+                   [[0x0000, 0x4040], [0x4000, 0xBF00]]], np.uint16)
+    w = oracle.dequant_int4asym(nib, sm, 2, 4, 2)
+    assert w.tolist() == [[-2.0, 5.5, 1.25, 2.75], [3.0, 3.0, 15.5, 3.5]]
+
+
+def test_int4asym_with_min_of_minus_eight_scales_is_int4sym():
+    """m = -8 s and unsigned code q + 8 give the symmetric format's q s exactly
+    (-8 s is exact in bf16), for the weights and for a whole layer."""
+    cfg = synth.LayerConfig(name="asym_as_sym", T=11, H=64, E=5, k=2, I=32, has_shared=True,
+                            wfmt=synth.WFMT_INT4_SYM, G=32, wr_std=0.3, zipf_s=0.0, seed=7)
+    sym = synth.make_layer(cfg)
+
+    def to_asym(nib, scale):
+        lo, hi = nib & 0xF, nib >> 4
+        u = (((lo ^ 8) | ((hi ^ 8) << 4))).astype(np.uint8)   # two's complement q -> q + 8
+        s = synth.bf16_bits_to_f32(scale)
+        sm = np.stack([scale, bf16(-8.0 * s)], axis=-1).astype(np.uint16)
+        return u, sm
+
+    asym = dict(sym)
+    asym["cfg"] = cfg.with_(wfmt=synth.WFMT_INT4_ASYM)
+    asym["gu_nib"], asym["gu_scale"] = to_asym(sym["gu_nib"], sym["gu_scale"])
+    asym["dn_nib"], asym["dn_scale"] = to_asym(sym["dn_nib"], sym["dn_scale"])
+    a = oracle.dequant_int4asym(asym["gu_nib"][2], asym["gu_scale"][2], 2 * cfg.I, cfg.H, cfg.G)
+    b = oracle.dequant_int4sym(sym["gu_nib"][2], sym["gu_scale"][2], 2 * cfg.I, cfg.H, cfg.G)
+    assert np.array_equal(a, b)
+    assert np.array_equal(oracle.layer_forward(asym)["y"], oracle.layer_forward(sym)["y"])
+
+
+def test_int4asym_generator_roundtrip():
+    rng = np.random.default_rng(9)
+    N, K, G = 8, 256, 64
+    w = rng.normal(0.0, 0.02, size=(N, K)).astype(np.float32) + rng.normal(0.0, 0.01, size=(N, 1)).astype(np.float32)
+    nib, sm = synth.quantize_int4_asym(w, G)
+    got = oracle.dequant_int4asym(nib, sm, N, K, G)
+    s = np.repeat(synth.bf16_bits_to_f32(sm[..., 0]), G, axis=1)
+    m = np.repeat(synth.bf16_bits_to_f32(sm[..., 1]), G, axis=1)
+    # rounding to the grid (s/2), the bf16 minimum (|m| 2^-9) and the bf16 scale at q <= 15
+    bound = s / 2 + np.abs(m) * 2.0 ** -9 + 15 * s * 2.0 ** -9 + 1e-12
+    assert np.all(np.abs(got - w) <= bound)
+    codes = np.stack([nib & 0xF, nib >> 4], axis=-1).reshape(N, K)
+    cg = codes.reshape(N, K // G, G)
+    assert np.all(cg.min(axis=2) == 0) and np.all(cg.max(axis=2) >= 14)
+
+
 def _q4k_block(d_bits, dmin_bits, sc, m, q):
     """Hand-built 144-byte super-block: fields placed bit by bit."""
     blk = np.zeros(144, np.uint8)
@@ -325,6 +376,9 @@ def _dequant_all(layer):
         if cfg.wfmt == synth.WFMT_INT4_SYM:
             gu.append(oracle.dequant_int4sym(layer["gu_nib"][e], layer["gu_scale"][e], 2 * I, H, cfg.G))
             dn.append(oracle.dequant_int4sym(layer["dn_nib"][e], layer["dn_scale"][e], H, I, cfg.G))
+        elif cfg.wfmt == synth.WFMT_INT4_ASYM:
+            gu.append(oracle.dequant_int4asym(layer["gu_nib"][e], layer["gu_scale"][e], 2 * I, H, cfg.G))
+            dn.append(oracle.dequant_int4asym(layer["dn_nib"][e], layer["dn_scale"][e], H, I, cfg.G))
         else:
             gu.append(oracle.dequant_q4k(layer["gu_q4k"][e], 2 * I, H))
             dn.append(oracle.dequant_q4k(layer["dn_q4k"][e], H, I))
@@ -369,6 +423,7 @@ def dense_reference(layer):
     dict(T=17, H=64, E=8, k=3, I=64, has_shared=True, G=16),
     dict(T=9, H=32, E=5, k=5, I=32, has_shared=True, G=32, renorm=False),
     dict(T=7, H=256, E=4, k=2, I=256, has_shared=True, G=256, wfmt=synth.WFMT_Q4K),
+    dict(T=9, H=64, E=6, k=3, I=64, has_shared=True, G=32, wfmt=synth.WFMT_INT4_ASYM),
 ])
 def test_layer_matches_dense_bruteforce(variant):
     v = dict(wfmt=synth.WFMT_INT4_SYM, wr_std=0.3, zipf_s=0.0, seed=11, renorm=True)
