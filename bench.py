@@ -47,9 +47,13 @@ def expert_bytes(cfg) -> tuple:
         gu = 2 * cfg.I * (cfg.H // 256) * 144
         dn = cfg.H * (cfg.I // 256) * 144
     else:
-        gu = 2 * cfg.I * cfg.H // 2 + 2 * cfg.I * (cfg.H // cfg.G) * 2
-        dn = cfg.H * cfg.I // 2 + cfg.H * (cfg.I // cfg.G) * 2
+        mb = 4 if cfg.wfmt == 2 else 2   # bf16 scale (and minimum for int4-asym) per group
+        gu = 2 * cfg.I * cfg.H // 2 + 2 * cfg.I * (cfg.H // cfg.G) * mb
+        dn = cfg.H * cfg.I // 2 + cfg.H * (cfg.I // cfg.G) * mb
     return gu, dn
+
+
+WFMT_NAMES = {0: "int4-sym", 1: "q4k", 2: "int4-asym"}
 
 
 def kernel_source_hash() -> str:
@@ -353,12 +357,27 @@ def main():
     peak_src = "measured"
     if not hbm_peak:
         hbm_peak, peak_src = 6650.0, "fallback"
-    achieved = alg[dominant] / (per_kernel_ms[dominant] * 1e-3) / 1e9
     tag = {"gate_up_gemm": "gate_up", "down_gemm": "down"}[dominant]
-    roofline = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": ncu_traffic(tag, cfg.name),
-                "algorithmic_bytes_per_launch": alg[dominant], "ms_per_launch": per_kernel_ms[dominant],
-                "peak_source": peak_src}
+    # the kernel's own roofline: the slower of its bytes at HBM peak and its
+    # FLOPs at the bf16 tensor peak (burst figure: each kernel is timed alone)
+    rows = T * cfg.k + (T if cfg.has_shared else 0)
+    flops_k = {"gate_up_gemm": 2.0 * rows * 2 * cfg.I * H, "down_gemm": 2.0 * rows * H * cfg.I}[dominant]
+    tc_peak = peaks.get("bf16_tflops") or 1590.0
+    t_hbm = alg[dominant] / (hbm_peak * 1e9)
+    t_tc = flops_k / (tc_peak * 1e12)
+    secs = per_kernel_ms[dominant] * 1e-3
+    if t_tc > t_hbm:
+        achieved = flops_k / secs / 1e12
+        roofline = {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": tc_peak,
+                    "unit": "TFLOP/s", "frac": achieved / tc_peak, "traffic": ncu_traffic(tag, cfg.name),
+                    "algorithmic_flops_per_launch": flops_k, "algorithmic_bytes_per_launch": alg[dominant],
+                    "ms_per_launch": per_kernel_ms[dominant], "peak_source": peak_src}
+    else:
+        achieved = alg[dominant] / secs / 1e9
+        roofline = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": achieved / hbm_peak, "traffic": ncu_traffic(tag, cfg.name),
+                    "algorithmic_bytes_per_launch": alg[dominant], "ms_per_launch": per_kernel_ms[dominant],
+                    "peak_source": peak_src}
     # whole-layer roofline: max(FLOPs at tensor peak, bytes at HBM peak)
     layer_bytes = touched * (gu_b + dn_b) + E * H * 4 + 4 * T * H
     t_hbm = layer_bytes / (hbm_peak * 1e9)
@@ -409,9 +428,9 @@ def main():
             "metric": "MoE-layer prefill tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded N(0,1) bf16 activations; N(0,0.02) weights, int4-sym quantised)",
+            "data": f"synthetic (seeded N(0,1) bf16 activations; N(0,0.02) weights, {WFMT_NAMES[cfg.wfmt]} quantised)",
             "config": {"workload": cfg.name, "T": T, "H": H, "E": E, "k": k, "I": cfg.I,
-                       "shared_expert": bool(cfg.has_shared), "weights": "int4-sym" if cfg.wfmt == 0 else "q4k",
+                       "shared_expert": bool(cfg.has_shared), "weights": WFMT_NAMES[cfg.wfmt],
                        "G": cfg.G, "tokens_per_rank": T, "parallelism": f"replicas x{world} (token-sharded)",
                        "l2": "inputs larger than L2 (expert weights %.0f MB)" % (packed.weight_bytes() / 1e6)},
             "tflops": tflops, "flop_per_token": fpt,

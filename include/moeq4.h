@@ -55,15 +55,17 @@ extern "C" {
 /* Expert weight formats. */
 #define MOE_WFMT_INT4_SYM 0 /* int4 two's complement, one bf16 scale per G weights along K */
 #define MOE_WFMT_Q4K 1      /* Q4_K-style 256-weight super-blocks (see moe_pack_weights)   */
+#define MOE_WFMT_INT4_ASYM 2 /* unsigned int4, a bf16 scale and a bf16 minimum per G weights */
 
 /* Shapes of one layer.  Admitted: H % 128 == 0, I % 128 == 0, 1 <= k <= E <= 1024,
- * int4-sym: G a power of two, G >= 32, G divides H and I; Q4K: H % 256 == 0, I % 256 == 0. */
+ * int4-sym / int4-asym: G a power of two, G >= 32, G divides H and I; Q4K: H % 256 == 0,
+ * I % 256 == 0. */
 typedef struct moe_config {
     int32_t H;          /* hidden size                                   */
     int32_t I;          /* expert intermediate size (shared expert too)  */
     int32_t E;          /* routed experts                                */
     int32_t k;          /* experts per token                             */
-    int32_t G;          /* int4-sym group size along K (ignored for Q4K) */
+    int32_t G;          /* int4 group size along K (ignored for Q4K)     */
     int32_t has_shared; /* 1: one always-on shared expert                */
     int32_t renorm;     /* 1: renormalise the top-k weights to sum to 1  */
     int32_t wfmt;       /* MOE_WFMT_*                                    */
@@ -124,6 +126,10 @@ int moe_packed_sizes(const moe_config_t *cfg, size_t *gu_q_bytes, size_t *gu_met
  *             sc_0..7 then m_0..7), 128 bytes of unsigned 4-bit q (weight
  *             i in byte i/2, low nibble when i is even);
  *             w = d*sc_j*q - dmin*m_j for sub-block j = i / 32.
+ *   int4-asym: codes uint8 [rows, K/2] (unsigned q, element 2i in the low
+ *             nibble) and, per group, the bf16 pair (scale s, minimum m):
+ *             uint16 [rows, K/G, 2]; w = q*s + m (the pages' asymmetric
+ *             mq4r file; the recipe is this library's reading);
  *   gu_scale / dn_scale are ignored (may be NULL) for Q4K.
  * Outputs go to caller buffers of the sizes moe_packed_sizes() returns.
  * Source: hipfire 0.4.3 benchmarks, "Read this before comparing columns"

@@ -120,13 +120,13 @@ int check_config(const moe_config_t *c)
         return fail(MOE_ERR_INVALID_ARG, "cfg: null pointer");
     if (c->H <= 0 || c->I <= 0 || c->E <= 0 || c->k <= 0)
         return fail(MOE_ERR_INVALID_ARG, "cfg: H, I, E, k must be positive");
-    if (c->wfmt != MOE_WFMT_INT4_SYM && c->wfmt != MOE_WFMT_Q4K)
+    if (c->wfmt != MOE_WFMT_INT4_SYM && c->wfmt != MOE_WFMT_Q4K && c->wfmt != MOE_WFMT_INT4_ASYM)
         return fail(MOE_ERR_UNSUPPORTED, "cfg: unknown weight format %d", c->wfmt);
     if (c->H % 128 || c->I % 128)
         return fail(MOE_ERR_UNSUPPORTED, "cfg: H (%d) and I (%d) must be multiples of 128", c->H, c->I);
     if (c->E > 1024 || c->k > 32 || c->k > c->E)
         return fail(MOE_ERR_UNSUPPORTED, "cfg: need k <= min(E, 32) and E <= 1024 (E=%d k=%d)", c->E, c->k);
-    if (c->wfmt == MOE_WFMT_INT4_SYM) {
+    if (c->wfmt == MOE_WFMT_INT4_SYM || c->wfmt == MOE_WFMT_INT4_ASYM) {
         if (c->G < 32 || (c->G & (c->G - 1)) || c->H % c->G || c->I % c->G)
             return fail(MOE_ERR_UNSUPPORTED, "cfg: int4 group G=%d must be a power of two >= 32 dividing H and I",
                         c->G);
@@ -317,8 +317,8 @@ int moe_pack_weights(const moe_config_t *cfg, const void *gu_canon, const void *
     if (rc)
         return rc;
     REQUIRE(gu_canon && dn_canon, "canonical weights: null pointer");
-    if (cfg->wfmt == MOE_WFMT_INT4_SYM)
-        REQUIRE(gu_scale && dn_scale, "int4-sym scales: null pointer");
+    if (cfg->wfmt == MOE_WFMT_INT4_SYM || cfg->wfmt == MOE_WFMT_INT4_ASYM)
+        REQUIRE(gu_scale && dn_scale, "int4 scales: null pointer");
     REQUIRE_PTR(gu_q);
     REQUIRE_PTR(gu_meta);
     REQUIRE_PTR(dn_q);

@@ -9,9 +9,11 @@
 //          bytes hold K elements ks*64 + c*32 .. +31 of row r of matrix m
 //          as four 32-bit words of 8 elements: element 2i of the word in
 //          nibble i, element 2i+1 in nibble i+4 (i = 0..3).  int4-sym codes
-//          are stored offset-binary (q + 8), Q4K codes as they are (0..15).
+//          are stored offset-binary (q + 8), Q4K and int4-asym codes as they
+//          are (0..15).
 //   meta:  per (expert, tile f) a contiguous block, ordered [m][group][row]:
 //          int4-sym: bf16 scale of group g (K/G groups);
+//          int4-asym: bf16 scale (low half) and bf16 minimum (high half);
 //          Q4K:      the 16-byte super-block header (fp16 d, fp16 dmin,
 //                    12 bytes of 6-bit sc/m fields) of super-block g.
 // One thread owns one row and one 32-element half of a k-step, so reads of
@@ -34,7 +36,9 @@ __host__ __device__ constexpr int code_block_bytes(int nmat) { return nmat * 2 *
 
 __host__ __device__ inline int meta_block_bytes(int nmat, int wfmt, int K, int G)
 {
-    return wfmt == MOE_WFMT_Q4K ? nmat * (K / 256) * kTileRows * 16 : nmat * (K / G) * kTileRows * 2;
+    return wfmt == MOE_WFMT_Q4K        ? nmat * (K / 256) * kTileRows * 16
+           : wfmt == MOE_WFMT_INT4_ASYM ? nmat * (K / G) * kTileRows * 4
+                                        : nmat * (K / G) * kTileRows * 2;
 }
 
 __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b)
@@ -74,6 +78,42 @@ __device__ __forceinline__ void dequant_int4sym_chunk(const uint4 codes, uint16_
             out[wi * 4 + i] = bf16x2_mul(bf16x2_sub(t, off), s2);
         }
     }
+}
+
+__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// int4-asym: 32 unsigned codes and the group's (scale, minimum) pair ->
+// 16 words of bf16 pairs.  (128 + u) - 128 = u exactly; u * s + m is
+// rounded once to bf16 by the fused multiply-add.
+__device__ __forceinline__ void dequant_int4asym_chunk(const uint4 codes, uint32_t scale_min, uint32_t (&out)[16])
+{
+    const uint32_t s2 = __byte_perm(scale_min, 0, 0x1010);   // scale in both halves
+    const uint32_t m2 = __byte_perm(scale_min, 0, 0x3232);   // minimum in both halves
+    const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t t = ((w[wi] >> (4 * i)) & 0x000F000Fu) | 0x43004300u;   // bf16 pair (128+u_lo, 128+u_hi)
+            out[wi * 4 + i] = bf16x2_fma(bf16x2_sub(t, 0x43004300u), s2, m2);
+        }
+    }
+}
+
+__device__ __forceinline__ float int4asym_value(const uint4 codes, uint32_t scale_min, int e)
+{
+    const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+    const int wi = e / 8, j = e % 8;
+    const int nib = (j & 1) ? (j >> 1) + 4 : (j >> 1);
+    const int u = (w[wi] >> (4 * nib)) & 0xF;
+    const float s = __uint_as_float(scale_min << 16);
+    const float m = __uint_as_float(scale_min & 0xFFFF0000u);
+    return fmaf((float)u, s, m);   // u * s is exact in fp32; one rounding
 }
 
 // Exact fp32 values of the same chunk (for export): element e of 0..31.

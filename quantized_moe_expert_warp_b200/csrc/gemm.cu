@@ -656,6 +656,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                                 float dsc, dm;
                                 q4k_subblock_scale(hdr, (kpos % 256) / 32, dsc, dm);
                                 dequant_q4k_chunk(codes, dsc, dm, words[m]);
+                            } else if (WFMT == MOE_WFMT_INT4_ASYM) {
+                                const int g = kpos >> gshift;
+                                const uint32_t sm = lds32(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 4);
+                                dequant_int4asym_chunk(codes, sm, words[m]);
                             } else {
                                 const int g = kpos >> gshift;
                                 const uint16_t sbits = lds16(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 2);
@@ -926,8 +930,9 @@ int gemm_tile_tokens(int T, int E, int k) { return (long long)T * k <= 64LL * E 
 template <int MODE, int BN>
 static cudaError_t launch_fmt(const GemmArgs &a, int wfmt, int num_sms, cudaStream_t st)
 {
-    return wfmt == MOE_WFMT_Q4K ? launch_one<MODE, MOE_WFMT_Q4K, BN>(a, num_sms, st)
-                                : launch_one<MODE, MOE_WFMT_INT4_SYM, BN>(a, num_sms, st);
+    return wfmt == MOE_WFMT_Q4K         ? launch_one<MODE, MOE_WFMT_Q4K, BN>(a, num_sms, st)
+           : wfmt == MOE_WFMT_INT4_ASYM ? launch_one<MODE, MOE_WFMT_INT4_ASYM, BN>(a, num_sms, st)
+                                        : launch_one<MODE, MOE_WFMT_INT4_SYM, BN>(a, num_sms, st);
 }
 
 cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int tile_tokens, int num_sms, cudaStream_t st)

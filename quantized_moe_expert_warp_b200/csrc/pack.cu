@@ -3,8 +3,9 @@
 //
 // Formats: symmetric int4 with one bf16 scale per G weights (hipfire 0.4.3
 // benchmarks, "Read this before comparing columns": the mq4rs file's
-// symmetric experts), and Q4_K-style super-blocks (hipEngine post, "GGUF":
-// Q4_K_S / Q4_K_M).  The pages give neither bit layout; the canonical
+// symmetric experts), asymmetric int4 with a bf16 scale and minimum per G
+// weights (the same table's mq4r file), and Q4_K-style super-blocks
+// (hipEngine post, "GGUF": Q4_K_S / Q4_K_M).  The pages give neither bit layout; the canonical
 // layouts are described in moeq4.h, the kernel layout in dequant.cuh.
 // Packing is a pure byte shuffle (plus the offset-binary flip of int4-sym
 // codes); the load-time "symmetry scan" of the benchmarks page ("Other
@@ -31,7 +32,7 @@ static MatGeom geom(const moe_config_t &c, int which)
     g.KS = g.K / kKStep;
     g.rows_total = g.nmat * g.rows_per_mat;
     g.meta_bytes = meta_block_bytes(g.nmat, c.wfmt, g.K, c.G);
-    g.ngroups = c.wfmt == MOE_WFMT_Q4K ? g.K / 256 : g.K / c.G;
+    g.ngroups = c.wfmt == MOE_WFMT_Q4K ? g.K / 256 : g.K / c.G;   // int4-sym and int4-asym: K / G
     return g;
 }
 
@@ -61,7 +62,7 @@ __global__ void pack_codes_kernel(const uint8_t *__restrict__ canon, uint8_t *__
         src += (size_t)(k0 / 256) * 144 + 16 + (k0 % 256) / 2;
     else
         src += k0 / 2;
-    const uint32_t flip = wfmt == MOE_WFMT_Q4K ? 0u : 8u;
+    const uint32_t flip = wfmt == MOE_WFMT_INT4_SYM ? 8u : 0u;   // int4-sym codes become offset-binary
     uint32_t words[4];
 #pragma unroll
     for (int wi = 0; wi < 4; ++wi) {
@@ -77,7 +78,8 @@ __global__ void pack_codes_kernel(const uint8_t *__restrict__ canon, uint8_t *__
     *(uint4 *)(out + idx * kChunkBytes) = make_uint4(words[0], words[1], words[2], words[3]);
 }
 
-// int4-sym: one thread per bf16 scale; Q4K: one thread per 16-byte header
+// int4-sym: one thread per bf16 scale; int4-asym: per (scale, minimum) pair;
+// Q4K: one thread per 16-byte header
 __global__ void pack_meta_kernel(const uint8_t *__restrict__ canon, const uint16_t *__restrict__ scale,
                                  uint8_t *__restrict__ out, size_t n, int wfmt, int G, MatGeom g)
 {
@@ -99,6 +101,9 @@ __global__ void pack_meta_kernel(const uint8_t *__restrict__ canon, const uint16
             w[i] = (uint32_t)src[4 * i] | ((uint32_t)src[4 * i + 1] << 8) | ((uint32_t)src[4 * i + 2] << 16) |
                    ((uint32_t)src[4 * i + 3] << 24);
         *(uint4 *)(out + idx * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else if (wfmt == MOE_WFMT_INT4_ASYM) {
+        const size_t i = ((e * g.rows_total + row) * (size_t)(g.K / G) + grp) * 2;
+        ((uint32_t *)out)[idx] = (uint32_t)scale[i] | ((uint32_t)scale[i + 1] << 16);
     } else {
         ((uint16_t *)out)[idx] = scale[(e * g.rows_total + row) * (size_t)(g.K / G) + grp];
     }
@@ -151,6 +156,12 @@ __global__ void dequant_export_kernel(const uint8_t *__restrict__ q, const uint8
         dequant_q4k_chunk(codes, dsc, dm, words);
         for (int i = 0; i < 32; ++i)
             vals[i] = q4k_value(codes, dsc, dm, i);
+    } else if (wfmt == MOE_WFMT_INT4_ASYM) {
+        const int grp = kpos / G;
+        const uint32_t sm = *(const uint32_t *)(mb + ((m * g.ngroups + grp) * kTileRows + r) * 4);
+        dequant_int4asym_chunk(codes, sm, words);
+        for (int i = 0; i < 32; ++i)
+            vals[i] = int4asym_value(codes, sm, i);
     } else {
         const int grp = kpos / G;
         const uint16_t sbits = *(const uint16_t *)(mb + ((m * g.ngroups + grp) * kTileRows + r) * 2);

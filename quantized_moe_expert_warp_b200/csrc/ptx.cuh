@@ -30,6 +30,13 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr)
     return v;
 }
 
+__device__ __forceinline__ uint32_t lds32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ uint16_t lds16(uint32_t addr)
 {
     uint16_t v;

@@ -40,6 +40,7 @@ def small_cfg(name, **kw):
     (synth.get_config("tiny_t64"), [0, 7, 15]),
     (small_cfg("g128", H=512, I=256, E=4, G=128, has_shared=True), [0, 4]),
     (small_cfg("q4k", H=512, I=256, E=3, G=256, wfmt=synth.WFMT_Q4K, has_shared=True), [0, 2, 3]),
+    (small_cfg("asym", H=512, I=256, E=3, G=64, wfmt=synth.WFMT_INT4_ASYM, has_shared=True), [0, 3]),
 ])
 def test_dequant_export_bitexact(dev, cfg, experts):
     import quantized_moe_expert_warp_b200 as mq
@@ -59,7 +60,8 @@ def test_dequant_export_bitexact(dev, cfg, experts):
             else:
                 nib = layer["gu_nib"][e] if which == 0 else layer["dn_nib"][e]
                 sc = layer["gu_scale"][e] if which == 0 else layer["dn_scale"][e]
-                ref = oracle.dequant_int4sym(nib, sc, rows, K, cfg.G)
+                dq = oracle.dequant_int4asym if cfg.wfmt == synth.WFMT_INT4_ASYM else oracle.dequant_int4sym
+                ref = dq(nib, sc, rows, K, cfg.G)
             got = f32.cpu().numpy()
             assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), (e, which)
             got16 = b16.cpu().numpy().view(np.uint16)
@@ -204,6 +206,9 @@ SMALL_LAYERS = [
     small_cfg("big_groups", T=600, H=256, E=4, k=2, I=384, G=128, wr_std=0.02),
     # 64-token tiles (T k <= 64 E): ragged multi-tile shared expert, some routed experts over 64 rows
     small_cfg("small_tiles_shared", T=200, H=512, E=8, k=2, I=256, has_shared=True, G=128, wr_std=0.04),
+    # asymmetric int4 (scale and minimum per group of 64), shared expert
+    small_cfg("asym_shared", T=150, H=512, E=8, k=2, I=256, has_shared=True, G=64, wr_std=0.03,
+              wfmt=synth.WFMT_INT4_ASYM),
 ]
 
 
@@ -260,7 +265,8 @@ def test_fused_equals_composed_bitwise(dev, cfg):
     assert torch.equal(y.view(torch.int16), fused["y_bf16"].view(torch.int16))
 
 
-@pytest.mark.parametrize("cfg", [SMALL_LAYERS[5], SMALL_LAYERS[3], SMALL_LAYERS[1]], ids=lambda c: c.name)
+@pytest.mark.parametrize("cfg", [SMALL_LAYERS[5], SMALL_LAYERS[3], SMALL_LAYERS[1], SMALL_LAYERS[7]],
+                         ids=lambda c: c.name)
 @pytest.mark.parametrize("ctas", [1, 3])
 def test_layer_on_few_ctas_is_bitwise_equal(dev, cfg, ctas, monkeypatch):
     """Each work unit is computed the same way whichever CTA takes it, so a
@@ -287,7 +293,7 @@ def test_layer_is_deterministic(dev):
 
 # --------------------------------------------------------- full-size layers
 
-FULL = [("a3b_t512", 96), ("a3b_t8192_zipf", 48), ("a3b_t4096_q4k", 40),
+FULL = [("a3b_t512", 96), ("a3b_t8192_zipf", 48), ("a3b_t4096_q4k", 40), ("a3b_t512_asym", 64),
         ("a3b_decode_t1", None), ("a3b_decode_t8", None), ("a3b_decode_t32", None)]
 
 
