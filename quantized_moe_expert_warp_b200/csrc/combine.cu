@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace moeq4 {
 
@@ -29,6 +30,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict
                                                       const float *__restrict__ gate_logit, int T, int H, int k,
                                                       uint16_t *__restrict__ y)
 {
+    pdl_wait();
+    pdl_allow_successor();
     const int chunks = H / 8;
     const int per_cta_tokens = blockDim.x / chunks > 0 ? blockDim.x / chunks : 1;
     if ((int)threadIdx.x / chunks >= per_cta_tokens)
@@ -81,8 +84,8 @@ cudaError_t launch_combine(const uint16_t *y_perm, const int32_t *dest_pos, cons
     const int chunks = H / 8;
     const int threads = 256;
     const int per = threads / chunks > 0 ? threads / chunks : 1;
-    combine_kernel<<<(T + per - 1) / per, threads, 0, st>>>(y_perm, dest_pos, w, shared_out, gate_logit, T, H, k, y);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, (T + per - 1) / per, threads, 0, st, y_perm, dest_pos, w, shared_out, gate_logit,
+                      T, H, k, y);
 }
 
 }  // namespace moeq4

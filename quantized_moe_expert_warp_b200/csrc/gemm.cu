@@ -305,6 +305,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
         bars->never_abort = 0;
         fence_mbar_init();
     }
+    // everything below reads what the previous kernels in the stream wrote
+    pdl_wait();
+    pdl_allow_successor();
     build_schedule<BN>(p, s_tile_start, s_row_start, s_row_count, s_part);
     if (warp == 3) {
         tmem_alloc(&bars->tmem_base, L::kTmemCols);
@@ -894,8 +897,7 @@ static cudaError_t launch_one(const GemmArgs &a_in, int num_sms, cudaStream_t st
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
-    kern<<<num_sms, kThreads, smem, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(kern, num_sms, kThreads, smem, st, a);
 }
 
 size_t gemm_smem_required(int nmat, int meta_bytes, int E_total)

@@ -3,11 +3,42 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cstdlib>
+#include <utility>
 #include <cuda_runtime.h>
 
 #include "moeq4.h"
 
 namespace moeq4 {
+
+// Launch with programmatic dependent launch: the kernel may be scheduled
+// while its predecessor in the stream is still running (once every CTA of
+// the predecessor has allowed it) and waits inside (griddepcontrol.wait)
+// until the predecessor has finished and its writes are visible.  Every
+// hot-path kernel waits before its first global read or write, so the
+// ordering of the stream is unchanged; only launch latency is hidden.
+// MOEQ4_NO_PDL=1 launches without it.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args)
+{
+    static const bool off = [] {
+        const char *e = getenv("MOEQ4_NO_PDL");
+        return e && e[0] == '1';
+    }();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = off ? 0 : 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 
 struct GemmArgs {
     const uint8_t *wq;          // codes, kernel layout

@@ -37,6 +37,8 @@ size_t permute_scratch_bytes(int T, int E, int k)
 __global__ void __launch_bounds__(kPermThreads) permute_hist_kernel(const int32_t *__restrict__ ids, int S, int E,
                                                                     int chunk, int32_t *hist, int *status)
 {
+    pdl_wait();
+    pdl_allow_successor();
     extern __shared__ int32_t s_hist[];   // [E]
     for (int e = threadIdx.x; e < E; e += blockDim.x)
         s_hist[e] = 0;
@@ -137,6 +139,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(const int
                                                                        int32_t *counts, int32_t *offsets,
                                                                        int32_t *sorted_slot, int32_t *dest_pos)
 {
+    pdl_wait();
+    pdl_allow_successor();
     extern __shared__ int32_t s_mem[];
     const int nblk = gridDim.x, b = blockIdx.x;
     auto tot_e = [&](int e) {
@@ -164,6 +168,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_single_kernel(const int3
                                                                       int32_t *sorted_slot, int32_t *dest_pos,
                                                                       int *status)
 {
+    pdl_wait();
+    pdl_allow_successor();
     extern __shared__ int32_t s_mem[];
     int32_t *s_hist = s_mem + E + kPermThreads + (32 * E + 1) / 2;   // [E], after the scatter's scratch
     for (int e = threadIdx.x; e < E; e += blockDim.x)
@@ -202,15 +208,14 @@ cudaError_t launch_permute(const int32_t *ids, int T, int E, int k, int32_t *cou
             if (e1 != cudaSuccess)
                 return e1;
         }
-        permute_single_kernel<<<1, kPermThreads, smem1, st>>>(ids, S, E, counts, offsets, sorted_slot, dest_pos,
-                                                               status);
-        return cudaGetLastError();
+        return launch_pdl(permute_single_kernel, 1, kPermThreads, smem1, st, ids, S, E, counts, offsets, sorted_slot,
+                          dest_pos, status);
     }
     const int chunk = perm_chunk(S);
     const int nblk = perm_blocks(S);
     int32_t *hist = (int32_t *)scratch;
-    permute_hist_kernel<<<nblk, kPermThreads, E * sizeof(int32_t), st>>>(ids, S, E, chunk, hist, status);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err =
+        launch_pdl(permute_hist_kernel, nblk, kPermThreads, E * sizeof(int32_t), st, ids, S, E, chunk, hist, status);
     if (err != cudaSuccess)
         return err;
     const size_t smem = (E + kPermThreads) * sizeof(int32_t) + 32 * E * sizeof(uint16_t);
@@ -219,9 +224,8 @@ cudaError_t launch_permute(const int32_t *ids, int T, int E, int k, int32_t *cou
         if (err != cudaSuccess)
             return err;
     }
-    permute_scatter_kernel<<<nblk, kPermThreads, smem, st>>>(ids, S, E, chunk, hist, counts, offsets, sorted_slot,
-                                                              dest_pos);
-    return cudaGetLastError();
+    return launch_pdl(permute_scatter_kernel, nblk, kPermThreads, smem, st, ids, S, E, chunk, (const int32_t *)hist,
+                      counts, offsets, sorted_slot, dest_pos);
 }
 
 
@@ -292,8 +296,8 @@ cudaError_t launch_permute_noalloc(const int32_t *ids, int T, int E, int k, int3
     const int nblk = perm_blocks(S);
     // ids outside [0, E) are not reported through a status word here; their
     // dest_pos entries come back as -1
-    permute_hist_kernel<<<nblk, kPermThreads, E * sizeof(int32_t), st>>>(ids, S, E, chunk, hist, nullptr);
-    err = cudaGetLastError();
+    err = launch_pdl(permute_hist_kernel, nblk, kPermThreads, E * sizeof(int32_t), st, ids, S, E, chunk, hist,
+                     (int *)nullptr);
     if (err != cudaSuccess)
         return err;
     const size_t smem = (E + kPermThreads) * sizeof(int32_t) + 32 * E * sizeof(uint16_t);
@@ -302,9 +306,8 @@ cudaError_t launch_permute_noalloc(const int32_t *ids, int T, int E, int k, int3
         if (err != cudaSuccess)
             return err;
     }
-    permute_scatter_kernel<<<nblk, kPermThreads, smem, st>>>(ids, S, E, chunk, hist, counts, offsets, sorted_slot,
-                                                              dest_pos);
-    return cudaGetLastError();
+    return launch_pdl(permute_scatter_kernel, nblk, kPermThreads, smem, st, ids, S, E, chunk, (const int32_t *)hist,
+                      counts, offsets, sorted_slot, dest_pos);
 }
 
 }  // namespace moeq4

@@ -278,6 +278,12 @@ __device__ __forceinline__ bool elect_one()
     return pred != 0;
 }
 
+// Programmatic dependent launch: wait until the predecessor grid has
+// finished (no-op without the launch attribute), and let the successor be
+// scheduled now (it still waits for this grid to finish before it reads).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_allow_successor() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ copies
 
 // 16-byte cp.async; src_bytes = 0 writes zeros (the source is not read).

@@ -10,6 +10,7 @@
 #include <math_constants.h>
 
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace moeq4 {
 
@@ -39,6 +40,8 @@ __global__ void __launch_bounds__(128) route_kernel(const float *__restrict__ lo
                                                     const float *__restrict__ part, int nsplit,
                                                     const float *__restrict__ bias, float *logits_out)
 {
+    pdl_wait();
+    pdl_allow_successor();
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
     const int lane = threadIdx.x % 32;
     if (warp >= T)
@@ -149,24 +152,24 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
     const int npl = (E + 31) / 32;
 #define ROUTE_ARGS logits, T, E, k, renorm, ids, w, part, nsplit, bias, logits_out
     if (npl <= 1)
-        route_kernel<1><<<blocks, 128, 0, st>>>(ROUTE_ARGS);
-    else if (npl <= 2)
-        route_kernel<2><<<blocks, 128, 0, st>>>(ROUTE_ARGS);
-    else if (npl <= 4)
-        route_kernel<4><<<blocks, 128, 0, st>>>(ROUTE_ARGS);
-    else if (npl <= 8)
-        route_kernel<8><<<blocks, 128, 0, st>>>(ROUTE_ARGS);
-    else if (npl <= 16)
-        route_kernel<16><<<blocks, 128, 0, st>>>(ROUTE_ARGS);
-    else
-        route_kernel<32><<<blocks, 128, 0, st>>>(ROUTE_ARGS);
+        return launch_pdl(route_kernel<1>, blocks, 128, 0, st, ROUTE_ARGS);
+    if (npl <= 2)
+        return launch_pdl(route_kernel<2>, blocks, 128, 0, st, ROUTE_ARGS);
+    if (npl <= 4)
+        return launch_pdl(route_kernel<4>, blocks, 128, 0, st, ROUTE_ARGS);
+    if (npl <= 8)
+        return launch_pdl(route_kernel<8>, blocks, 128, 0, st, ROUTE_ARGS);
+    if (npl <= 16)
+        return launch_pdl(route_kernel<16>, blocks, 128, 0, st, ROUTE_ARGS);
+    return launch_pdl(route_kernel<32>, blocks, 128, 0, st, ROUTE_ARGS);
 #undef ROUTE_ARGS
-    return cudaGetLastError();
 }
 
 __global__ void __launch_bounds__(256) router_reduce_kernel(const float *__restrict__ part, int nsplit, int T, int E,
                                                             const float *__restrict__ bias, float *logits)
 {
+    pdl_wait();
+    pdl_allow_successor();
     const size_t TE = (size_t)T * E;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < TE; i += (size_t)gridDim.x * blockDim.x)
         logits[i] = sum_partials(part, nsplit, TE, i, bias, (int)(i % E));
@@ -179,8 +182,7 @@ cudaError_t launch_router_reduce(const float *part, int nsplit, int T, int E, co
     if (TE == 0)
         return cudaSuccess;
     const int blocks = (int)((TE + 255) / 256 < 4096 ? (TE + 255) / 256 : 4096);
-    router_reduce_kernel<<<blocks, 256, 0, st>>>(part, nsplit, T, E, bias, logits);
-    return cudaGetLastError();
+    return launch_pdl(router_reduce_kernel, blocks, 256, 0, st, part, nsplit, T, E, bias, logits);
 }
 
 }  // namespace moeq4
