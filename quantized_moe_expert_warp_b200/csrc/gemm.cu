@@ -92,7 +92,13 @@ __device__ unsigned long long g_trace[4][16][kTraceSteps];
     } while (0)
 #endif
 
-constexpr int kAStages = 4;  // TMEM A-operand ring depth (dequantised k-steps)
+constexpr int kMaxAStages = 8;   // TMEM A-operand ring depth (dequantised k-steps), upper bound
+#ifndef MOEQ4_A_STAGES_GU
+#define MOEQ4_A_STAGES_GU 4
+#endif
+#ifndef MOEQ4_A_STAGES_DN
+#define MOEQ4_A_STAGES_DN 8
+#endif
 constexpr int kMaxCodeChunks = 8;   // code ring: chunks of several k-steps, one bulk copy each
 constexpr int kMaxMetaBufs = 4;
 constexpr int kEpiTok = 16;  // tokens per epilogue chunk
@@ -112,8 +118,14 @@ struct Geo {
     static constexpr int kNA = MODE == MODE_DOWN ? 1 : 2;                               // A operands per k-step
     static constexpr int kNAcc = MODE == MODE_GATE_UP ? 2 : 1;                          // accumulators per unit
     static constexpr int kNAcc_ = MODE == MODE_GATE_UP ? 2 : 1;
-    // as many accumulator buffers (up to 2) as TMEM holds next to the A stages:
-    // with two, the epilogue of one tile overlaps the MMAs of the next
+    // TMEM (512 columns): A stages of kNA x 32 columns, then as many
+    // accumulator buffers (up to 2) as fit; with two, the epilogue of one
+    // tile overlaps the MMAs of the next.  The requested A-stage count is cut
+    // to leave room for one accumulator buffer.
+    static constexpr int kAStagesReq = MODE == MODE_GATE_UP ? MOEQ4_A_STAGES_GU : MODE == MODE_DOWN ? MOEQ4_A_STAGES_DN : 4;
+    static constexpr int kAStagesFit = (512 - kNAcc_ * BN) / (kNA * 32);
+    static constexpr int kAStages = kAStagesReq < kAStagesFit ? kAStagesReq : kAStagesFit;
+    static_assert(kAStages >= 2 && kAStages <= kMaxAStages, "TMEM A stages");
     static constexpr int kAccBufs = (512 - kAStages * kNA * 32) / (kNAcc_ * BN) >= 2 ? 2 : 1;
     static constexpr int kNCode = MODE == MODE_GATE_UP ? 2 : MODE == MODE_DOWN ? 1 : 0; // code matrices
     // dequant warp groups: groups of four warps, each warp a full k-step of
@@ -137,8 +149,8 @@ struct Geo {
 };
 
 struct Barriers {
-    uint64_t a_full[kAStages];    // k-step dequantised into TMEM (8 dequant warps)
-    uint64_t a_empty[kAStages];   // MMAs reading that TMEM stage completed
+    uint64_t a_full[kMaxAStages];    // k-step dequantised into TMEM (one dequant group)
+    uint64_t a_empty[kMaxAStages];   // MMAs reading that TMEM stage completed
     uint64_t b_full[8];           // token rows landed in shared memory (32 cp.async arrivals)
     uint64_t b_empty[8];
     uint64_t code_full[kMaxCodeChunks];
@@ -280,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
     const int lane = threadIdx.x % 32;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kAStages; ++s) {
+        for (int s = 0; s < L::kAStages; ++s) {
             mbar_init(&bars->a_full[s], L::kGroupWarps);
             mbar_init(&bars->a_empty[s], 1);
         }
@@ -385,9 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
             }
             CYC(0);
             for (int ks = 0; ks < un.nks; ++ks, ++step) {
-                const int sa = step % kAStages, sb = step % L::kBStages;
+                const int sa = step % L::kAStages, sb = step % L::kBStages;
                 // every lane polls the same barriers, so the outcome is warp-uniform
-                if (!mbar_wait(&bars->a_full[sa], (step / kAStages) & 1, wc, 3)) {
+                if (!mbar_wait(&bars->a_full[sa], (step / L::kAStages) & 1, wc, 3)) {
                     ok = false;
                     break;
                 }
@@ -507,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                     ++bi;
                     t_last = globaltimer_ns();
                 }
-                if (ai < n_steps && test(smem_u32(&bars->a_full[ai % kAStages]), (ai / kAStages) & 1)) {
+                if (ai < n_steps && test(smem_u32(&bars->a_full[ai % L::kAStages]), (ai / L::kAStages) & 1)) {
                     TRACE_EVENT(10, ai);
                     ++ai;
                     t_last = globaltimer_ns();
@@ -587,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
             for (int ks = kbeg + ((grp - step0) % L::kGroups + L::kGroups) % L::kGroups; ks < kend;
                  ks += L::kGroups) {
                 step = step0 + (ks - kbeg);
-                const int sa = step % kAStages;
+                const int sa = step % L::kAStages;
                 const uint32_t a_col = tmem + lane_off + L::kAccCols + sa * L::kNA * 32;
                 CYC(6);
                 if (MODE == MODE_ROUTER) {
@@ -608,7 +620,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
 #pragma unroll
                     for (int jj = 0; jj < 16; ++jj)
                         split2(v[2 * jj], v[2 * jj + 1], words[0][jj], words[1 % L::kNA][jj]);
-                    if (step >= kAStages && !mbar_wait(&bars->a_empty[sa], ((step / kAStages) & 1) ^ 1, wc, 10)) {
+                    if (step >= L::kAStages &&
+                        !mbar_wait(&bars->a_empty[sa], ((step / L::kAStages) & 1) ^ 1, wc, 10)) {
                         ok = false;
                         break;
                     }
@@ -674,8 +687,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                             if (lane == 0 && warp == 4)
                                 TRACE_EVENT(11, step);
                             // the MMAs that read this TMEM stage kAStages k-steps ago have finished
-                            if (step >= kAStages &&
-                                !mbar_wait(&bars->a_empty[sa], ((step / kAStages) & 1) ^ 1, wc, 10)) {
+                            if (step >= L::kAStages &&
+                                !mbar_wait(&bars->a_empty[sa], ((step / L::kAStages) & 1) ^ 1, wc, 10)) {
                                 ok = false;
                                 break;
                             }
