@@ -42,8 +42,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict
     const int S = T * k;
     const int32_t *dp = dest_pos + (size_t)t * k;
     const float *wt = w + (size_t)t * k;
+    // the shared expert's gate, once per token
+    const float g = shared_out && gate_logit ? 1.0f / (1.0f + expf(-gate_logit[t])) : 1.0f;
     for (int c = threadIdx.x % chunks; c < chunks; c += blockDim.x) {
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // the shared expert's row is loaded with the first batch, added last
+        const uint4 sv = shared_out ? *(const uint4 *)(shared_out + (size_t)t * H + c * 8) : make_uint4(0, 0, 0, 0);
         // batches of 8 rows: all loads of a batch are in flight together
         for (int j0 = 0; j0 < k; j0 += 8) {
             uint4 v[8];
@@ -60,10 +64,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict
                 if (j0 + j < k)
                     add8(acc, v[j], wj[j]);
         }
-        if (shared_out) {
-            const float g = gate_logit ? 1.0f / (1.0f + expf(-gate_logit[t])) : 1.0f;
-            add8(acc, *(const uint4 *)(shared_out + (size_t)t * H + c * 8), g);
-        }
+        if (shared_out)
+            add8(acc, sv, g);
         uint4 o;
         uint32_t *ou = &o.x;
 #pragma unroll

@@ -71,21 +71,36 @@ __device__ __forceinline__ void permute_rank_scatter(const int32_t *__restrict__
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
 
     // expert totals, this chunk's prefix, and the exclusive scan over experts
+    // (warp shuffles, then one warp over the 32 warp totals)
     int tot = 0, pre = 0;
     if (tid < E) {
         tot = tot_e(tid);
         pre = pre_e(tid);
     }
-    s_scan[tid] = tot;
-    __syncthreads();
-    for (int off = 1; off < kPermThreads; off <<= 1) {
-        const int v = tid >= off ? s_scan[tid - off] : 0;
-        __syncthreads();
-        s_scan[tid] += v;
-        __syncthreads();
+    int incl = tot;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off)
+            incl += n;
     }
+    if (lane == 31)
+        s_scan[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int wsum = s_scan[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int n = __shfl_up_sync(0xFFFFFFFFu, wsum, off);
+            if (lane >= off)
+                wsum += n;
+        }
+        s_scan[32 + lane] = wsum;   // inclusive prefix of the warp totals
+    }
+    __syncthreads();
+    incl += warp > 0 ? s_scan[32 + warp - 1] : 0;
     if (tid < E) {
-        const int off_e = s_scan[tid] - tot;
+        const int off_e = incl - tot;
         s_base[tid] = off_e + pre;
         if (writer) {
             counts[tid] = tot;
@@ -93,7 +108,7 @@ __device__ __forceinline__ void permute_rank_scatter(const int32_t *__restrict__
         }
     }
     if (writer && tid == 0)
-        offsets[E] = s_scan[kPermThreads - 1];
+        offsets[E] = s_scan[32 + 31];
     for (int i = tid; i < 32 * E; i += kPermThreads)
         s_wcnt[i] = 0;
     __syncthreads();
