@@ -149,6 +149,12 @@ def dist_setup():
     return rank, world, local
 
 
+def replica_config(cfg, rank: int):
+    """Weak-scaling replicas: every rank runs the same layer (same weights)
+    on its own T tokens (its own activation stream)."""
+    return cfg if rank == 0 else cfg.with_(x_stream=cfg.x_stream + 7919 * rank)
+
+
 def max_over_ranks(v: float, world: int, device) -> float:
     if world == 1:
         return v
@@ -251,7 +257,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     # every rank: the same layer weights, its own tokens
-    rcfg = cfg if rank == 0 else cfg.with_(x_stream=cfg.x_stream + 7919 * rank)
+    rcfg = replica_config(cfg, rank)
     layer = synth.make_layer(rcfg)
     packed = upload_layer(layer, dev)
     T, H, E, k = cfg.T, cfg.H, cfg.E, cfg.k
