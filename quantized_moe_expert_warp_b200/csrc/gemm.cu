@@ -234,21 +234,37 @@ __device__ void build_schedule(const GemmArgs &p, int *s_tile_start, int *s_row_
         s_row_count[e] = cnt;
         local += (cnt + BN - 1) / BN;
     }
-    s_part[threadIdx.x] = local;
-    __syncthreads();
-    for (int off = 1; off < kThreads; off <<= 1) {
-        const int v = threadIdx.x >= off ? s_part[threadIdx.x - off] : 0;
-        __syncthreads();
-        s_part[threadIdx.x] += v;
-        __syncthreads();
+    // exclusive scan of the per-thread tile counts: warp shuffles, then one
+    // warp over the warp totals
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off)
+            incl += v;
     }
-    int run = s_part[threadIdx.x] - local;
+    if (lane == 31)
+        s_part[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < kThreads / 32 ? s_part[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, w, off);
+            if (lane >= off)
+                w += v;
+        }
+        s_part[32 + lane] = w;   // inclusive prefix of the warp totals
+    }
+    __syncthreads();
+    int run = incl - local + (warp > 0 ? s_part[32 + warp - 1] : 0);
     for (int e = e0; e < min(n, e0 + per); ++e) {
         s_tile_start[e] = run;
         run += (s_row_count[e] + BN - 1) / BN;
     }
     if (threadIdx.x == kThreads - 1)
-        s_tile_start[n] = s_part[kThreads - 1];
+        s_tile_start[n] = s_part[32 + kThreads / 32 - 1];
 }
 
 // fp32 -> two bf16 parts (hi, lo): w - hi is exact in fp32, so hi + lo
