@@ -261,6 +261,21 @@ int moe_layer_forward(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *
                       void *stream, const moe_debug_t *dbg);
 
 /*
+ * Chunked prefill: the layer over T tokens as consecutive chunks of at most
+ * `chunk` tokens (the last one ragged), each a moe_layer_forward call on
+ * the same stream and the same workspace, which only has to hold one chunk
+ * (moe_layer_workspace_size(cfg, min(chunk, T)) bytes).  Tokens never
+ * interact inside the layer, so every token's output is that of the
+ * one-shot call wherever both pick the same router split (always for
+ * chunk >= 4096 with E = 256, H = 2048).  The hipfire 0.4.3 benchmarks run
+ * long prompts as such chunks ("Late prefill steps on mq4rs": 16000 tokens as 8192 +
+ * 7808); the chunk loop is this library's.  MOE_ERR_INVALID_ARG for
+ * chunk < 1; errors of a chunk stop the loop and are returned.
+ */
+int moe_layer_forward_chunked(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *y, int chunk, void *ws,
+                              size_t ws_bytes, void *stream);
+
+/*
  * Read (and, when clear != 0, reset) the device status word kept in a
  * workspace of moe_layer_forward / moe_expert_ffn_q4 / moe_permute.
  * Synchronises `stream`.  *status = MOE_OK or the first MOE_ERR_* code a

@@ -644,6 +644,32 @@ int moe_layer_forward(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *
     return ok();
 }
 
+int moe_layer_forward_chunked(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *y, int chunk, void *ws,
+                              size_t ws_bytes, void *stream)
+{
+    int rc = check_layer(L);
+    if (rc)
+        return rc;
+    REQUIRE(T >= 0, "T must be >= 0");
+    REQUIRE(chunk >= 1, "chunk must be >= 1");
+    const int Tc = T < chunk ? T : chunk;
+    const size_t need = moe_layer_workspace_size(&L->cfg, Tc);
+    if (!ws || ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "layer workspace: need %zu bytes, got %zu", need, ws ? ws_bytes : (size_t)0);
+    if (T == 0)
+        return ok();
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(y);
+    const size_t H = (size_t)L->cfg.H;
+    for (int off = 0; off < T; off += chunk) {
+        const int n = T - off < chunk ? T - off : chunk;
+        rc = moe_layer_forward(L, x + (size_t)off * H, n, y + (size_t)off * H, ws, ws_bytes, stream, nullptr);
+        if (rc)
+            return rc;
+    }
+    return ok();
+}
+
 int moe_read_status(void *ws, void *stream, int clear, int *status, int *detail)
 {
     REQUIRE_PTR(ws);

@@ -126,6 +126,17 @@ def test_workspace_too_small_is_reported(L):
     assert rc == mq.MOE_ERR_WORKSPACE
 
 
+def test_chunked_layer_checks_chunk_and_workspace(L):
+    layer = mq.Layer(cfg(), 0x1000, None, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000)
+    rc = L.moe_layer_forward_chunked(C.byref(layer), 0x1000, 16000, 0x1000, 0, 0x1000, 1 << 40, None)
+    assert rc == mq.MOE_ERR_INVALID_ARG and b"chunk" in L.moe_last_error()
+    # the workspace has to hold one chunk, not all T tokens
+    one = L.moe_layer_workspace_size(C.byref(cfg()), 8192)
+    assert one < L.moe_layer_workspace_size(C.byref(cfg()), 16000)
+    rc = L.moe_layer_forward_chunked(C.byref(layer), 0x1000, 16000, 0x1000, 8192, 0x1000, one - 256, None)
+    assert rc == mq.MOE_ERR_WORKSPACE
+
+
 def test_layer_rejects_missing_shared_gate(L):
     layer = mq.Layer(cfg(), 0x1000, None, None, 0x1000, 0x1000, 0x1000, 0x1000)
     need = L.moe_layer_workspace_size(C.byref(cfg()), 512)

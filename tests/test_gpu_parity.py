@@ -314,3 +314,66 @@ def test_full_size_layer_sampled(dev, name, nsample):
         assert np.array_equal(got["sorted_slot"], ref["sorted_slot"])
     assert got["counts"].sum() == cfg.T * cfg.k
     print(f"{name}: max|err|/max|ref| {stats[0]:.2e} rel L2 {stats[1]:.2e} near-ties {len(ties)}")
+
+
+# ------------------------------------------------------ multi-chunk prefill
+
+def _chunks_one_by_one(layer, dev, packed, chunk):
+    """Each chunk as its own moe_layer_forward (with every debug export)."""
+    cfg = layer["cfg"]
+    outs = []
+    for off in range(0, cfg.T, chunk):
+        n = min(chunk, cfg.T - off)
+        sub = dict(layer, cfg=cfg.with_T(n, f"{cfg.name}_at{off}"), x=layer["x"][off:off + n])
+        outs.append((off, sub, run_layer(sub, dev, packed=packed)))
+    return outs
+
+
+def _forward_chunked(layer, dev, packed, chunk):
+    import quantized_moe_expert_warp_b200 as mq
+    from quantized_moe_expert_warp_b200.host import x_to_device
+    cfg = layer["cfg"]
+    x = x_to_device(layer["x"], dev)
+    y = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
+    n = mq.moe_layer_workspace_size(cfg, min(cfg.T, chunk))
+    ws = torch.zeros(n, dtype=torch.uint8, device=dev)
+    mq.moe_layer_forward_chunked(packed, x, cfg.T, y, chunk, ws, n)
+    assert mq.moe_read_status(ws)[0] == 0
+    return y
+
+
+@pytest.mark.parametrize("cfg,chunk", [(SMALL_LAYERS[1], 128), (SMALL_LAYERS[3], 130), (SMALL_LAYERS[7], 1)],
+                         ids=["ragged_shared_c128", "q4k_one_chunk", "asym_c1"])
+def test_chunked_layer_equals_chunks_and_oracle(dev, cfg, chunk):
+    """A long prompt in chunks: every chunk is exactly one layer call on its
+    rows (bitwise), and the concatenation matches the oracle on all T rows."""
+    from quantized_moe_expert_warp_b200.host import upload_layer
+    if chunk == 1:
+        cfg = cfg.with_T(9, "asym_t9")
+    layer = synth.make_layer(cfg)
+    packed = upload_layer(layer, dev)
+    y = _forward_chunked(layer, dev, packed, chunk)
+    parts = _chunks_one_by_one(layer, dev, packed, chunk)
+    ref_y = torch.cat([p[2]["y_bf16"] for p in parts])
+    assert torch.equal(y.view(torch.int16), ref_y.view(torch.int16))
+    for off, sub, got in parts:
+        compare_layer(sub, got)
+
+
+def test_chunked_full_size_prefill_16000(dev):
+    """16000 prompt tokens of the full-size layer as 8192 + 7808 rows: bitwise
+    equal to the two layer calls, each sampled against the oracle."""
+    from quantized_moe_expert_warp_b200.host import upload_layer
+    cfg = synth.get_config("a3b_t8192_zipf").with_T(16000, "a3b_t16000_zipf")
+    layer = synth.make_layer(cfg)
+    packed = upload_layer(layer, dev)
+    y = _forward_chunked(layer, dev, packed, 8192)
+    parts = _chunks_one_by_one(layer, dev, packed, 8192)
+    assert [p[1]["cfg"].T for p in parts] == [8192, 7808]
+    ref_y = torch.cat([p[2]["y_bf16"] for p in parts])
+    assert torch.equal(y.view(torch.int16), ref_y.view(torch.int16))
+    rng = np.random.default_rng(77)
+    for off, sub, got in parts:
+        n = sub["cfg"].T
+        sample = np.sort(np.concatenate([[0, n - 1], rng.choice(np.arange(1, n - 1), 22, replace=False)]))
+        compare_layer(sub, got, sample=sample)
