@@ -67,17 +67,17 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 // SMs of the current device (148 when it cannot be queried).
 int device_sms()
 {
-    static int cache[64] = {0};
+    static std::atomic<int> cache[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return 148;
-    if (!cache[dev]) {
-        int n = 0;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (!n) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             n = 148;
-        cache[dev] = n;
+        cache[dev].store(n, std::memory_order_relaxed);
     }
-    return cache[dev];
+    return n;
 }
 
 // CTAs of the persistent kernels: one per SM.  MOEQ4_GRID_CTAS (1 .. SM
@@ -661,8 +661,8 @@ int moe_layer_forward_chunked(const moe_layer_t *L, const uint16_t *x, int T, ui
     REQUIRE_PTR(x);
     REQUIRE_PTR(y);
     const size_t H = (size_t)L->cfg.H;
-    for (int off = 0; off < T; off += chunk) {
-        const int n = T - off < chunk ? T - off : chunk;
+    for (int64_t off = 0; off < T; off += chunk) {
+        const int n = (int)(T - off < chunk ? T - off : chunk);
         rc = moe_layer_forward(L, x + (size_t)off * H, n, y + (size_t)off * H, ws, ws_bytes, stream, nullptr);
         if (rc)
             return rc;
