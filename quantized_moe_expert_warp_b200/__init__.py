@@ -108,11 +108,19 @@ def lib():
 
 
 def _ptr(t):
-    """Device address of a torch tensor / int / None."""
+    """Device address of a torch tensor / int / None.
+
+    A tensor must be a dense CUDA tensor: the kernels take bare addresses
+    with the row-major layouts of moeq4.h, so a host tensor or a strided
+    view is refused here rather than read wrongly on the device."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_cuda:
+        raise ValueError(f"expected a CUDA tensor, got one on {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"expected a contiguous tensor, got strides {tuple(t.stride())}")
     return t.data_ptr()
 
 

@@ -150,3 +150,23 @@ def test_zero_tokens_is_a_no_op(L):
     need = L.moe_layer_workspace_size(C.byref(cfg()), 0)
     assert L.moe_layer_forward(C.byref(layer), None, 0, None, 0x1000, need, None, None) == 0
     assert L.moe_route(None, 0, 16, 2, 1, None, None, None) == 0
+
+
+def test_binding_refuses_host_and_strided_tensors(L):
+    torch = pytest.importorskip("torch")
+    logits = torch.zeros((4, 16), dtype=torch.float32)
+    ids = torch.zeros((4, 2), dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mq.moe_route(logits, 4, 16, 2, True, ids, ids.float(), stream=0)
+
+    class FakeCuda:
+        is_cuda = True
+
+        def is_contiguous(self):
+            return False
+
+        def stride(self):
+            return (1, 4)
+
+    with pytest.raises(ValueError, match="contiguous"):
+        mq.moe_route(FakeCuda(), 4, 16, 2, True, 0x1000, 0x1000, stream=0)
