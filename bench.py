@@ -54,6 +54,7 @@ def expert_bytes(cfg) -> tuple:
 
 
 WFMT_NAMES = {0: "int4-sym", 1: "q4k", 2: "int4-asym"}
+L2_BYTES = 126e6   # B200 L2
 
 
 def kernel_source_hash() -> str:
@@ -234,6 +235,7 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=96, help="tokens of the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true", help="short run for ncu: no e2e / cpu legs")
+    ap.add_argument("--decode", action="store_true", help="T <= 8 through the fused decode kernel")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if not args.profile else args.warmup
 
@@ -270,12 +272,44 @@ def main():
     T, H, E, k = cfg.T, cfg.H, cfg.E, cfg.k
     x = x_to_device(layer["x"], dev)
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-    nbytes = mq.moe_layer_workspace_size(cfg, T)
-    ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    # --decode: batches of T <= 8 through the fused single-kernel layer (measured
+    # slower than the kernel chain so far, so the chain is the default)
+    decode = args.decode and mq.moe_layer_decode_workspace_size(cfg, T) > 0
+    layer_call = mq.moe_layer_decode if decode else mq.moe_layer_forward
+    nbytes = mq.moe_layer_decode_workspace_size(cfg, T) if decode else mq.moe_layer_workspace_size(cfg, T)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
 
     def step():
-        mq.moe_layer_forward(packed, x, T, y, ws, nbytes, stream)
+        layer_call(packed, x, T, y, ws, nbytes, stream)
+
+    # When one step reads less than twice the L2 (126 MB), L2 is flushed
+    # (a 256 MB write) before every timed step and only the steps are timed;
+    # otherwise the step's own weights already exceed L2.
+    gu_b, dn_b = expert_bytes(cfg)
+    step_bytes_bound = min(T * k + 1, E + 1) * (gu_b + dn_b)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if step_bytes_bound < 2 * L2_BYTES else None
+
+    def timed_steps(fn, n):
+        """Mean device ms of n calls of fn: one event pair around all of
+        them, or (with the L2 flush) around each one."""
+        if flush is None:
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(n):
+                fn()
+            b.record(stream)
+            b.synchronize()
+            return a.elapsed_time(b) / n
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for i in range(n):
+            flush.fill_(i & 0xFF)
+            pairs[i][0].record(stream)
+            fn()
+            pairs[i][1].record(stream)
+        pairs[-1][1].synchronize()
+        return sum(a.elapsed_time(b) for a, b in pairs) / n
 
     for _ in range(args.warmup):
         step()
@@ -286,17 +320,11 @@ def main():
 
     # ---------------------------------------------------------- timed region
     sampler = ClockSampler(local)
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
     with sampler:
         barrier(world)
         torch.cuda.synchronize(dev)
         launches0 = mq.moe_kernel_launches()
-        ev0.record(stream)
-        for _ in range(args.steps):
-            step()
-        ev1.record(stream)
-        ev1.synchronize()
+        ms = timed_steps(step, args.steps)
         launches = mq.moe_kernel_launches() - launches0
         torch.cuda.synchronize(dev)
         barrier(world)
@@ -307,7 +335,6 @@ def main():
             for _ in range(20):
                 step()
             torch.cuda.synchronize(dev)
-    ms = ev0.elapsed_time(ev1) / args.steps
     ms_max = max_over_ranks(ms, world, dev)
     st, det = mq.moe_read_status(ws, stream)
     if st != 0:
@@ -347,6 +374,8 @@ def main():
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(args.steps)]
     torch.cuda.synchronize(dev)
     for s in range(args.steps):
+        if flush is not None:
+            flush.fill_(s & 0xFF)
         evs[s][0].record(stream)
         for i, c in enumerate(calls):
             c()
@@ -356,7 +385,6 @@ def main():
                      for i, n in enumerate(names)}
     composed_ms = sum(per_kernel_ms.values())
     touched = int((counts.cpu().numpy() > 0).sum()) + (1 if cfg.has_shared else 0)
-    gu_b, dn_b = expert_bytes(cfg)
     alg = {
         "gate_up_gemm": touched * gu_b + 2 * T * H,
         "down_gemm": touched * dn_b,
@@ -393,6 +421,12 @@ def main():
                     "peak_source": peak_src}
     # whole-layer roofline: max(FLOPs at tensor peak, bytes at HBM peak)
     layer_bytes = touched * (gu_b + dn_b) + E * H * 4 + 4 * T * H
+    if decode:
+        # one kernel is the whole step: its algorithmic bytes are the layer's
+        achieved = layer_bytes / (ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "kernel": "decode_layer", "achieved": achieved, "peak": hbm_peak,
+                    "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": ncu_traffic("decode", cfg.name),
+                    "algorithmic_bytes_per_launch": layer_bytes, "ms_per_launch": ms, "peak_source": peak_src}
     t_hbm = layer_bytes / (hbm_peak * 1e9)
     tc_peak = peaks.get("bf16_tflops", 1590.0)
     t_tc = T * fpt / (tc_peak * 1e12)
@@ -410,21 +444,14 @@ def main():
 
         def e2e_step():
             x_in.copy_(x_host, non_blocking=True)
-            mq.moe_layer_forward(packed, x_in, T, y_out, ws, nbytes, stream)
+            layer_call(packed, x_in, T, y_out, ws, nbytes, stream)
             y_host.copy_(y_out.view(torch.int16), non_blocking=True)
 
         for _ in range(3):
             e2e_step()
         torch.cuda.synchronize(dev)
         barrier(world)
-        a0 = torch.cuda.Event(enable_timing=True)
-        a1 = torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        a1.record(stream)
-        a1.synchronize()
-        e_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps, world, dev)
+        e_ms = max_over_ranks(timed_steps(e2e_step, args.steps), world, dev)
         e2e = {"value": world * T / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
                "d2h_bytes_per_step": T * H * 2, "ms_per_step": e_ms}
 
@@ -445,7 +472,11 @@ def main():
             "config": {"workload": cfg.name, "T": T, "H": H, "E": E, "k": k, "I": cfg.I,
                        "shared_expert": bool(cfg.has_shared), "weights": WFMT_NAMES[cfg.wfmt],
                        "G": cfg.G, "tokens_per_rank": T, "parallelism": f"replicas x{world} (token-sharded)",
-                       "l2": "inputs larger than L2 (expert weights %.0f MB)" % (packed.weight_bytes() / 1e6)},
+                       "path": "fused decode kernel" if decode else "kernel chain",
+                       "l2": ("flushed before each timed step (256 MB write); a step reads %.0f MB of weights"
+                              % (touched * (gu_b + dn_b) / 1e6)) if flush is not None else
+                             ("inputs larger than L2 (a step reads %.0f MB of expert weights)"
+                              % (touched * (gu_b + dn_b) / 1e6))},
             "tflops": tflops, "flop_per_token": fpt,
             "roofline": roofline, "layer_roofline": layer_roof,
             "per_kernel_ms": per_kernel_ms, "composed_ms_per_step": composed_ms,

@@ -276,8 +276,40 @@ int moe_layer_forward_chunked(const moe_layer_t *L, const uint16_t *x, int T, ui
                               size_t ws_bytes, void *stream);
 
 /*
+ * Fused decode layer: the same layer for 1 <= T <= 8 tokens as ONE
+ * cooperative kernel (one CTA per SM, grid barriers between the router,
+ * the gate/up and the down steps).  The pages measure decode as generated
+ * tokens per second with one token per step (hipfire 0.4.3 benchmarks,
+ * "Qwen3.6-35B-A3B mq4rs · decode on the R9700, 0.4.3 → 0.4.3.1", where
+ * the gain comes from replaying the step's launches instead of issuing
+ * them); at such sizes the separate kernels of moe_layer_forward cost more
+ * in launches and pipeline fill than in memory traffic.
+ *
+ * Results: routing as in moe_route (on this kernel's fp32 logits), expert
+ * FFNs with the exact dequantised weights in fp32 on CUDA cores, no
+ * intermediate rounded to bf16 before y.  Within the layer tolerance of
+ * the oracle, but not bitwise equal to moe_layer_forward.  Independent of
+ * the number of CTAs (work is split by output rows only).
+ *
+ * ws: moe_layer_decode_workspace_size(cfg, T) bytes (0 = shape or T not
+ * admitted: T > 8, or x or the expert intermediates do not fit in shared
+ * memory; the call then returns MOE_ERR_UNSUPPORTED).  Its first 256 bytes
+ * (status word and the grid barrier's words) must be zero before the first
+ * call: allocate it zeroed or call moe_read_status(ws, stream, 1, ...)
+ * once.  Calls leave them valid; after MOE_ERR_TIMEOUT is recorded further
+ * calls on this workspace stop at once until moe_read_status clears it.
+ * dbg may export logits, gate_logit, topk_ids and topk_w, and may give
+ * override_ids / override_w; its counts, offsets, sorted_slot and
+ * dest_pos are not written.
+ */
+size_t moe_layer_decode_workspace_size(const moe_config_t *cfg, int T);
+int moe_layer_decode(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *y, void *ws, size_t ws_bytes,
+                     void *stream, const moe_debug_t *dbg);
+
+/*
  * Read (and, when clear != 0, reset) the device status word kept in a
- * workspace of moe_layer_forward / moe_expert_ffn_q4 / moe_permute.
+ * workspace of moe_layer_forward / moe_layer_decode / moe_expert_ffn_q4 /
+ * moe_permute; clearing zeroes the workspace's whole 256-byte status block.
  * Synchronises `stream`.  *status = MOE_OK or the first MOE_ERR_* code a
  * kernel recorded; *detail (optional) = where it was recorded.
  */

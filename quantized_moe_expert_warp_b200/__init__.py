@@ -16,7 +16,7 @@ __all__ = [
     "MoeError", "Config", "lib", "moe_version", "moe_last_error", "moe_packed_sizes", "moe_pack_weights",
     "moe_dequant_export", "moe_router_workspace_size", "moe_router_logits", "moe_route", "moe_permute_workspace_size", "moe_permute",
     "moe_expert_ffn_workspace_size", "moe_expert_ffn_q4", "moe_combine", "moe_layer_workspace_size",
-    "moe_layer_forward", "moe_layer_forward_chunked", "moe_read_status", "moe_kernel_launches", "moe_expert_gate_up_q4", "moe_expert_down_q4",
+    "moe_layer_forward", "moe_layer_forward_chunked", "moe_layer_decode_workspace_size", "moe_layer_decode", "moe_read_status", "moe_kernel_launches", "moe_expert_gate_up_q4", "moe_expert_down_q4",
     "moe_permute_noalloc", "PackedLayer", "WFMT_INT4_SYM", "WFMT_Q4K", "WFMT_INT4_ASYM", "LIB_PATH",
 ]
 
@@ -97,6 +97,8 @@ def lib():
             "moe_layer_workspace_size": (sz, [vp, i32]),
             "moe_layer_forward": (i32, [vp, vp, i32, vp, vp, sz, vp, vp]),
             "moe_layer_forward_chunked": (i32, [vp, vp, i32, vp, i32, vp, sz, vp]),
+            "moe_layer_decode_workspace_size": (sz, [vp, i32]),
+            "moe_layer_decode": (i32, [vp, vp, i32, vp, vp, sz, vp, vp]),
             "moe_read_status": (i32, [vp, vp, i32, vp, vp]),
         }
         for name, (res, args) in sig.items():
@@ -242,6 +244,20 @@ def moe_layer_forward(layer: "PackedLayer", x, T, y, ws, ws_bytes, stream=None, 
 def moe_layer_forward_chunked(layer: "PackedLayer", x, T, y, chunk, ws, ws_bytes, stream=None):
     _call("moe_layer_forward_chunked", C.byref(layer.c_layer), _ptr(x), T, _ptr(y), int(chunk), _ptr(ws), ws_bytes,
           _stream(stream))
+
+
+def moe_layer_decode_workspace_size(cfg, T) -> int:
+    """0 when the fused decode kernel does not take this shape or T (> 8)."""
+    c = Config.of(cfg)
+    return lib().moe_layer_decode_workspace_size(C.byref(c), T)
+
+
+def moe_layer_decode(layer: "PackedLayer", x, T, y, ws, ws_bytes, stream=None, debug: dict | None = None):
+    dbg = None
+    if debug:
+        dbg = Debug(**{k: _ptr(v) for k, v in debug.items()})
+    _call("moe_layer_decode", C.byref(layer.c_layer), _ptr(x), T, _ptr(y), _ptr(ws), ws_bytes, _stream(stream),
+          C.byref(dbg) if dbg is not None else None)
 
 
 def moe_read_status(ws, stream=None, clear=True):

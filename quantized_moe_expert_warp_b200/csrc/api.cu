@@ -200,6 +200,52 @@ LayerWs layer_layout(const moe_config_t *c, int T, uint8_t *base)
     return w;
 }
 
+// Workspace of the fused decode kernel: the 256-byte status block (status
+// word, detail, and at byte 64 the grid barrier's count, generation and
+// abort flag), then logits, gate logits, routing and the fp32 expert outputs.
+struct DecodeWs {
+    int *status;
+    unsigned *bar;
+    float *logits, *gate_logit, *w, *h, *o;
+    int32_t *ids;
+    size_t bytes;
+};
+
+DecodeWs decode_layout(const moe_config_t *c, int T, uint8_t *base)
+{
+    DecodeWs w{};
+    const size_t Tk = (size_t)T * c->k;
+    const size_t NP = Tk + (c->has_shared ? T : 0);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t *p = base + off;
+        off += align256(bytes);
+        return p;
+    };
+    w.status = (int *)take(256);
+    w.bar = (unsigned *)((uint8_t *)w.status + 64);
+    w.logits = (float *)take(sizeof(float) * (size_t)T * c->E);
+    w.gate_logit = (float *)take(sizeof(float) * (size_t)T);
+    w.ids = (int32_t *)take(sizeof(int32_t) * Tk);
+    w.w = (float *)take(sizeof(float) * Tk);
+    w.h = (float *)take(sizeof(float) * NP * c->I);
+    w.o = (float *)take(sizeof(float) * NP * c->H);
+    w.bytes = off;
+    return w;
+}
+
+constexpr size_t kMaxDynamicSmem = 227 * 1024;
+
+// Why the decode kernel does not take (cfg, T), or null.
+const char *decode_refusal(const moe_config_t *c, int T)
+{
+    if (T > kDecodeMaxT)
+        return "the fused decode kernel takes at most 8 tokens";
+    if (decode_smem_layout(T, c->k, c->H, c->I, c->has_shared).bytes > kMaxDynamicSmem)
+        return "x or the expert intermediates of this shape exceed shared memory";
+    return nullptr;
+}
+
 int check_layer(const moe_layer_t *L)
 {
     if (!L)
@@ -670,6 +716,85 @@ int moe_layer_forward_chunked(const moe_layer_t *L, const uint16_t *x, int T, ui
     return ok();
 }
 
+size_t moe_layer_decode_workspace_size(const moe_config_t *cfg, int T)
+{
+    if (check_config(cfg) || T < 0 || decode_refusal(cfg, T))
+        return 0;
+    return decode_layout(cfg, T, nullptr).bytes;
+}
+
+int moe_layer_decode(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *y, void *ws, size_t ws_bytes,
+                     void *stream, const moe_debug_t *dbg)
+{
+    int rc = check_layer(L);
+    if (rc)
+        return rc;
+    const moe_config_t &c = L->cfg;
+    REQUIRE(T >= 0, "T must be >= 0");
+    if (const char *why = decode_refusal(&c, T))
+        return fail(MOE_ERR_UNSUPPORTED, "moe_layer_decode: %s (T = %d)", why, T);
+    const size_t need = moe_layer_decode_workspace_size(&c, T);
+    if (!ws || ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "decode workspace: need %zu bytes, got %zu", need, ws ? ws_bytes : (size_t)0);
+    REQUIRE_PTR(ws);
+    if (T == 0)
+        return ok();
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(y);
+    const bool override_route = dbg && dbg->override_ids;
+    if (override_route) {
+        REQUIRE_PTR(dbg->override_ids);
+        REQUIRE_PTR(dbg->override_w);
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    const DecodeWs w = decode_layout(&c, T, (uint8_t *)ws);
+    DecodeArgs a{};
+    a.x = x;
+    a.T = T;
+    a.H = c.H;
+    a.I = c.I;
+    a.E = c.E;
+    a.k = c.k;
+    a.G = c.G;
+    a.wfmt = c.wfmt;
+    a.renorm = c.renorm;
+    a.has_shared = c.has_shared ? 1 : 0;
+    a.router_w = L->router_w;
+    a.router_bias = L->router_bias;
+    a.shared_gate = c.has_shared ? L->shared_gate : nullptr;
+    a.gu_q = (const uint8_t *)L->gu_q;
+    a.gu_meta = (const uint8_t *)L->gu_meta;
+    a.dn_q = (const uint8_t *)L->dn_q;
+    a.dn_meta = (const uint8_t *)L->dn_meta;
+    a.gu_meta_bytes = meta_block_bytes(2, c.wfmt, c.H, c.G);
+    a.dn_meta_bytes = meta_block_bytes(1, c.wfmt, c.I, c.G);
+    a.override_ids = override_route ? dbg->override_ids : nullptr;
+    a.override_w = override_route ? dbg->override_w : nullptr;
+    a.logits = w.logits;
+    a.gate_logit = w.gate_logit;
+    a.topk_ids = w.ids;
+    a.topk_w = w.w;
+    a.h = w.h;
+    a.o = w.o;
+    a.y = y;
+    a.status = w.status;
+    a.bar = w.bar;
+    CUDA_TRY(launch_decode_layer(a, num_sms(), st), "fused decode layer");
+    g_launches += 1;
+    if (dbg) {
+        auto cp = [&](void *dst, const void *src, size_t bytes) -> cudaError_t {
+            return dst ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st) : cudaSuccess;
+        };
+        const size_t Tk = (size_t)T * c.k;
+        CUDA_TRY(cp(dbg->logits, w.logits, sizeof(float) * (size_t)T * c.E), "export logits");
+        if (c.has_shared)
+            CUDA_TRY(cp(dbg->gate_logit, w.gate_logit, sizeof(float) * T), "export gate logit");
+        CUDA_TRY(cp(dbg->topk_ids, w.ids, sizeof(int32_t) * Tk), "export ids");
+        CUDA_TRY(cp(dbg->topk_w, w.w, sizeof(float) * Tk), "export weights");
+    }
+    return ok();
+}
+
 int moe_read_status(void *ws, void *stream, int clear, int *status, int *detail)
 {
     REQUIRE_PTR(ws);
@@ -682,7 +807,8 @@ int moe_read_status(void *ws, void *stream, int clear, int *status, int *detail)
     if (detail)
         *detail = h[1];
     if (clear) {
-        CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof h, st), "clear status");
+        // the whole status block: also the decode kernel's grid-barrier words
+        CUDA_TRY(cudaMemsetAsync(ws, 0, 256, st), "clear status");
         CUDA_TRY(cudaStreamSynchronize(st), "clear status sync");
     }
     return ok();

@@ -170,3 +170,28 @@ def test_binding_refuses_host_and_strided_tensors(L):
 
     with pytest.raises(ValueError, match="contiguous"):
         mq.moe_route(FakeCuda(), 4, 16, 2, True, 0x1000, 0x1000, stream=0)
+
+
+def test_decode_admission_and_workspace(L):
+    c = cfg()
+    # a3b shape: T = 1..8 admitted, 9 and more go through moe_layer_forward
+    sizes = [L.moe_layer_decode_workspace_size(C.byref(c), t) for t in (1, 2, 8)]
+    assert 0 < sizes[0] < sizes[1] < sizes[2]
+    # h and the expert outputs in fp32 for T k + T pairs
+    assert sizes[2] >= (8 * 8 + 8) * (512 + 2048) * 4
+    assert L.moe_layer_decode_workspace_size(C.byref(c), 9) == 0
+    layer = mq.Layer(c, 0x1000, None, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000)
+    rc = L.moe_layer_decode(C.byref(layer), 0x1000, 9, 0x1000, 0x1000, 1 << 30, None, None)
+    assert rc == mq.MOE_ERR_UNSUPPORTED and b"8 tokens" in L.moe_last_error()
+    rc = L.moe_layer_decode(C.byref(layer), 0x1000, 4, 0x1000, 0x1000,
+                            L.moe_layer_decode_workspace_size(C.byref(c), 4) - 256, None, None)
+    assert rc == mq.MOE_ERR_WORKSPACE
+    # the intermediates of 8 tokens at k = 32, I = 1024 do not fit in shared memory (1 token does)
+    big = cfg(k=32, I=1024)
+    assert L.moe_layer_decode_workspace_size(C.byref(big), 8) == 0
+    assert L.moe_layer_decode_workspace_size(C.byref(big), 1) > 0
+    layer = mq.Layer(big, 0x1000, None, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000)
+    rc = L.moe_layer_decode(C.byref(layer), 0x1000, 8, 0x1000, 0x1000, 1 << 30, None, None)
+    assert rc == mq.MOE_ERR_UNSUPPORTED and b"shared memory" in L.moe_last_error()
+    # zero tokens: nothing to do
+    assert L.moe_layer_decode(C.byref(layer), None, 0, None, 0x1000, 1 << 20, None, None) == mq.MOE_OK
