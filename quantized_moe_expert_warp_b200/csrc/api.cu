@@ -8,6 +8,7 @@
 #include <cstring>
 #include <cuda_runtime.h>
 
+#include "decode.h"
 #include "dequant.cuh"
 #include "kernels.h"
 #include "moeq4.h"

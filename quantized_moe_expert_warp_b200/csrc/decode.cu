@@ -31,6 +31,7 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include "decode.h"
 #include "dequant.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
