@@ -27,6 +27,7 @@
 //
 // Work is split by output rows, never by K, and every sum runs in a fixed
 // order, so the result does not depend on the number of CTAs.
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <math_constants.h>
@@ -700,17 +701,17 @@ cudaError_t launch_decode_layer(const DecodeArgs &a, int grid, cudaStream_t st)
 {
     const DecodeSmem L = decode_smem_layout(a.T, a.k, a.H, a.I, a.has_shared);
     // the opt-in limit once per device (callers never ask for more: see the admission check)
-    static bool configured[64] = {};
+    static std::atomic<bool> configured[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
-    if (dev < 0 || dev >= 64 || !configured[dev]) {
+    if (dev < 0 || dev >= 64 || !configured[dev].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(decode_layer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess)
             return e;
         if (dev >= 0 && dev < 64)
-            configured[dev] = true;
+            configured[dev].store(true, std::memory_order_release);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
