@@ -42,6 +42,22 @@ def test_binding_names_match_header():
         assert hasattr(mq, n), n
 
 
+def test_binding_constants_match_header():
+    txt = open(os.path.join(ROOT, "include", "moeq4.h")).read()
+    defs = dict(re.findall(r"#define (MOE_[A-Z0-9_]+) \(?(-?\d+)\)?", txt))
+    assert len(defs) >= 9
+    for name, value in defs.items():
+        py = name.replace("MOE_WFMT_", "WFMT_")
+        assert getattr(mq, py) == int(value), name
+    # the ctypes structs mirror the header's field order
+    for struct, fields in (("moe_config_t", mq.Config._fields_), ("moe_layer_t", mq.Layer._fields_),
+                           ("moe_debug_t", mq.Debug._fields_)):
+        block = txt[:txt.index("} " + struct + ";")]
+        block = block[block.rindex("typedef struct"):]
+        names = re.findall(r"\b(\w+)\s*;", re.sub(r"/\*.*?\*/", "", block, flags=re.S))
+        assert names == [f[0] for f in fields], (struct, names)
+
+
 def cfg(**kw):
     d = dict(H=2048, I=512, E=256, k=8, G=128, has_shared=1, renorm=1, wfmt=mq.WFMT_INT4_SYM)
     d.update(kw)
