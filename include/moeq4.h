@@ -162,6 +162,9 @@ size_t moe_router_workspace_size(const moe_config_t *cfg, int T);
  *   in the caller's workspace ws (at least moe_router_workspace_size bytes,
  *   256-byte aligned; MOE_ERR_WORKSPACE if smaller) and are summed in slice
  *   order.
+ * Source: the router of the Qwen3.6-35B-A3B layer the hipfire 0.4.3
+ * benchmarks measure ("Qwen3.6-35B-A3B prefill on the R9700" table); the
+ * pages give no formula, so logits = x Wr^T + bias is this library's reading.
  */
 int moe_router_logits(const moe_layer_t *L, const uint16_t *x, int T, float *logits, float *gate_logit, void *ws,
                       size_t ws_bytes, void *stream);
@@ -169,7 +172,13 @@ int moe_router_logits(const moe_layer_t *L, const uint16_t *x, int T, float *log
 /*
  * Top-k routing, one warp per token.  logits [T, E] fp32 (finite),
  * topk_ids [T, k] int32 (descending logit, ties to the lower id),
- * topk_w [T, k] fp32.  1 <= k <= min(E, 32), E <= 1024.
+ * topk_w [T, k] fp32.  1 <= k <= min(E, 32), E <= 1024.  A position that
+ * cannot be filled because the remaining logits are NaN gets id -1 and
+ * weight 0 (moe_permute then reports the id as out of range).
+ * Source: the top-8 expert choice of the A3B layer (hipfire 0.4.3
+ * benchmarks, "Qwen3.6-35B-A3B prefill on the R9700" table); the tie rule
+ * and the renormalised softmax are this library's reading, the pages give
+ * neither.
  */
 int moe_route(const float *logits, int T, int E, int k, int renorm, int32_t *topk_ids, float *topk_w,
               void *stream);
@@ -182,6 +191,9 @@ size_t moe_permute_workspace_size(int T, int E, int k);
  *   counts [E], offsets [E + 1] (offsets[E] = T k), sorted_slot [T k]
  *   (slot t*k + j at position p), dest_pos [T k] (inverse).  Ids outside
  *   [0, E) are a device error (status word).  ws: moe_permute_workspace_size.
+ * Source: hipfire 0.4.3 benchmarks, "Read this before comparing columns"
+ * table, row "MoE prefill route" (per-expert buffers): the tokens of each
+ * expert gathered together; here one permutation replaces the buffers.
  */
 int moe_permute(const int32_t *topk_ids, int T, int E, int k, int32_t *counts, int32_t *offsets,
                 int32_t *sorted_slot, int32_t *dest_pos, void *ws, size_t ws_bytes, void *stream);
@@ -197,9 +209,10 @@ int moe_permute(const int32_t *topk_ids, int T, int E, int k, int32_t *counts, i
  *    sized for E <= 1024 experts (any T); each GPU that loads the library
  *    keeps it (128 KB) until the process exits.  E > 1024 returns
  *    MOE_ERR_UNSUPPORTED.  The call allocates nothing.
- *  - The first call on a device looks up the array's device address (a
- *    runtime call, no stream work); make that first call before any stream
- *    capture.
+ *  - The call runs on the current device, and `stream` must belong to it
+ *    (otherwise MOE_ERR_INVALID_ARG).  The first call on a device looks up
+ *    the array's device address for that device (a runtime call, no stream
+ *    work) and keeps it; make that first call before any stream capture.
  *  - All calls on a device share the array: calls that may overlap on the GPU
  *    (unordered streams) race and must be serialised by the caller.  Nothing
  *    needs clearing between calls.
@@ -219,7 +232,13 @@ size_t moe_expert_ffn_workspace_size(const moe_config_t *cfg, int T);
  *   t = sorted_slot[p] / k, and the intermediate rounded to bf16;
  * and with a shared expert shared_out[t] the same FFN with its weights for
  * every token t.  x [T, H], y_perm [T k, H], shared_out [T, H] (bf16).
- * offsets [E + 1] from moe_permute.
+ * offsets [E + 1] from moe_permute.  ws: moe_expert_ffn_workspace_size
+ * bytes (MOE_ERR_WORKSPACE if smaller); a wait that runs out of its budget
+ * inside a kernel is recorded in ws's status word (moe_read_status).
+ * Source: hipfire 0.4.3 benchmarks, "Read this before comparing columns"
+ * table and the text under it (the symmetric IU4 MoE prefill route for
+ * files whose experts hold symmetric int4 weights); hipEngine post, "GGUF"
+ * (Q4_K).  The SwiGLU expert is this library's reading of the Qwen3 FFN.
  */
 int moe_expert_ffn_q4(const moe_layer_t *L, const uint16_t *x, int T, const int32_t *sorted_slot,
                       const int32_t *offsets, uint16_t *y_perm, uint16_t *shared_out, void *ws, size_t ws_bytes,
@@ -242,6 +261,9 @@ int moe_expert_down_q4(const moe_layer_t *L, const uint16_t *h, int T, const int
  * Weighted combine: y[t] = bf16( sum_j topk_w[t,j] y_perm[dest_pos[t k + j]]
  *                                + sigmoid(shared_gate_logit[t]) shared_out[t] )
  * summed in fp32 in j order; shared_out / shared_gate_logit may be NULL.
+ * Source: the weighted sum over the chosen experts of the A3B layer
+ * (hipfire 0.4.3 benchmarks, "Qwen3.6-35B-A3B prefill on the R9700"
+ * table); the sigmoid gate of the shared expert is this library's reading.
  */
 int moe_combine(const uint16_t *y_perm, const int32_t *dest_pos, const float *topk_w, const uint16_t *shared_out,
                 const float *shared_gate_logit, int T, int H, int k, uint16_t *y, void *stream);

@@ -163,6 +163,9 @@ def layer_forward(layer: dict, sample=None, override_ids=None, override_w=None):
     intermediates (logits, gate_logit, ids, w, counts, offsets,
     sorted_slot, dest_pos).  ``sample`` lists the tokens whose outputs are
     computed (routing and permutation always cover all T tokens).
+    ``override_ids`` replaces the oracle's top-k choice; without
+    ``override_w`` the oracle weighs those ids itself from its own logits
+    (the same softmax as its routing step).
     """
     cfg = layer["cfg"]
     T, H, E, k, I = cfg.T, cfg.H, cfg.E, cfg.k, cfg.I

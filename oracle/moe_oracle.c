@@ -180,6 +180,24 @@ int oracle_router_logits(const uint16_t *x, int64_t T, int64_t H, const float *w
  * (renorm = 1: equal to softmax over all E followed by renormalisation of
  * the chosen k) or the plain softmax probability over all E (renorm = 0).
  */
+/* Weights of k chosen experts from the token's fp32 logits (the chosen ids
+ * in any order, the first taken as the reference for exp): softmax over the
+ * k chosen logits (renorm = 1) or over all E (renorm = 0). */
+static void topk_weights(const float *L, int64_t E, int64_t k, int renorm, const int32_t *ids, double *w)
+{
+    double top = (double)L[ids[0]];
+    double z = 0.0;
+    if (renorm) {
+        for (int64_t j = 0; j < k; ++j)
+            z += exp((double)L[ids[j]] - top);
+    } else {
+        for (int64_t e = 0; e < E; ++e)
+            z += exp((double)L[e] - top);
+    }
+    for (int64_t j = 0; j < k; ++j)
+        w[j] = exp((double)L[ids[j]] - top) / z;
+}
+
 static void route_one(const float *L, int64_t E, int64_t k, int renorm, int32_t *ids, double *w)
 {
     for (int64_t j = 0; j < k; ++j) {
@@ -196,17 +214,7 @@ static void route_one(const float *L, int64_t E, int64_t k, int renorm, int32_t 
         }
         ids[j] = (int32_t)best;
     }
-    double top = (double)L[ids[0]];
-    double z = 0.0;
-    if (renorm) {
-        for (int64_t j = 0; j < k; ++j)
-            z += exp((double)L[ids[j]] - top);
-    } else {
-        for (int64_t e = 0; e < E; ++e)
-            z += exp((double)L[e] - top);
-    }
-    for (int64_t j = 0; j < k; ++j)
-        w[j] = exp((double)L[ids[j]] - top) / z;
+    topk_weights(L, E, k, renorm, ids, w);
 }
 
 int oracle_route(const float *logits, int64_t T, int64_t E, int64_t k, int renorm, int32_t *ids,
@@ -342,7 +350,8 @@ typedef struct {
     const uint8_t *dn_q;         /* int4: nib [Et, H, I/2]; Q4K: [Et, H, I/256*144] */
     const uint16_t *dn_scale;    /* int4-sym: [Et, H, I/G]; int4-asym: [Et, H, I/G, 2]; Q4K: NULL */
     const int32_t *override_ids; /* optional [T, k]: routing to use instead of the oracle's */
-    const float *override_w;     /* optional [T, k] (with override_ids) */
+    const float *override_w;     /* optional [T, k] (with override_ids); NULL: the oracle weighs
+                                    the given ids itself from its own logits */
     const int32_t *sample;       /* tokens whose output rows are computed; NULL = all */
     int64_t n_sample;
     /* outputs */
@@ -434,8 +443,16 @@ int oracle_layer_forward(const oracle_layer_args *A)
     if (A->override_ids) {
         for (int64_t s = 0; s < S; ++s) {
             ids[s] = A->override_ids[s];
-            w[s] = A->override_w ? (double)A->override_w[s] : 0.0;
+            if (ids[s] < 0 || ids[s] >= E) {
+                rc = ORACLE_EINVAL;
+                goto done;
+            }
+            if (A->override_w)
+                w[s] = (double)A->override_w[s];
         }
+        if (!A->override_w)
+            for (int64_t t = 0; t < T; ++t)
+                topk_weights(logits + t * E, E, k, A->renorm, ids + t * k, w + t * k);
     } else {
         rc = oracle_route(logits, T, E, k, A->renorm, ids, NULL, w);
         if (rc)

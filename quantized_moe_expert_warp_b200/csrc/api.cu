@@ -500,9 +500,18 @@ int moe_permute_noalloc(const int32_t *topk_ids, int T, int E, int k, int32_t *c
         REQUIRE_PTR(sorted_slot);
         REQUIRE_PTR(dest_pos);
     }
+    {
+        // the scratch address is the current device's: the stream must belong to it
+        int cur = 0, sdev = 0;
+        CUDA_TRY(cudaGetDevice(&cur), "moe_permute_noalloc: cudaGetDevice");
+        CUDA_TRY(cudaStreamGetDevice((cudaStream_t)stream, &sdev), "moe_permute_noalloc: cudaStreamGetDevice");
+        if (sdev != cur)
+            return fail(MOE_ERR_INVALID_ARG,
+                        "moe_permute_noalloc: the stream belongs to device %d, the current device is %d", sdev, cur);
+    }
     CUDA_TRY(launch_permute_noalloc(topk_ids, T, E, k, counts, offsets, sorted_slot, dest_pos, (cudaStream_t)stream),
              "moe_permute_noalloc");
-    g_launches += permute_launch_count(T, k);
+    g_launches += (size_t)T * k > 0 ? 2 : 0;   // always the histogram and the scatter kernel
     return ok();
 }
 

@@ -110,7 +110,8 @@ __global__ void __launch_bounds__(128) route_kernel(const float *__restrict__ lo
                 bid = oid;
             }
         }
-        if ((bid & 31) == lane)
+        // bid stays 0x7FFFFFFF only when every remaining logit is NaN
+        if (bid != 0x7FFFFFFF && (bid & 31) == lane)
             taken |= 1u << (bid >> 5);
         if (j == 0)
             top = bv;
@@ -138,8 +139,11 @@ __global__ void __launch_bounds__(128) route_kernel(const float *__restrict__ lo
         z = part;
     }
     if (lane < k) {
-        ids[(size_t)warp * k + lane] = my_id;
-        w[(size_t)warp * k + lane] = ex / z;
+        // a position left unfilled (NaN logits) gets id -1 and weight 0; the
+        // permutation reports such ids as out of range
+        const bool filled = my_id != 0x7FFFFFFF;
+        ids[(size_t)warp * k + lane] = filled ? my_id : -1;
+        w[(size_t)warp * k + lane] = filled ? ex / z : 0.f;
     }
 }
 

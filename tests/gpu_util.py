@@ -91,17 +91,41 @@ def near_tie_tokens(oracle_logits, oracle_ids, gpu_ids, k):
     return bad
 
 
+def oracle_rows(layer, sample=None, override_ids=None, threads=None):
+    """oracle.layer_forward, with a long sample split over threads.
+
+    The oracle is single-threaded C called through ctypes, which releases
+    the GIL, so chunks of the sample run in parallel; every chunk routes and
+    permutes the whole batch the same way, and the rows are concatenated in
+    sample order.
+    """
+    import concurrent.futures as cf
+    import os
+    if sample is None and layer["cfg"].T > 64:
+        sample = np.arange(layer["cfg"].T)
+    if sample is None or len(sample) <= 32:
+        return oracle.layer_forward(layer, sample=sample, override_ids=override_ids)
+    n = threads or max(1, min(len(os.sched_getaffinity(0)), 32, len(sample) // 16))
+    parts = np.array_split(np.asarray(sample), n)
+    with cf.ThreadPoolExecutor(n) as ex:
+        outs = list(ex.map(lambda s: oracle.layer_forward(layer, sample=s, override_ids=override_ids), parts))
+    ref = dict(outs[0])
+    ref["y"] = np.concatenate([o["y"] for o in outs])
+    return ref
+
+
 def compare_layer(layer, got, sample=None):
-    """Oracle on the same inputs (near-tie tokens re-run with the GPU's ids)."""
+    """Oracle on the same inputs.  Near-tie tokens are re-run with the GPU's
+    expert ids only: the oracle weighs those ids itself, from its own
+    logits, so no floating-point value of the CUDA path enters the
+    reference."""
     cfg = layer["cfg"]
-    ref = oracle.layer_forward(layer, sample=sample)
+    ref = oracle_rows(layer, sample=sample)
     ties = near_tie_tokens(ref["logits"], ref["ids"], got["topk_ids"], cfg.k)
     if len(ties):
         ids = ref["ids"].copy()
-        w = ref["w"].copy()
         ids[ties] = got["topk_ids"][ties]
-        w[ties] = got["topk_w"][ties]
-        ref = oracle.layer_forward(layer, sample=sample, override_ids=ids, override_w=w)
+        ref = oracle_rows(layer, sample=sample, override_ids=ids)
     y = got["y"] if sample is None else got["y"][np.asarray(sample)]
     stats = check_close(y, ref["y"], cfg.name)
     return ref, ties, stats

@@ -167,6 +167,11 @@ def test_combine(dev, T, H, k, shared):
 
 # ---------------------------------------------------------- router logits
 
+# Largest router-logit error accepted: about twice the largest error measured
+# on a B200 over these cases; kept below the near-tie threshold of the layer
+# tests, so that a routing flip it causes is not accepted as a near-tie.
+ROUTER_ATOL = 6e-5
+
 @pytest.mark.parametrize("T", [1, 200, 600])
 def test_router_logits_close(dev, T):
     """T = 1 and 200 split the reduction over H into 32 slices, T = 600 into 8."""
@@ -183,9 +188,10 @@ def test_router_logits_close(dev, T):
     mq.moe_router_logits(packed, x, cfg.T, logits, gl, rws, rn)
     ref = oracle.router_logits(layer["x"], layer["router_w"], layer["router_bias"])
     # bf16 x is exact; fp32 weights enter as two bf16 parts (16 significand bits) with exact products,
-    # summed by the tensor cores' fp32 accumulation (truncating adds over
-    # H / 16 = 128 partial blocks): |err| ~ 1e-5 for |logit| up to ~8
-    np.testing.assert_allclose(logits.cpu().numpy(), ref, rtol=0, atol=1e-4)
+    # summed by the tensor cores' fp32 accumulation over H / 16 = 128 partial blocks
+    err = np.abs(logits.cpu().numpy().astype(np.float64) - ref)
+    print(f"router T={T}: max |logit err| {err.max():.3e} (|logit| up to {np.abs(ref).max():.2f})")
+    assert err.max() <= ROUTER_ATOL, f"router logits off by {err.max():.3e} > {ROUTER_ATOL}"
     xs = synth.bf16_bits_to_f32(layer["x"]).astype(np.float64)
     np.testing.assert_allclose(gl.cpu().numpy(), xs @ layer["shared_gate"].astype(np.float64), atol=2e-5)
 
@@ -293,7 +299,7 @@ def test_layer_is_deterministic(dev):
 
 # --------------------------------------------------------- full-size layers
 
-FULL = [("a3b_t512", 96), ("a3b_t8192_zipf", 48), ("a3b_t4096_q4k", 40), ("a3b_t512_asym", 64),
+FULL = [("a3b_t512", None), ("a3b_t8192_zipf", 512), ("a3b_t4096_q4k", 512), ("a3b_t512_asym", None),
         ("a3b_decode_t1", None), ("a3b_decode_t8", None), ("a3b_decode_t32", None)]
 
 

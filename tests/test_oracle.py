@@ -385,10 +385,12 @@ def _dequant_all(layer):
     return np.stack(gu).astype(np.float64), np.stack(dn).astype(np.float64)
 
 
-def dense_reference(layer):
+def dense_reference(layer, ids=None):
     """Every expert on every token, masked by the top-k gate (numpy, fp64).
 
-    Shares no step with the oracle's permutation or gather-combine.
+    Shares no step with the oracle's permutation or gather-combine.  With
+    ``ids`` the gate keeps those experts instead of the top k (weights still
+    from the fp32 logits).
     """
     cfg = layer["cfg"]
     x = synth.bf16_bits_to_f32(layer["x"]).astype(np.float64)
@@ -398,7 +400,7 @@ def dense_reference(layer):
     L32 = L.astype(np.float32)
     gate = np.zeros((cfg.T, cfg.E))
     for t in range(cfg.T):
-        top = brute_topk(L32[t], cfg.k)
+        top = brute_topk(L32[t], cfg.k) if ids is None else np.asarray(ids[t])
         p = np.exp(L32[t].astype(np.float64) - L32[t].max())
         z = p[top].sum() if cfg.renorm else p.sum()
         gate[t, top] = p[top] / z
@@ -455,3 +457,56 @@ def test_single_expert_reduces_to_dense_swiglu():
     a, u = x @ gu[0, :32].T, x @ gu[0, 32:].T
     h = a * (1.0 / (1.0 + np.exp(-a))) * u
     assert np.allclose(got["y"], h @ dn[0].T, rtol=1e-12, atol=1e-15)
+
+
+# ------------------------------------------- routing supplied from outside
+
+def test_override_ids_weighed_by_oracle_closed_form():
+    """Ids given without weights: the oracle weighs them from its own logits.
+
+    Logits (1, 2).  Ids in the non-descending order (0, 1) keep the same
+    softmax pair: sig(-1) for expert 0 and sig(1) for expert 1.  Top-1 on
+    the lower expert: weight 1 after renormalisation, softmax over both
+    (sig(-1)) without it.
+    """
+    layer, Y0, Y1, S = _closed_form_layer()
+    r = oracle.layer_forward(layer, override_ids=np.array([[0, 1]], np.int32))
+    assert np.allclose(r["w"][0], [sig(-1.0), sig(1.0)], rtol=1e-7, atol=0)
+    assert np.allclose(r["y"][0], sig(-1.0) * Y0 + sig(1.0) * Y1 + 0.5 * S, rtol=1e-14, atol=0)
+    layer, Y0, Y1, S = _closed_form_layer(k=1)
+    r = oracle.layer_forward(layer, override_ids=np.array([[0]], np.int32))
+    assert r["w"][0, 0] == 1.0
+    assert np.allclose(r["y"][0], Y0 + 0.5 * S, rtol=1e-14, atol=0)
+    layer, Y0, Y1, S = _closed_form_layer(k=1, renorm=False)
+    r = oracle.layer_forward(layer, override_ids=np.array([[0]], np.int32))
+    assert np.allclose(r["y"][0], sig(-1.0) * Y0 + 0.5 * S, rtol=1e-14, atol=0)
+
+
+def test_override_ids_match_dense_bruteforce():
+    """Arbitrary distinct ids per token, weighed by the oracle, against the
+    dense evaluation masked by the same ids."""
+    cfg = synth.LayerConfig(name="dense_override", T=11, H=64, E=7, k=3, I=32, has_shared=True,
+                            wfmt=synth.WFMT_INT4_SYM, G=32, wr_std=0.3, zipf_s=0.0, seed=5)
+    layer = synth.make_layer(cfg)
+    rng = np.random.default_rng(4)
+    ids = np.stack([rng.permutation(cfg.E)[:cfg.k] for _ in range(cfg.T)]).astype(np.int32)
+    got = oracle.layer_forward(layer, override_ids=ids)
+    assert np.array_equal(got["ids"], ids)
+    want = dense_reference(layer, ids=ids)
+    assert np.allclose(got["y"], want, rtol=1e-10, atol=1e-13 * np.abs(want).max())
+
+
+def test_override_with_own_ids_is_the_plain_layer():
+    layer = synth.make_layer(synth.get_config("tiny_t64"))
+    plain = oracle.layer_forward(layer)
+    again = oracle.layer_forward(layer, override_ids=plain["ids"])
+    assert np.array_equal(again["y"], plain["y"])
+    assert np.array_equal(again["w"], plain["w"])
+
+
+def test_override_rejects_out_of_range_ids():
+    layer = synth.make_layer(synth.get_config("tiny_t64"))
+    ids = oracle.layer_forward(layer)["ids"].copy()
+    ids[3, 1] = layer["cfg"].E
+    with pytest.raises(ValueError):
+        oracle.layer_forward(layer, override_ids=ids)
