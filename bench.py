@@ -4,8 +4,12 @@
 Metric: MoE-layer prefill tokens/s (with TFLOP/s and the fraction of the
 layer roofline) for one Qwen3.6-35B-A3B-shaped layer: hidden 2048, 256
 routed experts, top-8, expert intermediate 512, one sigmoid-gated shared
-expert, symmetric int4 weights in groups of 128; default batch T = 512
-tokens of synthetic bf16 N(0,1) activations and seeded random weights.
+expert, symmetric int4 weights in groups of 128.  The default workload is
+one 8192-token prefill chunk with Zipf(1.1)-skewed expert selection, the
+largest single-GPU workload (seeded synthetic bf16 N(0,1) activations and
+random weights); at N = 1 the same line also carries the 512-token batch,
+the 4096-token Q4_K-style layer and the decode batches of 1, 8 and 32
+tokens under "extra_configs".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
 
@@ -182,18 +186,28 @@ def barrier(world):
 
 # ------------------------------------------------------------------ oracle arm
 
-def oracle_sample_rate(layer, n_tokens: int):
-    """Time the CPU oracle (as it stands) on the first n_tokens of the batch.
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
-    Routing and the permutation still cover the whole batch (that is how
-    the oracle is written); the expert FFNs and the combine run for the
-    sampled tokens only.  Returns (tokens/s, seconds)."""
+
+def oracle_sample_rate(layer, n_tokens: int):
+    """Time the CPU oracle (as it stands, one thread) on the first n_tokens
+    of the batch, run as a batch of their own.  Tokens never interact in the
+    layer, so those tokens' outputs are the ones the whole batch would give;
+    routing, permutation, expert FFNs and combine all cover just them.
+    Returns (tokens/s, seconds)."""
     import oracle
     oracle.build()
+    cfg = layer["cfg"]
+    n = min(n_tokens, cfg.T)
+    sub = dict(layer, cfg=cfg.with_T(n, f"{cfg.name}_first{n}"), x=layer["x"][:n])
     t0 = time.perf_counter()
-    oracle.layer_forward(layer, sample=np.arange(n_tokens))
+    oracle.layer_forward(sub)
     dt = time.perf_counter() - t0
-    return n_tokens / dt, dt
+    return n / dt, dt
 
 
 def run_reference(args, cfg, rank, world):
@@ -201,23 +215,23 @@ def run_reference(args, cfg, rank, world):
         return
     import synth
     layer = synth.make_layer(cfg)
-    n = args.ref_sample
+    n = min(args.ref_sample, cfg.T)
     for _ in range(args.warmup):
         oracle_sample_rate(layer, n)
-    rates, secs = [], 0.0
+    secs = 0.0
     for _ in range(args.steps):
-        r, dt = oracle_sample_rate(layer, n)
-        rates.append(r)
+        _, dt = oracle_sample_rate(layer, n)
         secs += dt
     value = args.steps * n / secs
+    sample = f"first {n} of {cfg.T} tokens per step, run as their own batch (one host thread of {host_cores()})"
     line = {
         "metric": "MoE-layer prefill tokens/s", "impl": "reference", "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights quantised)",
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k, "I": cfg.I},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"first {n} of {cfg.T} tokens per step (routing of all {cfg.T})"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "host_cores": host_cores(),
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -225,17 +239,225 @@ def run_reference(args, cfg, rank, world):
 
 # --------------------------------------------------------------------- our arm
 
+def pct(xs, q):
+    """q-th percentile (linear interpolation) of a list."""
+    return float(np.percentile(np.asarray(xs, np.float64), q))
+
+
+def load_peaks():
+    mp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    peaks = json.load(open(mp)) if os.path.exists(mp) else {}
+    hbm, src = peaks.get("hbm_gbs"), "measured"
+    if not hbm:
+        hbm, src = 6650.0, "fallback"
+    tc = peaks.get("bf16_tflops") or 1590.0
+    return hbm, tc, src
+
+
+class Bench:
+    """One layer configuration resident on one GPU: weights packed, inputs
+    and workspace allocated, the step callable, and its timing."""
+
+    def __init__(self, cfg, dev, stream, rank=0, decode=False):
+        import torch
+        import synth
+        import quantized_moe_expert_warp_b200 as mq
+        from quantized_moe_expert_warp_b200.host import upload_layer, x_to_device
+        self.torch, self.mq = torch, mq
+        self.cfg, self.dev, self.stream = cfg, dev, stream
+        self.layer = synth.make_layer(replica_config(cfg, rank))
+        self.packed = upload_layer(self.layer, dev)
+        T, H = cfg.T, cfg.H
+        self.x = x_to_device(self.layer["x"], dev)
+        self.y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        self.decode = decode and mq.moe_layer_decode_workspace_size(cfg, T) > 0
+        self.call = mq.moe_layer_decode if self.decode else mq.moe_layer_forward
+        self.nbytes = (mq.moe_layer_decode_workspace_size(cfg, T) if self.decode
+                       else mq.moe_layer_workspace_size(cfg, T))
+        self.ws = torch.zeros(self.nbytes, dtype=torch.uint8, device=dev)
+        # When one step reads less than twice the L2 (126 MB), L2 is flushed
+        # (a 256 MB write) before every timed step, outside its events;
+        # otherwise the step's own weights already exceed L2.
+        gu_b, dn_b = expert_bytes(cfg)
+        self.gu_b, self.dn_b = gu_b, dn_b
+        step_bytes_bound = min(T * cfg.k + 1, cfg.E + 1) * (gu_b + dn_b)
+        self.flush = (torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+                      if step_bytes_bound < 2 * L2_BYTES else None)
+
+    def step(self):
+        self.call(self.packed, self.x, self.cfg.T, self.y, self.ws, self.nbytes, self.stream)
+
+    def check_status(self, where):
+        st, det = self.mq.moe_read_status(self.ws, self.stream)
+        if st != 0:
+            raise RuntimeError(f"{self.cfg.name}: device status {st} ({det}) {where}")
+
+    def timed(self, fn, n):
+        """Per-step device ms of n calls of fn (CUDA events on the launching
+        stream), and the ms from the first call's start to the last one's end
+        (no flush: consecutive events; with the flush the steps are timed
+        one by one and the total is their sum)."""
+        torch = self.torch
+        if self.flush is None:
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+            ev[0].record(self.stream)
+            for i in range(n):
+                fn()
+                ev[i + 1].record(self.stream)
+            ev[-1].synchronize()
+            per = [ev[i].elapsed_time(ev[i + 1]) for i in range(n)]
+            return per, ev[0].elapsed_time(ev[-1])
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for i in range(n):
+            self.flush.fill_(i & 0xFF)
+            pairs[i][0].record(self.stream)
+            fn()
+            pairs[i][1].record(self.stream)
+        pairs[-1][1].synchronize()
+        per = [a.elapsed_time(b) for a, b in pairs]
+        return per, sum(per)
+
+    def per_kernel(self, steps):
+        """Mean device ms of each step of the kernel chain, run one call at a
+        time (the same kernels as the fused call) with events between them."""
+        torch, mq, cfg = self.torch, self.mq, self.cfg
+        T, H, E, k, dev, st, packed, x = cfg.T, cfg.H, cfg.E, cfg.k, self.dev, self.stream, self.packed, self.x
+        e32 = lambda *s: torch.empty(s, dtype=torch.float32, device=dev)
+        i32 = lambda *s: torch.empty(s, dtype=torch.int32, device=dev)
+        logits, gl, ids, tw = e32(T, E), e32(T), i32(T, k), e32(T, k)
+        counts, offsets, ss, dp = i32(E), i32(E + 1), i32(T * k), i32(T * k)
+        pn = mq.moe_permute_workspace_size(T, E, k)
+        pws = torch.zeros(pn, dtype=torch.uint8, device=dev)
+        rn = mq.moe_router_workspace_size(cfg, T)
+        rws = torch.zeros(rn, dtype=torch.uint8, device=dev)
+        fn = mq.moe_expert_ffn_workspace_size(cfg, T)
+        fws = torch.zeros(fn, dtype=torch.uint8, device=dev)
+        h = torch.empty((T * k + T, cfg.I), dtype=torch.bfloat16, device=dev)
+        y_perm = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
+        sh = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        names = ["router_logits", "route", "permute", "gate_up_gemm", "down_gemm", "combine"]
+        calls = [
+            lambda: mq.moe_router_logits(packed, x, T, logits, gl, rws, rn, st),
+            lambda: mq.moe_route(logits, T, E, k, cfg.renorm, ids, tw, st),
+            lambda: mq.moe_permute(ids, T, E, k, counts, offsets, ss, dp, pws, pn, st),
+            lambda: mq.moe_expert_gate_up_q4(packed, x, T, ss, offsets, h, fws, fn, st),
+            lambda: mq.moe_expert_down_q4(packed, h, T, offsets, y_perm, sh, fws, fn, st),
+            lambda: mq.moe_combine(y_perm, dp, tw, sh, gl, T, H, k, y, st),
+        ]
+        for _ in range(2):
+            for c in calls:
+                c()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(steps)]
+        torch.cuda.synchronize(dev)
+        for s in range(steps):
+            if self.flush is not None:
+                self.flush.fill_(s & 0xFF)
+            evs[s][0].record(st)
+            for i, c in enumerate(calls):
+                c()
+                evs[s][i + 1].record(st)
+        torch.cuda.synchronize(dev)
+        per = {n: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(steps))
+               for i, n in enumerate(names)}
+        touched = int((counts.cpu().numpy() > 0).sum()) + (1 if cfg.has_shared else 0)
+        return per, touched
+
+    def rooflines(self, ms_step, per_kernel_ms, touched):
+        """The dominant GEMM's roofline (its algorithmic bytes or FLOPs over
+        its own time) and the whole layer's (max of FLOPs at the tensor peak
+        and bytes at the HBM peak, over the step time)."""
+        cfg = self.cfg
+        T, H, E = cfg.T, cfg.H, cfg.E
+        hbm_peak, tc_peak, peak_src = load_peaks()
+        alg = {"gate_up_gemm": touched * self.gu_b + 2 * T * H, "down_gemm": touched * self.dn_b}
+        rows = T * cfg.k + (T if cfg.has_shared else 0)
+        flops = {"gate_up_gemm": 2.0 * rows * 2 * cfg.I * H, "down_gemm": 2.0 * rows * H * cfg.I}
+        dominant = max(("gate_up_gemm", "down_gemm"), key=lambda n: per_kernel_ms[n])
+        tag = {"gate_up_gemm": "gate_up", "down_gemm": "down"}[dominant]
+        secs = per_kernel_ms[dominant] * 1e-3
+        if flops[dominant] / (tc_peak * 1e12) > alg[dominant] / (hbm_peak * 1e9):
+            achieved = flops[dominant] / secs / 1e12
+            roof = {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": tc_peak,
+                    "unit": "TFLOP/s", "frac": achieved / tc_peak, "traffic": ncu_traffic(tag, cfg.name),
+                    "algorithmic_flops_per_launch": flops[dominant],
+                    "algorithmic_bytes_per_launch": alg[dominant]}
+        else:
+            achieved = alg[dominant] / secs / 1e9
+            roof = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": achieved / hbm_peak, "traffic": ncu_traffic(tag, cfg.name),
+                    "algorithmic_bytes_per_launch": alg[dominant]}
+        roof.update({"ms_per_launch": per_kernel_ms[dominant], "peak_source": peak_src})
+        layer_bytes = touched * (self.gu_b + self.dn_b) + E * H * 4 + 4 * T * H
+        fpt = flops_per_token(cfg)
+        t_hbm = layer_bytes / (hbm_peak * 1e9)
+        t_tc = T * fpt / (tc_peak * 1e12)
+        if self.decode:
+            # one kernel is the whole step: its algorithmic bytes are the layer's
+            achieved = layer_bytes / (ms_step * 1e-3) / 1e9
+            roof = {"bound": "hbm", "kernel": "decode_layer", "achieved": achieved, "peak": hbm_peak,
+                    "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": ncu_traffic("decode", cfg.name),
+                    "algorithmic_bytes_per_launch": layer_bytes, "ms_per_launch": ms_step, "peak_source": peak_src}
+        layer_roof = {"bound": "hbm" if t_hbm >= t_tc else "tensor", "roofline_ms": 1e3 * max(t_hbm, t_tc),
+                      "frac": 1e3 * max(t_hbm, t_tc) / ms_step, "bytes": layer_bytes, "flops": T * fpt,
+                      "hbm_gbs_achieved": layer_bytes / (ms_step * 1e-3) / 1e9,
+                      "tflops_achieved": T * fpt / (ms_step * 1e-3) / 1e12}
+        return roof, layer_roof
+
+    def l2_note(self, touched):
+        mb = touched * (self.gu_b + self.dn_b) / 1e6
+        if self.flush is not None:
+            return "flushed before each timed step (256 MB write); a step reads %.0f MB of weights" % mb
+        return "inputs larger than L2 (a step reads %.0f MB of expert weights)" % mb
+
+
+def stats_of(per):
+    return {"median": statistics.median(per), "p10": pct(per, 10), "p90": pct(per, 90),
+            "mean": statistics.mean(per), "n": len(per)}
+
+
+def extra_config(name, dev, stream, steps, warmup, decode):
+    """A shorter measurement of another workload (rank 0, N = 1): per-step
+    device time (median, p10, p90), tokens/s at the median, the dominant
+    GEMM's and the layer's roofline fractions."""
+    import synth
+    import torch
+    cfg = synth.get_config(name)
+    b = Bench(cfg, dev, stream, decode=decode)
+    for _ in range(warmup):
+        b.step()
+    torch.cuda.synchronize(dev)
+    b.check_status("after warm-up")
+    per, _ = b.timed(b.step, steps)
+    b.check_status("in the timed steps")
+    med = statistics.median(per)
+    kms, touched = b.per_kernel(min(steps, 10))
+    roof, layer_roof = b.rooflines(med, kms, touched)
+    out = {"T": cfg.T, "weights": WFMT_NAMES[cfg.wfmt], "path": "fused decode kernel" if b.decode else "kernel chain",
+           "ms_per_step": stats_of(per), "tokens_per_s": cfg.T / (med * 1e-3),
+           "tflops": cfg.T * flops_per_token(cfg) / (med * 1e-3) / 1e12,
+           "roofline": roof, "layer_roofline": layer_roof, "per_kernel_ms": kms,
+           "experts_touched": touched, "l2": b.l2_note(touched)}
+    del b
+    torch.cuda.empty_cache()
+    return out
+
+
+DEFAULT_EXTRAS = ("a3b_t512", "a3b_t4096_q4k", "a3b_decode_t1", "a3b_decode_t8", "a3b_decode_t32")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="a3b_t512")
+    ap.add_argument("--config", default="a3b_t8192_zipf")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-sample", type=int, default=8, help="tokens per oracle step (reference arm)")
-    ap.add_argument("--cpu-sample", type=int, default=96, help="tokens of the CPU-baseline sample")
+    ap.add_argument("--cpu-sample", type=int, default=256, help="tokens of the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", action="store_true", help="short run for ncu: no e2e / cpu legs")
+    ap.add_argument("--no-extras", action="store_true", help="skip the other workloads (N = 1 only)")
+    ap.add_argument("--profile", action="store_true", help="short run for ncu: no e2e / cpu / extra legs")
     ap.add_argument("--decode", action="store_true", help="T <= 8 through the fused decode kernel")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if not args.profile else args.warmup
@@ -257,7 +479,6 @@ def main():
 
     import torch
     import quantized_moe_expert_warp_b200 as mq
-    from quantized_moe_expert_warp_b200.host import upload_layer, x_to_device
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -266,58 +487,15 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    # every rank: the same layer weights, its own tokens
-    rcfg = replica_config(cfg, rank)
-    layer = synth.make_layer(rcfg)
-    packed = upload_layer(layer, dev)
-    T, H, E, k = cfg.T, cfg.H, cfg.E, cfg.k
-    x = x_to_device(layer["x"], dev)
-    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
-    # --decode: batches of T <= 8 through the fused single-kernel layer (measured
-    # slower than the kernel chain so far, so the chain is the default)
-    decode = args.decode and mq.moe_layer_decode_workspace_size(cfg, T) > 0
-    layer_call = mq.moe_layer_decode if decode else mq.moe_layer_forward
-    nbytes = mq.moe_layer_decode_workspace_size(cfg, T) if decode else mq.moe_layer_workspace_size(cfg, T)
-    ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
-
-    def step():
-        layer_call(packed, x, T, y, ws, nbytes, stream)
-
-    # When one step reads less than twice the L2 (126 MB), L2 is flushed
-    # (a 256 MB write) before every timed step and only the steps are timed;
-    # otherwise the step's own weights already exceed L2.
-    gu_b, dn_b = expert_bytes(cfg)
-    step_bytes_bound = min(T * k + 1, E + 1) * (gu_b + dn_b)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if step_bytes_bound < 2 * L2_BYTES else None
-
-    def timed_steps(fn, n):
-        """Mean device ms of n calls of fn: one event pair around all of
-        them, or (with the L2 flush) around each one."""
-        if flush is None:
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(n):
-                fn()
-            b.record(stream)
-            b.synchronize()
-            return a.elapsed_time(b) / n
-        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
-        for i in range(n):
-            flush.fill_(i & 0xFF)
-            pairs[i][0].record(stream)
-            fn()
-            pairs[i][1].record(stream)
-        pairs[-1][1].synchronize()
-        return sum(a.elapsed_time(b) for a, b in pairs) / n
+    # every rank: the same layer weights, its own tokens
+    b = Bench(cfg, dev, stream, rank=rank, decode=args.decode)
+    T, H = cfg.T, cfg.H
 
     for _ in range(args.warmup):
-        step()
+        b.step()
     torch.cuda.synchronize(dev)
-    st, det = mq.moe_read_status(ws, stream)
-    if st != 0:
-        raise RuntimeError(f"device status {st} ({det}) after warm-up")
+    b.check_status("after warm-up")
 
     # ---------------------------------------------------------- timed region
     sampler = ClockSampler(local)
@@ -325,7 +503,7 @@ def main():
         barrier(world)
         torch.cuda.synchronize(dev)
         launches0 = mq.moe_kernel_launches()
-        ms = timed_steps(step, args.steps)
+        per, total_ms = b.timed(b.step, args.steps)
         launches = mq.moe_kernel_launches() - launches0
         torch.cuda.synchronize(dev)
         barrier(world)
@@ -334,135 +512,60 @@ def main():
         t_end = time.perf_counter() + (0.5 if not args.profile else 0.0)
         while time.perf_counter() < t_end:
             for _ in range(20):
-                step()
+                b.step()
             torch.cuda.synchronize(dev)
+    ms = total_ms / args.steps
     ms_max = max_over_ranks(ms, world, dev)
-    st, det = mq.moe_read_status(ws, stream)
-    if st != 0:
-        raise RuntimeError(f"device status {st} ({det}) in the timed region")
+    b.check_status("in the timed region")
 
     value = world * T / (ms_max * 1e-3)
     fpt = flops_per_token(cfg)
     tflops = value * fpt / 1e12
 
-    # ------------------------------------------- per-kernel times (same stream)
-    # the composed path (same kernels as the fused call), events between steps
-    e32 = lambda *s: torch.empty(s, dtype=torch.float32, device=dev)
-    i32 = lambda *s: torch.empty(s, dtype=torch.int32, device=dev)
-    logits, gl, ids, tw = e32(T, E), e32(T), i32(T, k), e32(T, k)
-    counts, offsets, ss, dp = i32(E), i32(E + 1), i32(T * k), i32(T * k)
-    pn = mq.moe_permute_workspace_size(T, E, k)
-    pws = torch.zeros(pn, dtype=torch.uint8, device=dev)
-    rn = mq.moe_router_workspace_size(cfg, T)
-    rws = torch.zeros(rn, dtype=torch.uint8, device=dev)
-    fn = mq.moe_expert_ffn_workspace_size(cfg, T)
-    fws = torch.zeros(fn, dtype=torch.uint8, device=dev)
-    h = torch.empty((T * k + T, cfg.I), dtype=torch.bfloat16, device=dev)
-    y_perm = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
-    sh = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-    names = ["router_logits", "route", "permute", "gate_up_gemm", "down_gemm", "combine"]
-    calls = [
-        lambda: mq.moe_router_logits(packed, x, T, logits, gl, rws, rn, stream),
-        lambda: mq.moe_route(logits, T, E, k, cfg.renorm, ids, tw, stream),
-        lambda: mq.moe_permute(ids, T, E, k, counts, offsets, ss, dp, pws, pn, stream),
-        lambda: mq.moe_expert_gate_up_q4(packed, x, T, ss, offsets, h, fws, fn, stream),
-        lambda: mq.moe_expert_down_q4(packed, h, T, offsets, y_perm, sh, fws, fn, stream),
-        lambda: mq.moe_combine(y_perm, dp, tw, sh, gl, T, H, k, y, stream),
-    ]
-    for _ in range(2):
-        for c in calls:
-            c()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(args.steps)]
-    torch.cuda.synchronize(dev)
-    for s in range(args.steps):
-        if flush is not None:
-            flush.fill_(s & 0xFF)
-        evs[s][0].record(stream)
-        for i, c in enumerate(calls):
-            c()
-            evs[s][i + 1].record(stream)
-    torch.cuda.synchronize(dev)
-    per_kernel_ms = {n: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps))
-                     for i, n in enumerate(names)}
-    composed_ms = sum(per_kernel_ms.values())
-    touched = int((counts.cpu().numpy() > 0).sum()) + (1 if cfg.has_shared else 0)
-    alg = {
-        "gate_up_gemm": touched * gu_b + 2 * T * H,
-        "down_gemm": touched * dn_b,
-    }
-    dominant = max(("gate_up_gemm", "down_gemm"), key=lambda n: per_kernel_ms[n])
-    peaks = {}
-    mp = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(mp):
-        peaks = json.load(open(mp))
-    hbm_peak = peaks.get("hbm_gbs")
-    peak_src = "measured"
-    if not hbm_peak:
-        hbm_peak, peak_src = 6650.0, "fallback"
-    tag = {"gate_up_gemm": "gate_up", "down_gemm": "down"}[dominant]
-    # the kernel's own roofline: the slower of its bytes at HBM peak and its
-    # FLOPs at the bf16 tensor peak (burst figure: each kernel is timed alone)
-    rows = T * cfg.k + (T if cfg.has_shared else 0)
-    flops_k = {"gate_up_gemm": 2.0 * rows * 2 * cfg.I * H, "down_gemm": 2.0 * rows * H * cfg.I}[dominant]
-    tc_peak = peaks.get("bf16_tflops") or 1590.0
-    t_hbm = alg[dominant] / (hbm_peak * 1e9)
-    t_tc = flops_k / (tc_peak * 1e12)
-    secs = per_kernel_ms[dominant] * 1e-3
-    if t_tc > t_hbm:
-        achieved = flops_k / secs / 1e12
-        roofline = {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": tc_peak,
-                    "unit": "TFLOP/s", "frac": achieved / tc_peak, "traffic": ncu_traffic(tag, cfg.name),
-                    "algorithmic_flops_per_launch": flops_k, "algorithmic_bytes_per_launch": alg[dominant],
-                    "ms_per_launch": per_kernel_ms[dominant], "peak_source": peak_src}
-    else:
-        achieved = alg[dominant] / secs / 1e9
-        roofline = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": achieved / hbm_peak, "traffic": ncu_traffic(tag, cfg.name),
-                    "algorithmic_bytes_per_launch": alg[dominant], "ms_per_launch": per_kernel_ms[dominant],
-                    "peak_source": peak_src}
-    # whole-layer roofline: max(FLOPs at tensor peak, bytes at HBM peak)
-    layer_bytes = touched * (gu_b + dn_b) + E * H * 4 + 4 * T * H
-    if decode:
-        # one kernel is the whole step: its algorithmic bytes are the layer's
-        achieved = layer_bytes / (ms * 1e-3) / 1e9
-        roofline = {"bound": "hbm", "kernel": "decode_layer", "achieved": achieved, "peak": hbm_peak,
-                    "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": ncu_traffic("decode", cfg.name),
-                    "algorithmic_bytes_per_launch": layer_bytes, "ms_per_launch": ms, "peak_source": peak_src}
-    t_hbm = layer_bytes / (hbm_peak * 1e9)
-    tc_peak = peaks.get("bf16_tflops", 1590.0)
-    t_tc = T * fpt / (tc_peak * 1e12)
-    layer_roof = {"bound": "hbm" if t_hbm >= t_tc else "tensor", "roofline_ms": 1e3 * max(t_hbm, t_tc),
-                  "frac": 1e3 * max(t_hbm, t_tc) / ms, "bytes": layer_bytes, "flops": T * fpt,
-                  "hbm_gbs_achieved": layer_bytes / (ms * 1e-3) / 1e9}
+    per_kernel_ms, touched = b.per_kernel(args.steps)
+    roofline, layer_roof = b.rooflines(ms, per_kernel_ms, touched)
 
     # ------------------------------------------------------------------ e2e
     e2e = None
     if not args.profile:
-        x_host = torch.from_numpy(np.ascontiguousarray(layer["x"]).view(np.int16)).pin_memory()
+        x_host = torch.from_numpy(np.ascontiguousarray(b.layer["x"]).view(np.int16)).pin_memory()
         y_host = torch.empty((T, H), dtype=torch.int16).pin_memory()
         x_in = torch.empty((T, H), dtype=torch.int16, device=dev)
         y_out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
 
         def e2e_step():
             x_in.copy_(x_host, non_blocking=True)
-            layer_call(packed, x_in, T, y_out, ws, nbytes, stream)
+            b.call(b.packed, x_in, T, y_out, b.ws, b.nbytes, stream)
             y_host.copy_(y_out.view(torch.int16), non_blocking=True)
 
         for _ in range(3):
             e2e_step()
         torch.cuda.synchronize(dev)
         barrier(world)
-        e_ms = max_over_ranks(timed_steps(e2e_step, args.steps), world, dev)
+        _, e_total = b.timed(e2e_step, args.steps)
+        e_ms = max_over_ranks(e_total / args.steps, world, dev)
         e2e = {"value": world * T / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
                "d2h_bytes_per_step": T * H * 2, "ms_per_step": e_ms}
+
+    # ------------------------------------------------ other workloads (N = 1)
+    extras = None
+    if rank == 0 and world == 1 and not args.profile and not args.no_extras:
+        extras = {}
+        for name in DEFAULT_EXTRAS:
+            if name == cfg.name:
+                continue
+            extras[name] = extra_config(name, dev, stream, min(args.steps, 30), args.warmup, decode=False)
+            if synth.get_config(name).T <= 8:
+                extras[name + "_fused"] = extra_config(name, dev, stream, min(args.steps, 30), args.warmup,
+                                                       decode=True)
 
     # ---------------------------------------------------------- cpu baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
         n = min(args.cpu_sample, T)
-        rate, dt = oracle_sample_rate(layer, n)
-        cpu = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-               "sample": f"first {n} of {T} tokens ({dt:.1f} s; routing and permutation of all {T})"}
+        rate, dt = oracle_sample_rate(b.layer, n)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": 1, "host_cores": host_cores(), "kind": "oracle",
+               "sample": f"first {n} of {T} tokens run as their own batch ({dt:.1f} s on one host thread)"}
 
     if rank == 0:
         line = {
@@ -470,20 +573,19 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": f"synthetic (seeded N(0,1) bf16 activations; N(0,0.02) weights, {WFMT_NAMES[cfg.wfmt]} quantised)",
-            "config": {"workload": cfg.name, "T": T, "H": H, "E": E, "k": k, "I": cfg.I,
+            "config": {"workload": cfg.name, "T": T, "H": H, "E": cfg.E, "k": cfg.k, "I": cfg.I,
                        "shared_expert": bool(cfg.has_shared), "weights": WFMT_NAMES[cfg.wfmt],
-                       "G": cfg.G, "tokens_per_rank": T, "parallelism": f"replicas x{world} (token-sharded)",
-                       "path": "fused decode kernel" if decode else "kernel chain",
-                       "l2": ("flushed before each timed step (256 MB write); a step reads %.0f MB of weights"
-                              % (touched * (gu_b + dn_b) / 1e6)) if flush is not None else
-                             ("inputs larger than L2 (a step reads %.0f MB of expert weights)"
-                              % (touched * (gu_b + dn_b) / 1e6))},
+                       "G": cfg.G, "zipf_s": cfg.zipf_s, "tokens_per_rank": T,
+                       "parallelism": f"replicas x{world} (token-sharded)",
+                       "path": "fused decode kernel" if b.decode else "kernel chain", "l2": b.l2_note(touched)},
+            "ms_per_step_stats": stats_of(per),
             "tflops": tflops, "flop_per_token": fpt,
             "roofline": roofline, "layer_roofline": layer_roof,
-            "per_kernel_ms": per_kernel_ms, "composed_ms_per_step": composed_ms,
+            "per_kernel_ms": per_kernel_ms, "composed_ms_per_step": sum(per_kernel_ms.values()),
             "experts_touched": touched,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": sampler.summary(),
+            "extra_configs": extras,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -334,6 +334,18 @@ int moe_layer_decode(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *y
  * moe_permute; clearing zeroes the workspace's whole 256-byte status block.
  * Synchronises `stream`.  *status = MOE_OK or the first MOE_ERR_* code a
  * kernel recorded; *detail (optional) = where it was recorded.
+ *
+ * The status block (the first 256 bytes of those workspaces), as int32
+ * words: [0] status, [1] detail, [16..18] the decode kernel's grid barrier
+ * (count, generation, abort flag), [20] the wait budget in microseconds of
+ * every bounded device wait of the kernels reading this workspace (0: 2 s;
+ * a wait that runs out records MOE_ERR_TIMEOUT and its kernel returns with
+ * its TMEM freed and its copies landed), [21] a test knob of
+ * moe_layer_decode: c > 0 makes CTA c - 1 withhold its arrival at the first
+ * grid barrier, so that the budget runs out (for testing the timeout path;
+ * keep it 0).  Other words are reserved and must stay zero.  The caller may
+ * set words 20 and 21 with a device copy before a call; clearing resets
+ * them.
  */
 int moe_read_status(void *ws, void *stream, int clear, int *status, int *detail);
 

@@ -86,9 +86,17 @@ __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes)
 
 // Grid barrier over all CTAs of a cooperative launch.  bar[0] counts
 // arrivals (back to 0 after every barrier), bar[1] is the generation,
-// bar[2] the abort flag.  Waits are bounded: on timeout the CTA records
+// bar[2] the abort flag.  Waits are bounded by the workspace's wait budget
+// (status word 20, microseconds; 0 = 2 s): on timeout the CTA records
 // MOE_ERR_TIMEOUT, raises the abort flag (so the others stop waiting) and
 // the caller returns.  Returns false when the kernel must stop.
+//
+// Test knob, status word 21: when it holds c > 0, CTA c - 1 waits at the
+// first barrier without arriving, so that every CTA's wait runs out of its
+// budget (the way a lost arrival would); the kernel then returns with
+// MOE_ERR_TIMEOUT and a usable context.
+constexpr int kStatusSkipArrivalWord = 21;
+
 __device__ bool grid_sync(unsigned *bar, int *status, int where, int *s_flag)
 {
     __syncthreads();
@@ -96,20 +104,22 @@ __device__ bool grid_sync(unsigned *bar, int *status, int where, int *s_flag)
         int ok = 1;
         __threadfence();
         const unsigned gen = ld_acquire(bar + 1);   // read before arriving: it cannot move until we do
-        const unsigned prev = atomicAdd(bar, 1u);
-        if (prev == gridDim.x - 1) {
+        const bool skip = where == 91 && status &&
+                          *(const volatile int *)(status + kStatusSkipArrivalWord) == (int)blockIdx.x + 1;
+        const unsigned prev = skip ? 0u : atomicAdd(bar, 1u);
+        if (!skip && prev == gridDim.x - 1) {
             atomicExch(bar, 0u);
             __threadfence();
             st_release(bar + 1, gen + 1);
         } else {
-            const uint64_t t0 = globaltimer_ns();
+            const uint64_t t0 = globaltimer_ns(), limit = wait_limit_ns(status);
             uint32_t spins = 0;
             while (ld_acquire(bar + 1) == gen) {
                 if (ld_relaxed(bar + 2)) {
                     ok = 0;
                     break;
                 }
-                if ((++spins & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+                if ((++spins & 63u) == 0 && globaltimer_ns() - t0 > limit) {
                     atomicExch(bar + 2, 1u);
                     record_error(status, MOE_ERR_TIMEOUT, where);
                     ok = 0;

@@ -20,7 +20,9 @@
 // exact in fp32 and accumulate into one fp32 accumulator.
 //
 // Warp roles of one persistent CTA (one per SM, 768 threads):
-//   warp 0      gathers token rows of B with cp.async (zero rows past the tail)
+//   warp 0      loads token rows of B: gate/up gathers them with cp.async
+//               (zero rows past the tail); down reads contiguous rows of h
+//               with one tiled TMA copy per k-step
 //   warp 1      issues tcgen05.mma (one thread) and commits stage releases
 //   warp 2      streams code blocks and per-tile scale blocks with bulk copies
 //   warp 3      owns the TMEM allocation; in the router pass it also forms
@@ -31,6 +33,8 @@
 // Every wait is bounded; on timeout the CTA records MOE_ERR_TIMEOUT and
 // unwinds.
 #include <cstdint>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #ifdef MOEQ4_TRACE
@@ -99,6 +103,12 @@ constexpr int kMaxAStages = 8;   // TMEM A-operand ring depth (dequantised k-ste
 #ifndef MOEQ4_A_STAGES_DN
 #define MOEQ4_A_STAGES_DN 8
 #endif
+#ifndef MOEQ4_B_STAGES_64
+#define MOEQ4_B_STAGES_64 8
+#endif
+#ifndef MOEQ4_B_STAGES_128
+#define MOEQ4_B_STAGES_128 4
+#endif
 constexpr int kMaxCodeChunks = 8;   // code ring: chunks of several k-steps, one bulk copy each
 constexpr int kMaxMetaBufs = 4;
 constexpr int kEpiTok = 16;  // tokens per epilogue chunk
@@ -140,12 +150,18 @@ struct Geo {
     static constexpr int kCodeBlock = kNCode ? code_block_bytes(kNCode) : 0;
     // the gathered token rows wait on L2 / HBM latency, so their shared-memory
     // ring is deeper than the TMEM ring
-    static constexpr int kBStages = BN == 64 ? 8 : 4;
+    static constexpr int kBStages = BN == 64 ? MOEQ4_B_STAGES_64 : BN == 128 ? MOEQ4_B_STAGES_128 : 4;
+    static_assert(kBStages <= 8, "B stages");
+    // 256-token tiles only for the down pass: one accumulator of 256 columns
+    // leaves room for eight A stages
+    static_assert(BN != 256 || MODE == MODE_DOWN, "256-token tiles: down pass only");
     static constexpr int kBBytes = kBStages * BN * 128;
     static constexpr int kAccCols = kAccBufs * kNAcc * BN;
     static constexpr int kTmemCols = 512;
     static_assert(kAccCols + kAStages * kNA * 32 <= kTmemCols, "TMEM budget");
     static constexpr bool kGather = MODE == MODE_GATE_UP;
+    // the down pass's token rows are contiguous rows of h: one TMA tile per k-step
+    static constexpr bool kTmaB = MODE == MODE_DOWN;
 };
 
 struct Barriers {
@@ -277,8 +293,23 @@ __device__ __forceinline__ void split2(float w0, float w1, uint32_t &hi, uint32_
     lo = pack_bf16x2(r0, r1);
 }
 
+// A producer that stops early (a wait ran out, or another role gave up)
+// still waits, with a fresh bounded budget, until the copies it issued have
+// landed, so that none writes into this CTA's shared memory after it exits:
+// the last `depth` of the n_issued ring slots it filled.  On the normal path
+// every such phase has completed already.
+__device__ __forceinline__ void drain_ring(uint64_t *full, int n_issued, int depth, int *status, int where,
+                                           int *never_abort)
+{
+    WaitCtx wd{never_abort, status, globaltimer_ns(), kWaitLimitNs};
+    for (int i = max(0, n_issued - depth); i < n_issued; ++i)
+        if (!warp_wait(&full[i % depth], (i / depth) & 1, wd, where))
+            break;
+}
+
 template <int MODE, int WFMT, int BN>
-__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArgs p)
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ GemmArgs p, const __grid_constant__ CUtensorMap tmap_b)
 {
     using L = Geo<MODE, BN>;
     constexpr int kBN = BN;
@@ -313,7 +344,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
             mbar_init(&bars->a_empty[s], 1);
         }
         for (int s = 0; s < L::kBStages; ++s) {
-            mbar_init(&bars->b_full[s], 32);   // one cp.async completion arrival per lane of the B producer
+            // gather: one cp.async completion arrival per lane of the B producer;
+            // TMA: one arrival with the stage's byte count
+            mbar_init(&bars->b_full[s], L::kTmaB ? 1 : 32);
             mbar_init(&bars->b_empty[s], 1);
         }
         for (int s = 0; s < NCS; ++s) {
@@ -348,10 +381,36 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
 
     const int total_units = s_tile_start[p.E_total] * p.F * p.ksplit;
     const int KS = p.K / kKStep;
-    WaitCtx wc{&bars->abort_flag, p.status, globaltimer_ns()};
+    WaitCtx wc{&bars->abort_flag, p.status, globaltimer_ns(), wait_limit_ns(p.status)};
     CYC_DECL
 
-    if (warp == 0) {
+    if (warp == 0 && L::kTmaB) {
+        // ------------------------------------------------ B producer (TMA tiles of contiguous rows)
+        // A tile of BN rows from the unit's first row: rows of the next
+        // expert only feed MMA columns the epilogue discards, rows past the
+        // end of h arrive as zeros.
+        if (elect_one())
+            tma_prefetch_desc(&tmap_b);
+        __syncwarp();
+        int step = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+            const Unit un = decode_unit<BN>(u, p, sched);
+            for (int ks = un.ks0; ks < un.ks0 + un.nks; ++ks, ++step) {
+                const int s = step % L::kBStages;
+                if (step >= L::kBStages && !warp_wait(&bars->b_empty[s], ((step / L::kBStages) & 1) ^ 1, wc, 1)) {
+                    ok = false;
+                    break;
+                }
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&bars->b_full[s], (uint32_t)(kBN * 128));
+                    tma_load_2d(sB + s * kBN * 128, &tmap_b, ks * kKStep, un.row0, &bars->b_full[s]);
+                }
+                __syncwarp();
+            }
+        }
+        drain_ring(bars->b_full, step, L::kBStages, p.status, 12, &bars->never_abort);
+    } else if (warp == 0) {
         // ------------------------------------------------ B producer (cp.async row gather)
         int step = 0;
         bool ok = true;
@@ -396,6 +455,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                     TRACE_OTHER(0, step);
             }
         }
+        cp_async_wait_group<0>();
+        __syncwarp();
+        drain_ring(bars->b_full, step, L::kBStages, p.status, 12, &bars->never_abort);
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (converged warp, one elected lane)
         int step = 0, uidx = 0;
@@ -464,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
         if (elect_one())
             mma_commit(&bars->drain);
         __syncwarp();
-        WaitCtx wd{&bars->never_abort, p.status, globaltimer_ns()};   // drain even after an abort
+        WaitCtx wd{&bars->never_abort, p.status, globaltimer_ns(), kWaitLimitNs};   // drain even after an abort
         warp_wait(&bars->drain, 0, wd, 5);
     } else if (warp == 2) {
         // ------------------------------------------------ code / meta producer (converged warp)
@@ -472,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
         // copy moves CK k-steps: the copy engine's throughput is set by the
         // number of copies more than by their size.
         if (MODE != MODE_ROUTER) {
-            int cidx = 0, munit = 0;
+            int cidx = 0, munit = 0, nmeta = 0;   // cidx: code chunks issued; nmeta: meta blocks issued
             bool ok = true;
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++munit) {
                 const Unit un = decode_unit<BN>(u, p, sched);
@@ -486,6 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                     bulk_g2s(sMeta + mb * meta_al, p.wmeta + tile_id * meta_bytes, meta_bytes, &bars->meta_full[mb]);
                 }
                 __syncwarp();
+                ++nmeta;
                 for (int c0 = 0; c0 < KS; c0 += CK, ++cidx) {
                     const int s = cidx & (NCS - 1);
                     if (cidx >= NCS && !warp_wait(&bars->code_empty[s], ((cidx >> p.ncs_log2) & 1) ^ 1, wc, 7)) {
@@ -503,6 +566,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
                         TRACE_OTHER(1, cidx);
                 }
             }
+            drain_ring(bars->code_full, cidx, NCS, p.status, 13, &bars->never_abort);
+            drain_ring(bars->meta_full, nmeta, NMETA, p.status, 14, &bars->never_abort);
         }
     } else if (warp == 3) {
 #ifdef MOEQ4_TRACE
@@ -909,10 +974,51 @@ static Rings gemm_rings(int meta_bytes, int E_total, int KS)
     return r;
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda); null if the driver does not provide it.
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+        return (PFN_cuTensorMapEncodeTiled_v12000)f;
+    }();
+    return fn;
+}
+
+// Tensor map of the B rows (bf16 [b_rows, ldb], row-major) in tiles of
+// 64 elements (128 bytes, 128-byte swizzle: the MMA's K-major layout) by
+// BN rows.
+static cudaError_t encode_b_map(CUtensorMap *m, const GemmArgs &a, int bn)
+{
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc)
+        return cudaErrorNotSupported;
+    if ((reinterpret_cast<uintptr_t>(a.b_src) & 15) || a.b_rows < 1 || ((size_t)a.ldb * 2) % 16)
+        return cudaErrorInvalidValue;
+    const cuuint64_t dims[2] = {(cuuint64_t)a.ldb, (cuuint64_t)a.b_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)a.ldb * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kKStep, (cuuint32_t)bn};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(a.b_src), dims, strides,
+                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int MODE, int WFMT, int BN>
 static cudaError_t launch_one(const GemmArgs &a_in, int num_sms, cudaStream_t st)
 {
     auto kern = grouped_gemm_kernel<MODE, WFMT, BN>;
+    CUtensorMap tmap{};
+    if (Geo<MODE, BN>::kTmaB) {
+        const cudaError_t e = encode_b_map(&tmap, a_in, BN);
+        if (e != cudaSuccess)
+            return e;
+    }
     GemmArgs a = a_in;
     if (a.ksplit < 1)
         a.ksplit = 1;
@@ -926,7 +1032,7 @@ static cudaError_t launch_one(const GemmArgs &a_in, int num_sms, cudaStream_t st
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
-    return launch_pdl(kern, num_sms, kThreads, smem, st, a);
+    return launch_pdl(kern, num_sms, kThreads, smem, st, a, tmap);
 }
 
 size_t gemm_smem_required(int nmat, int meta_bytes, int E_total)
@@ -936,7 +1042,7 @@ size_t gemm_smem_required(int nmat, int meta_bytes, int E_total)
     const size_t a = nmat == 2 ? gemm_smem_bytes<MODE_GATE_UP, 64>(meta_bytes, E_total, r)
                                : gemm_smem_bytes<MODE_DOWN, 64>(meta_bytes, E_total, r);
     const size_t b = nmat == 2 ? gemm_smem_bytes<MODE_GATE_UP, 128>(meta_bytes, E_total, r)
-                               : gemm_smem_bytes<MODE_DOWN, 128>(meta_bytes, E_total, r);
+                               : gemm_smem_bytes<MODE_DOWN, 256>(meta_bytes, E_total, r);
     return a > b ? a : b;
 }
 
@@ -958,6 +1064,17 @@ int router_ksplit(int T, int E, int H, int sms)
 
 int gemm_tile_tokens(int T, int E, int k) { return (long long)T * k <= 64LL * E ? 64 : 128; }
 
+// The down pass reads its token rows with TMA and has a single matrix, so
+// when experts average at least 128 rows it takes 256-token tiles: twice the
+// MMA work per dequantised k-step and per pipeline round trip.
+#ifndef MOEQ4_DOWN_TILE_MAX
+#define MOEQ4_DOWN_TILE_MAX 256
+#endif
+int gemm_down_tile_tokens(int T, int E, int k)
+{
+    return MOEQ4_DOWN_TILE_MAX >= 256 && (long long)T * k >= 128LL * E ? 256 : gemm_tile_tokens(T, E, k);
+}
+
 template <int MODE, int BN>
 static cudaError_t launch_fmt(const GemmArgs &a, int wfmt, int num_sms, cudaStream_t st)
 {
@@ -971,8 +1088,9 @@ cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int tile_
     if (nmat == 2)
         return tile_tokens == 64 ? launch_fmt<MODE_GATE_UP, 64>(a, wfmt, num_sms, st)
                                  : launch_fmt<MODE_GATE_UP, 128>(a, wfmt, num_sms, st);
-    return tile_tokens == 64 ? launch_fmt<MODE_DOWN, 64>(a, wfmt, num_sms, st)
-                             : launch_fmt<MODE_DOWN, 128>(a, wfmt, num_sms, st);
+    return tile_tokens == 64    ? launch_fmt<MODE_DOWN, 64>(a, wfmt, num_sms, st)
+           : tile_tokens == 128 ? launch_fmt<MODE_DOWN, 128>(a, wfmt, num_sms, st)
+                                : launch_fmt<MODE_DOWN, 256>(a, wfmt, num_sms, st);
 }
 
 // Router logits on tensor cores: logits[t, e] = x[t] . Wr[e] (+ bias[e]),

@@ -72,9 +72,11 @@ struct GemmArgs {
     int *status;                // [code, detail]
 };
 
-// Token-tile width of the grouped GEMMs: 64 when experts average at most 64
-// rows (T k <= 64 E), else 128.  Both passes of one FFN must use the same.
+// Token-tile width of the gate/up GEMM: 64 when experts average at most 64
+// rows (T k <= 64 E), else 128.
 int gemm_tile_tokens(int T, int E, int k);
+// Token-tile width of the down pass: 256 when experts average >= 128 rows, else as above.
+int gemm_down_tile_tokens(int T, int E, int k);
 cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int tile_tokens, int num_sms, cudaStream_t st);
 size_t gemm_smem_required(int nmat, int meta_bytes, int E_total);
 

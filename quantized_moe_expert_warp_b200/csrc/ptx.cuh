@@ -82,7 +82,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
 #define MOEQ4_WAIT_HINT_NS 10000000
 #endif
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity, bool sleep = true)
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity, bool sleep = true,
+                                              uint32_t hint_ns = (uint32_t)MOEQ4_WAIT_HINT_NS)
 {
     uint32_t ok;
 #if MOEQ4_WAIT_HINT_NS > 0
@@ -101,7 +102,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity, bo
         "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"((uint32_t)MOEQ4_WAIT_HINT_NS)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
         : "memory");
 #else
     asm volatile(
@@ -121,6 +122,7 @@ struct WaitCtx {
     volatile int *abort_flag;   // shared memory
     int *status;                // global status words [code, detail] (may be null)
     uint64_t t0;
+    uint64_t limit;             // ns after t0 at which a wait gives up
 #ifdef MOEQ4_TRACE
     uint32_t polls[16] = {};    // failed polls per call site (instrumented builds)
     uint32_t waits[16] = {};    // waits per call site that polled more than once
@@ -157,6 +159,16 @@ struct WaitCtx {
 #endif
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: kernels here take well under 10 ms
+// Word of a workspace's status block holding the caller's wait budget in
+// microseconds (0: the 2 s default).
+constexpr int kStatusWaitLimitWord = 20;
+
+// The wait budget of a launch: the status block's word, else 2 s.
+__device__ __forceinline__ uint64_t wait_limit_ns(const int *status)
+{
+    const int us = status ? *(const volatile int *)(status + kStatusWaitLimitWord) : 0;
+    return us > 0 ? (uint64_t)us * 1000ull : kWaitLimitNs;
+}
 // failed try_waits between clock reads: each one may already have slept up to the hint
 constexpr uint32_t kClockEvery = MOEQ4_WAIT_HINT_NS > 0 ? 1u : 64u;
 
@@ -221,7 +233,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, WaitCt
         if (lds_volatile_s32(smem_u32((const void *)w.abort_flag)))
             return false;
         ns = ns * 2 < ns_max ? ns * 2 : ns_max;
-        if ((++spins & 15u) == 0 && globaltimer_ns() - w.t0 > kWaitLimitNs) {
+        if ((++spins & 15u) == 0 && globaltimer_ns() - w.t0 > w.limit) {
             *w.abort_flag = 1;
             if (w.status && atomicCAS(w.status, 0, MOE_ERR_TIMEOUT) == 0)
                 w.status[1] = where;
@@ -230,11 +242,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, WaitCt
     }
 #else
     const bool sleep = !((MOEQ4_NOHINT_SITES >> where) & 1u);
-    if (mbar_try_wait(bar, parity, sleep))
+    // a suspended try_wait returns at the latest after its hint, so the hint
+    // is capped at the budget: the budget is then checked at least that often
+    const uint32_t hint = (uint32_t)(w.limit < (uint64_t)MOEQ4_WAIT_HINT_NS ? w.limit : (uint64_t)MOEQ4_WAIT_HINT_NS);
+    if (mbar_try_wait(bar, parity, sleep, hint))
         return true;
     uint32_t spins = 0;
     while (true) {
-        if (mbar_try_wait(bar, parity, sleep)) {
+        if (mbar_try_wait(bar, parity, sleep, hint)) {
             MOEQ4_WAIT_HOOK(where, spins);
             return true;
         }
@@ -243,7 +258,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, WaitCt
         if ((MOEQ4_BACKOFF_SITES >> where) & 1u)
             __nanosleep(MOEQ4_BACKOFF_NS);
         if (++spins % kClockEvery == 0) {
-            if (globaltimer_ns() - w.t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - w.t0 > w.limit) {
                 *w.abort_flag = 1;
                 if (w.status && atomicCAS(w.status, 0, MOE_ERR_TIMEOUT) == 0)
                     w.status[1] = where;
@@ -324,6 +339,24 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
             smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Tiled 2-D tensor copy global -> shared on the TMA engine (no multicast):
+// the box at element coordinates (x, y) of the tensor map, completion
+// counted in bytes on `bar`.  x * element size must be a multiple of 16
+// bytes; rows past the tensor's extent arrive as zeros.
+__device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int x, int y, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const void *tmap)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05
