@@ -340,10 +340,11 @@ int moe_layer_decode(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *y
  * (count, generation, abort flag), [20] the wait budget in microseconds of
  * every bounded device wait of the kernels reading this workspace (0: 2 s;
  * a wait that runs out records MOE_ERR_TIMEOUT and its kernel returns with
- * its TMEM freed and its copies landed), [21] a test knob of
- * moe_layer_decode: c > 0 makes CTA c - 1 withhold its arrival at the first
- * grid barrier, so that the budget runs out (for testing the timeout path;
- * keep it 0).  Other words are reserved and must stay zero.  The caller may
+ * its TMEM freed and its copies landed), [21] a test knob: c > 0 makes
+ * CTA c - 1 of every launch reading the block drop one of its own signals
+ * (moe_layer_decode: its arrival at the first grid barrier; the grouped
+ * expert GEMMs: its weight copies), so that waits run out of the budget
+ * (for testing the timeout path; keep it 0).  Other words are reserved and must stay zero.  The caller may
  * set words 20 and 21 with a device copy before a call; clearing resets
  * them.
  */

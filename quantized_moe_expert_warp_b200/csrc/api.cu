@@ -149,16 +149,23 @@ int e_total(const moe_config_t *c) { return c->E + (c->has_shared ? 1 : 0); }
 // ---------------------------------------------------------------- workspaces
 
 struct FfnWs {
-    uint16_t *h;
+    uint16_t *h;       // [T k (+ T), I] gate/up output
+    uint16_t *x_perm;  // [T k, H] token rows in permuted order (null when the caller lends a buffer)
     size_t bytes;
 };
 
-FfnWs ffn_layout(const moe_config_t *c, int T, uint8_t *base)
+// with_xperm = false: the caller lends the permuted-row buffer (the fused
+// layer lends y_perm, which is dead until the down pass writes it).
+FfnWs ffn_layout(const moe_config_t *c, int T, uint8_t *base, bool with_xperm = true)
 {
     FfnWs w{};
     size_t off = 0;
     w.h = (uint16_t *)(base + off);
     off += align256(sizeof(uint16_t) * ((size_t)T * c->k + (c->has_shared ? T : 0)) * c->I);
+    if (with_xperm) {
+        w.x_perm = (uint16_t *)(base + off);
+        off += align256(sizeof(uint16_t) * (size_t)T * c->k * c->H);
+    }
     w.bytes = off;
     return w;
 }
@@ -194,7 +201,7 @@ LayerWs layer_layout(const moe_config_t *c, int T, uint8_t *base)
     w.sorted_slot = (int32_t *)take(sizeof(int32_t) * Tk);
     w.dest_pos = (int32_t *)take(sizeof(int32_t) * Tk);
     w.perm_scratch = take(permute_scratch_bytes(T, c->E, c->k));
-    w.ffn = take(ffn_layout(c, T, nullptr).bytes);
+    w.ffn = take(ffn_layout(c, T, nullptr, false).bytes);
     w.y_perm = (uint16_t *)take(sizeof(uint16_t) * Tk * c->H);
     w.shared_out = (uint16_t *)take(sizeof(uint16_t) * (size_t)T * c->H);
     w.bytes = off;
@@ -207,7 +214,7 @@ LayerWs layer_layout(const moe_config_t *c, int T, uint8_t *base)
 struct DecodeWs {
     int *status;
     unsigned *bar;
-    float *logits, *gate_logit, *w, *h, *o;
+    float *logits, *gate_logit, *w, *h;
     int32_t *ids;
     size_t bytes;
 };
@@ -230,7 +237,6 @@ DecodeWs decode_layout(const moe_config_t *c, int T, uint8_t *base)
     w.ids = (int32_t *)take(sizeof(int32_t) * Tk);
     w.w = (float *)take(sizeof(float) * Tk);
     w.h = (float *)take(sizeof(float) * NP * c->I);
-    w.o = (float *)take(sizeof(float) * NP * c->H);
     w.bytes = off;
     return w;
 }
@@ -242,6 +248,8 @@ const char *decode_refusal(const moe_config_t *c, int T)
 {
     if (T > kDecodeMaxT)
         return "the fused decode kernel takes at most 8 tokens";
+    if (c->I > 1024)
+        return "the fused decode kernel takes an expert intermediate of at most 1024";
     if (decode_smem_layout(T, c->k, c->H, c->I, c->has_shared).bytes > kMaxDynamicSmem)
         return "x or the expert intermediates of this shape exceed shared memory";
     return nullptr;
@@ -271,14 +279,16 @@ int check_layer(const moe_layer_t *L)
 // (defaults to the one inside the FFN workspace).
 int run_expert_ffn(const moe_layer_t *L, const uint16_t *x, int T, const int32_t *sorted_slot,
                    const int32_t *offsets, uint16_t *y_perm, uint16_t *shared_out, uint8_t *ffn_ws, int *status,
-                   cudaStream_t st, int pass = 3, uint16_t *h = nullptr)
+                   cudaStream_t st, int pass = 3, uint16_t *h = nullptr, uint16_t *x_perm = nullptr)
 {
     const moe_config_t &c = L->cfg;
-    const FfnWs w = ffn_layout(&c, T, ffn_ws);
+    const FfnWs w = ffn_layout(&c, T, ffn_ws, x_perm == nullptr);
     const int Et = e_total(&c);
     const int Tk = T * c.k;
     if (!h)
         h = w.h;
+    if (!x_perm)
+        x_perm = w.x_perm;
     GemmArgs a{};
     a.sorted_slot = sorted_slot;
     a.topk = c.k;
@@ -290,12 +300,17 @@ int run_expert_ffn(const moe_layer_t *L, const uint16_t *x, int T, const int32_t
     a.G = c.G;
     a.status = status;
     if (pass & 1) {
+        // the routed experts' token rows, permuted into contiguous blocks
+        CUDA_TRY(launch_gather_rows(x, sorted_slot, Tk, c.k, c.H, x_perm, num_sms(), st), "gather rows");
+        g_launches += 1;
         // gate/up + SwiGLU -> h [Tk + T, I]
         a.wq = (const uint8_t *)L->gu_q;
         a.wmeta = (const uint8_t *)L->gu_meta;
-        a.b_src = x;
+        a.b_src = x_perm;
         a.ldb = c.H;
-        a.b_rows = T;
+        a.b_rows = Tk;
+        a.b_src2 = c.has_shared ? x : nullptr;
+        a.b_rows2 = T;
         a.K = c.H;
         a.F = c.I / kTileRows;
         a.meta_bytes = meta_block_bytes(2, c.wfmt, c.H, c.G);
@@ -312,6 +327,8 @@ int run_expert_ffn(const moe_layer_t *L, const uint16_t *x, int T, const int32_t
         a.b_src = h;
         a.ldb = c.I;
         a.b_rows = Tk + (c.has_shared ? T : 0);
+        a.b_src2 = nullptr;
+        a.b_rows2 = 0;
         a.K = c.I;
         a.F = c.H / kTileRows;
         a.meta_bytes = meta_block_bytes(1, c.wfmt, c.I, c.G);
@@ -676,7 +693,7 @@ int moe_layer_forward(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *
              "permute");
     g_launches += permute_launch_count(T, c.k);
     rc = run_expert_ffn(L, x, T, w.sorted_slot, w.offsets, w.y_perm, c.has_shared ? w.shared_out : nullptr, w.ffn,
-                        w.status, st);
+                        w.status, st, 3, nullptr, w.y_perm);
     if (rc)
         return rc;
     CUDA_TRY(launch_combine(w.y_perm, w.dest_pos, tw, c.has_shared ? w.shared_out : nullptr,
@@ -785,7 +802,6 @@ int moe_layer_decode(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *y
     a.topk_ids = w.ids;
     a.topk_w = w.w;
     a.h = w.h;
-    a.o = w.o;
     a.y = y;
     a.status = w.status;
     a.bar = w.bar;

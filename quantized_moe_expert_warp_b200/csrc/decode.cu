@@ -4,18 +4,20 @@
 // With T <= 8 tokens the layer reads a few experts (k per token plus the
 // shared one) and does little arithmetic, so a chain of separate kernels
 // spends most of its time in launch gaps and pipeline fill.  Here one CTA
-// per SM runs five phases separated by grid barriers (bounded waits):
+// per SM runs four phases separated by two grid barriers (bounded waits):
 //
-//   A  router: logits[t, e] = x[t] . Wr[e] (+ bias), gate[t] = x[t] . g
-//      (fp32 FMAs on CUDA cores; rows of Wr spread over the CTAs)
-//   B  every CTA routes all T tokens itself (top-k as in route.cu), groups
-//      the (token, expert) pairs by expert and starts L2 prefetches of the
-//      chosen experts' weights
-//   C  gate/up + SwiGLU: one warp per (expert, 4 rows of I), full K = H:
-//      h[p, i] = silu(x[t] . Wg_e[i]) * (x[t] . Wu_e[i])   (fp32)
-//   D  down: one warp per (expert, 4 rows of H), full K = I:
-//      o[p, j] = h[p] . Wd_e[j]                              (fp32)
-//   E  combine: y[t] = bf16( sum_j w[t,j] o[p(t,j)] + sigmoid(gate[t]) o[shared t] )
+//   A  router: logits[t, e] = x[t] . Wr[e] (+ bias), gate[t] = x[t] . g;
+//      one warp per router row, rows spread over the CTAs
+//   B  every CTA routes all T tokens itself (top-k as in route.cu) and
+//      groups the (token, expert) pairs by expert
+//   C  gate/up + SwiGLU: a unit is (expert, 16 features), i.e. 16 rows of
+//      Wg and the 16 matching rows of Wu, one row per lane; the 16 warps
+//      split K = H, and the next unit's codes are loaded while the current
+//      one is computed:  h[p, i] = silu(x[t] . Wg_e[i]) * (x[t] . Wu_e[i])
+//   D  down and combine: a unit is 16 output columns of every chosen
+//      expert; lanes split K = I, and the combine of those columns happens
+//      in the same CTA:  y[t, c] = bf16( sum_j w[t,j] (h[p(t,j)] . Wd_e[c])
+//                                         + sigmoid(gate[t]) (h[shared t] . Wd_s[c]) )
 //
 // The expert weights stay in the packed 4-bit layout of dequant.cuh.  Each
 // 32-weight chunk is decoded to its integer codes (exact small integers in
@@ -25,8 +27,13 @@
 // dequantised values of the format (the GEMM path rounds them to bf16 for
 // the tensor cores), and no intermediate is rounded to bf16 before y.
 //
-// Work is split by output rows, never by K, and every sum runs in a fixed
-// order, so the result does not depend on the number of CTAs.
+// Each phase runs its code a few times per launch at most, so instruction
+// fetch is a large share of its time: loops over tokens, chunks and units
+// stay rolled, and the kernel is instantiated per weight format.
+//
+// Work is split by output rows and columns with fixed K slices, and every
+// sum runs in a fixed order, so the result does not depend on the number of
+// CTAs.
 #include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -39,7 +46,7 @@
 
 #ifdef MOEQ4_TRACE
 // phase timestamps (%globaltimer) of the first four CTAs, thread 0
-__device__ unsigned long long g_dec_trace[4][10];
+__device__ unsigned long long g_dec_trace[4][16];
 #define DEC_MARK(i)                                                   \
     do {                                                              \
         if (blockIdx.x < 4 && threadIdx.x == 0)                       \
@@ -57,8 +64,11 @@ namespace {
 
 constexpr int kThreads = kDecodeThreads;
 constexpr int kWarps = kThreads / 32;
-constexpr int kPad = 36;           // floats per 32-element chunk row in shared memory (bank spread)
-constexpr int kPrefetchBytes = 32768;
+constexpr int kN = kDecodeMaxT;
+constexpr int kPad = 36;    // floats per 32-element chunk row in shared memory (bank spread)
+constexpr int kFeat = 16;   // features per gate/up unit: 16 gate rows + 16 up rows, one per lane
+constexpr int kCols = 16;   // output columns per down unit
+constexpr int kDnBatch = 8; // down: slot passes whose codes are in flight at once
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned *p)
 {
@@ -79,11 +89,6 @@ __device__ __forceinline__ void st_release(unsigned *p, unsigned v)
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 // Grid barrier over all CTAs of a cooperative launch.  bar[0] counts
 // arrivals (back to 0 after every barrier), bar[1] is the generation,
 // bar[2] the abort flag.  Waits are bounded by the workspace's wait budget
@@ -91,12 +96,10 @@ __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes)
 // MOE_ERR_TIMEOUT, raises the abort flag (so the others stop waiting) and
 // the caller returns.  Returns false when the kernel must stop.
 //
-// Test knob, status word 21: when it holds c > 0, CTA c - 1 waits at the
+// Test knob (status word 21): when it holds c > 0, CTA c - 1 waits at the
 // first barrier without arriving, so that every CTA's wait runs out of its
 // budget (the way a lost arrival would); the kernel then returns with
 // MOE_ERR_TIMEOUT and a usable context.
-constexpr int kStatusSkipArrivalWord = 21;
-
 __device__ bool grid_sync(unsigned *bar, int *status, int where, int *s_flag)
 {
     __syncthreads();
@@ -104,8 +107,7 @@ __device__ bool grid_sync(unsigned *bar, int *status, int where, int *s_flag)
         int ok = 1;
         __threadfence();
         const unsigned gen = ld_acquire(bar + 1);   // read before arriving: it cannot move until we do
-        const bool skip = where == 91 && status &&
-                          *(const volatile int *)(status + kStatusSkipArrivalWord) == (int)blockIdx.x + 1;
+        const bool skip = where == 91 && test_knob_hits_this_cta(status);
         const unsigned prev = skip ? 0u : atomicAdd(bar, 1u);
         if (!skip && prev == gridDim.x - 1) {
             atomicExch(bar, 0u);
@@ -141,22 +143,26 @@ __device__ __forceinline__ bool better(float v, int id, float bv, int bid)
 
 // (a, b) of one 32-weight chunk so that weight_i = a * c_i + b, where c_i
 // is the decoded code: q = u - 8 for int4-sym (b = 0), u for the others.
-__device__ __forceinline__ void chunk_coeffs(const DecodeArgs &A, const uint8_t *mblock, int m, int ngroups, int r,
-                                             int kpos, float &a, float &b)
+// gshift: log2 of the int4 group size.
+template <int WFMT>
+__device__ __forceinline__ void chunk_coeffs(const uint8_t *mblock, int m, int ngroups, int r, int kpos, int gshift,
+                                             float &a, float &b)
 {
-    if (A.wfmt == MOE_WFMT_Q4K) {
-        const int sb = kpos / 256;
-        const uint4 hdr = *(const uint4 *)(mblock + ((size_t)(m * ngroups + sb) * kTileRows + r) * 16);
+    if (WFMT == MOE_WFMT_Q4K) {
+        const int sb = kpos >> 8;
+        const uint4 hdr = __ldg((const uint4 *)(mblock + ((size_t)(m * ngroups + sb) * kTileRows + r) * 16));
         float dsc, dm;
-        q4k_subblock_scale(hdr, (kpos % 256) / 32, dsc, dm);
+        q4k_subblock_scale(hdr, (kpos & 255) >> 5, dsc, dm);
         a = dsc;
         b = -dm;
-    } else if (A.wfmt == MOE_WFMT_INT4_ASYM) {
-        const uint32_t sm = *(const uint32_t *)(mblock + ((size_t)(m * ngroups + kpos / A.G) * kTileRows + r) * 4);
+    } else if (WFMT == MOE_WFMT_INT4_ASYM) {
+        const uint32_t sm =
+            __ldg((const uint32_t *)(mblock + ((size_t)(m * ngroups + (kpos >> gshift)) * kTileRows + r) * 4));
         a = __uint_as_float(sm << 16);
         b = __uint_as_float(sm & 0xFFFF0000u);
     } else {
-        const uint16_t s = *(const uint16_t *)(mblock + ((size_t)(m * ngroups + kpos / A.G) * kTileRows + r) * 2);
+        const uint16_t s =
+            __ldg((const uint16_t *)(mblock + ((size_t)(m * ngroups + (kpos >> gshift)) * kTileRows + r) * 2));
         a = __uint_as_float((uint32_t)s << 16);
         b = 0.f;
     }
@@ -166,10 +172,11 @@ __device__ __forceinline__ void chunk_coeffs(const DecodeArgs &A, const uint8_t 
 // Element 8w + 2i sits in nibble i of word w, element 8w + 2i + 1 in
 // nibble i + 4.  Two codes at a time become a bf16 pair 128 + u (exact),
 // minus 136 (int4-sym: q = u - 8) or 128 (the others), both exact.
-__device__ __forceinline__ void decode_codes(const uint4 codes, bool sym, float (&c)[32])
+template <bool SYM>
+__device__ __forceinline__ void decode_codes(const uint4 codes, float (&c)[32])
 {
     const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
-    const uint32_t off = sym ? 0x43084308u : 0x43004300u;
+    const uint32_t off = SYM ? 0x43084308u : 0x43004300u;
 #pragma unroll
     for (int wi = 0; wi < 4; ++wi) {
 #pragma unroll
@@ -181,56 +188,126 @@ __device__ __forceinline__ void decode_codes(const uint4 codes, bool sym, float 
     }
 }
 
-// sum_i c_i v_i over one padded 32-float row in shared memory
+// sum_i c_i v_i over one padded 32-float row in shared memory, four
+// independent partial sums added in a fixed order
 __device__ __forceinline__ float dot32(const float (&c)[32], const float *v)
 {
-    float acc = 0.f;
+    float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
         const float4 x4 = *(const float4 *)(v + 4 * q);
-        acc = fmaf(c[4 * q], x4.x, acc);
-        acc = fmaf(c[4 * q + 1], x4.y, acc);
-        acc = fmaf(c[4 * q + 2], x4.z, acc);
-        acc = fmaf(c[4 * q + 3], x4.w, acc);
+        p0 = fmaf(c[4 * q], x4.x, p0);
+        p1 = fmaf(c[4 * q + 1], x4.y, p1);
+        p2 = fmaf(c[4 * q + 2], x4.z, p2);
+        p3 = fmaf(c[4 * q + 3], x4.w, p3);
     }
-    return acc;
+    return (p0 + p1) + (p2 + p3);
 }
 
-// L2 prefetch of the weights of `nslots` experts, piece q of all pieces
-// handled by thread (q mod grid threads); slot_e(d) gives the expert.
-template <typename SlotE>
-__device__ void prefetch_experts(const DecodeArgs &A, int nslots, SlotE slot_e)
+// sum of the 32 floats of a padded chunk row, in order
+__device__ __forceinline__ float chunk_sum(const float *p)
 {
-    const size_t gu_codes = (size_t)(A.I / kTileRows) * (A.H / kKStep) * code_block_bytes(2);
-    const size_t gu_meta = (size_t)(A.I / kTileRows) * A.gu_meta_bytes;
-    const size_t dn_codes = (size_t)(A.H / kTileRows) * (A.I / kKStep) * code_block_bytes(1);
-    const size_t dn_meta = (size_t)(A.H / kTileRows) * A.dn_meta_bytes;
-    auto pieces = [](size_t b) { return (int)((b + kPrefetchBytes - 1) / kPrefetchBytes); };
-    const int n0 = pieces(gu_codes), n1 = pieces(gu_meta), n2 = pieces(dn_codes), n3 = pieces(dn_meta);
-    const int pps = n0 + n1 + n2 + n3;
-    const int total = nslots * pps;
-    for (int q = blockIdx.x + gridDim.x * threadIdx.x; q < total; q += gridDim.x * blockDim.x) {
-        const size_t e = (size_t)slot_e(q / pps);
-        int w = q % pps;
-        const uint8_t *base;
-        size_t size;
-        if (w < n0) {
-            base = A.gu_q + e * gu_codes;
-            size = gu_codes;
-        } else if ((w -= n0) < n1) {
-            base = A.gu_meta + e * gu_meta;
-            size = gu_meta;
-        } else if ((w -= n1) < n2) {
-            base = A.dn_q + e * dn_codes;
-            size = dn_codes;
-        } else {
-            w -= n2;
-            base = A.dn_meta + e * dn_meta;
-            size = dn_meta;
+    float s = 0.f;
+    for (int q = 0; q < 32; ++q)
+        s += p[q];
+    return s;
+}
+
+// Top-k of one token by one warp (lane l holds logits l, l + 32, ...):
+// ties to the lower id, weights softmax over the kept k (renorm) or over
+// all E.  Lane j < k returns the j-th id and weight; a position left
+// unfilled (NaN logits) returns id -1.
+template <int NPL>
+__device__ __forceinline__ void topk_warp(const float *Lrow, int E, int k, int renorm, int lane, int &my_id,
+                                          float &my_w)
+{
+    float v[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const int e = i * 32 + lane;
+        v[i] = e < E ? __ldcg(Lrow + e) : -CUDART_INF_F;
+    }
+    uint32_t taken = 0;
+    float top = 0.f, my_val = 0.f;
+    my_id = -1;
+    for (int j = 0; j < k; ++j) {
+        float bv = -CUDART_INF_F;
+        int bid = 0x7FFFFFFF;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = i * 32 + lane;
+            if (e < E && !((taken >> i) & 1u) && better(v[i], e, bv, bid)) {
+                bv = v[i];
+                bid = e;
+            }
         }
-        const size_t off = (size_t)w * kPrefetchBytes;
-        const size_t left = size - off;
-        prefetch_l2(base + off, (uint32_t)(left < (size_t)kPrefetchBytes ? left : (size_t)kPrefetchBytes));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
+            const int oid = __shfl_xor_sync(0xFFFFFFFFu, bid, off);
+            if (better(ov, oid, bv, bid)) {
+                bv = ov;
+                bid = oid;
+            }
+        }
+        if (bid != 0x7FFFFFFF && (bid & 31) == lane)
+            taken |= 1u << (bid >> 5);
+        if (j == 0)
+            top = bv;
+        if (lane == j) {
+            my_val = bv;
+            my_id = bid == 0x7FFFFFFF ? -1 : bid;
+        }
+    }
+    const float ex = lane < k ? expf(my_val - top) : 0.f;
+    float z;
+    if (renorm) {
+        z = 0.f;
+        for (int j = 0; j < k; ++j)
+            z += __shfl_sync(0xFFFFFFFFu, ex, j);
+    } else {
+        float part = 0.f;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i)
+            if (i * 32 + lane < E)
+                part += expf(v[i] - top);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            part += __shfl_xor_sync(0xFFFFFFFFu, part, off);
+        z = part;
+    }
+    my_w = ex / z;
+}
+
+// Codes and chunk coefficients of one gate/up unit, this thread's share:
+// lane = row (gate rows 0-15, up rows 16-31 of the unit's 16 features),
+// chunks j = warp + 16 n of K = H (n < 4; H <= 2048 per pass of j0).
+struct GuLoad {
+    uint4 cd[4];
+    float ca[4], cb[4];
+};
+
+template <int WFMT>
+__device__ __forceinline__ void gu_load(const DecodeArgs &A, int e, int f0, int j0, int nchH, int ngroups, int gshift,
+                                        int warp, int lane, GuLoad &g)
+{
+    const int F = A.I / kTileRows, KS = A.H / kKStep;
+    const int m = lane >> 4, R = f0 + (lane & 15);
+    const size_t tile = (size_t)e * F + R / kTileRows;
+    const int r = R % kTileRows;
+    const uint8_t *qb = A.gu_q + tile * KS * code_block_bytes(2) + ((size_t)m * 2 * kTileRows + r) * kChunkBytes;
+    const uint8_t *mb = A.gu_meta + tile * A.gu_meta_bytes;
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+        const int j = j0 + warp + n * kWarps;
+        if (j < nchH) {
+            g.cd[n] = __ldg((const uint4 *)(qb + (size_t)(j >> 1) * code_block_bytes(2) +
+                                            (size_t)(j & 1) * kTileRows * kChunkBytes));
+            chunk_coeffs<WFMT>(mb, m, ngroups, r, j * 32, gshift, g.ca[n], g.cb[n]);
+        } else {
+            g.cd[n] = make_uint4(0, 0, 0, 0);
+            g.ca[n] = g.cb[n] = 0.f;
+        }
     }
 }
 
@@ -242,18 +319,19 @@ DecodeSmem decode_smem_layout(int T, int k, int H, int I, int has_shared)
     const int tk = T * k;
     const int np = tk + (has_shared ? T : 0);
     const int nd = tk + (has_shared ? 1 : 0);
-    const size_t big = (size_t)kPad * ((size_t)T * (H / 32) > (size_t)np * (I / 32) ? (size_t)T * (H / 32)
-                                                                                        : (size_t)np * (I / 32));
-    const size_t sums = (size_t)T * (H / 32) > (size_t)np * (I / 32) ? (size_t)T * (H / 32) : (size_t)np * (I / 32);
+    const size_t xrows = (size_t)T * (H / 32), hrows = (size_t)np * (I / 32);
+    const size_t rows = xrows > hrows ? xrows : hrows;
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t o = off;
         off += (bytes + 15) & ~(size_t)15;
         return (int)o;
     };
-    s.big = take(sizeof(float) * big);
-    s.sums = take(sizeof(float) * sums);
-    s.red = take(sizeof(float) * kWarps * kDecodeMaxT);
+    s.big = take(sizeof(float) * kPad * rows);
+    s.sums = take(sizeof(float) * rows);
+    // gate/up partials [warp][token][lane]; reused for the down outputs [pair][column]
+    const size_t red = (size_t)kWarps * kN * 32 > (size_t)np * kCols ? (size_t)kWarps * kN * 32 : (size_t)np * kCols;
+    s.red = take(sizeof(float) * red);
     s.ids = take(sizeof(int) * (tk > 0 ? tk : 1));
     s.w = take(sizeof(float) * np);
     s.pidx = take(sizeof(int) * (tk > 0 ? tk : 1));
@@ -269,6 +347,9 @@ DecodeSmem decode_smem_layout(int T, int k, int H, int I, int has_shared)
     return s;
 }
 
+namespace {
+
+template <int WFMT>
 __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeArgs A, const DecodeSmem L)
 {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -287,11 +368,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     int *wprefix = (int *)(smem + L.wprefix);
     int *flag = (int *)(smem + L.flag);
 
+    constexpr bool kSym = WFMT == MOE_WFMT_INT4_SYM;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = A.T, H = A.H, I = A.I, E = A.E, k = A.k;
     const int tk = T * k;
     const int nchH = H / 32, nchI = I / 32;
-    const bool sym = A.wfmt == MOE_WFMT_INT4_SYM;
+    const int gshift = __ffs(A.G > 0 ? A.G : 1) - 1;
 
     // a previous launch on this workspace gave up in a barrier: stop before touching it
     if (ld_relaxed(A.bar + 2)) {
@@ -303,17 +385,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     if (tid < 32)
         bitmap[tid] = 0;
 
-    // the shared expert is known in advance: start its prefetch now
-    if (A.has_shared)
-        prefetch_experts(A, 1, [&](int) { return E; });
-
     // ------------------------------------------------ A: x -> smem, router
     {
-        float *xs = big;
-        for (int i = tid; i < T * H / 8; i += kThreads) {
+        for (int i = tid; i < T * (H / 8); i += kThreads) {
             const int t = i / (H / 8), kk = (i % (H / 8)) * 8;
             const uint4 v = *(const uint4 *)(A.x + (size_t)t * H + kk);
-            float *dst = xs + (size_t)t * nchH * kPad + (kk / 32) * kPad + kk % 32;
+            float *dst = big + ((size_t)t * nchH + kk / 32) * kPad + kk % 32;
             const uint32_t u[4] = {v.x, v.y, v.z, v.w};
             *(float4 *)dst = make_float4(__uint_as_float(u[0] << 16), __uint_as_float(u[0] & 0xFFFF0000u),
                                          __uint_as_float(u[1] << 16), __uint_as_float(u[1] & 0xFFFF0000u));
@@ -321,58 +398,52 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
                                                __uint_as_float(u[3] << 16), __uint_as_float(u[3] & 0xFFFF0000u));
         }
         __syncthreads();
-        // chunk sums of x (the offset term of asymmetric formats)
-        for (int i = tid; i < T * nchH; i += kThreads) {
-            const float *src = xs + (size_t)i * kPad;
-            float s = 0.f;
-            for (int q = 0; q < 32; ++q)
-                s += src[q];
-            sums[i] = s;
-        }
+        for (int i = tid; i < T * nchH; i += kThreads)
+            sums[i] = chunk_sum(big + (size_t)i * kPad);
+        // one warp per router row (and the shared gate vector); a lane holds
+        // 16 float4 of a 2048-wide slice of the row, loaded before any use
+        float *racc = red + warp * kN;
         const int rows = E + (A.has_shared ? 1 : 0);
-        for (int e = blockIdx.x; e < rows; e += gridDim.x) {
+        for (int e = blockIdx.x + gridDim.x * warp; e < rows; e += gridDim.x * kWarps) {
             const float *wrow = e < E ? A.router_w + (size_t)e * H : A.shared_gate;
-            float part[kDecodeMaxT];
+            for (int seg = 0; seg < H; seg += 2048) {
+                float4 wv[16];
 #pragma unroll
-            for (int t = 0; t < kDecodeMaxT; ++t)
-                part[t] = 0.f;
-            for (int q = tid; q < H / 4; q += kThreads) {
-                const float4 wv = __ldg((const float4 *)wrow + q);
-                const int kk = 4 * q;
-                const float *xp = xs + (kk / 32) * kPad + kk % 32;
+                for (int q = 0; q < 16; ++q) {
+                    const int kk = seg + (q * 32 + lane) * 4;
+                    wv[q] = kk < H ? __ldg((const float4 *)(wrow + kk)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                for (int t = 0; t < T; ++t) {
+                    const float *xt = big + (size_t)t * nchH * kPad;
+                    float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-                for (int t = 0; t < kDecodeMaxT; ++t) {
-                    if (t < T) {
-                        const float4 xv = *(const float4 *)(xp + (size_t)t * nchH * kPad);
-                        float a = part[t];
-                        a = fmaf(wv.x, xv.x, a);
-                        a = fmaf(wv.y, xv.y, a);
-                        a = fmaf(wv.z, xv.z, a);
-                        a = fmaf(wv.w, xv.w, a);
-                        part[t] = a;
+                    for (int q = 0; q < 16; ++q) {
+                        const int kk = seg + (q * 32 + lane) * 4;
+                        if (kk < H) {
+                            const float4 xv = *(const float4 *)(xt + (kk / 32) * kPad + kk % 32);
+                            a0 = fmaf(wv[q].x, xv.x, a0);
+                            a1 = fmaf(wv[q].y, xv.y, a1);
+                            a0 = fmaf(wv[q].z, xv.z, a0);
+                            a1 = fmaf(wv[q].w, xv.w, a1);
+                        }
                     }
+                    float v = a0 + a1;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1)
+                        v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+                    if (lane == 0)
+                        racc[t] = seg == 0 ? v : racc[t] + v;
                 }
             }
-#pragma unroll
-            for (int t = 0; t < kDecodeMaxT; ++t) {
-                float v = part[t];
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
-                    v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-                if (lane == 0 && t < T)
-                    red[warp * kDecodeMaxT + t] = v;
-            }
-            __syncthreads();
-            if (tid < T) {
-                float s = 0.f;
-                for (int w = 0; w < kWarps; ++w)
-                    s += red[w * kDecodeMaxT + tid];
+            __syncwarp();
+            if (lane < T) {
+                const float s = racc[lane];
                 if (e < E)
-                    A.logits[(size_t)tid * E + e] = A.router_bias ? s + A.router_bias[e] : s;
+                    A.logits[(size_t)lane * E + e] = A.router_bias ? s + A.router_bias[e] : s;
                 else
-                    A.gate_logit[tid] = s;
+                    A.gate_logit[lane] = s;
             }
-            __syncthreads();
+            __syncwarp();
         }
     }
     DEC_MARK(1);
@@ -390,65 +461,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
                 my_id = A.override_ids[(size_t)t * k + lane];
                 my_w = A.override_w[(size_t)t * k + lane];
             }
+        } else if (E <= 256) {
+            topk_warp<8>(A.logits + (size_t)t * E, E, k, A.renorm, lane, my_id, my_w);
         } else {
-            constexpr int NPL = 32;   // E <= 1024
-            const int npl = (E + 31) / 32;
-            float v[NPL];
-            const float *Lrow = A.logits + (size_t)t * E;
-#pragma unroll
-            for (int i = 0; i < NPL; ++i) {
-                const int e = i * 32 + lane;
-                v[i] = (i < npl && e < E) ? __ldcg(Lrow + e) : -CUDART_INF_F;
-            }
-            uint32_t taken = 0;
-            float top = 0.f, my_val = 0.f;
-            for (int j = 0; j < k; ++j) {
-                float bv = -CUDART_INF_F;
-                int bid = 0x7FFFFFFF;
-#pragma unroll
-                for (int i = 0; i < NPL; ++i) {
-                    const int e = i * 32 + lane;
-                    if (i < npl && e < E && !((taken >> i) & 1u) && better(v[i], e, bv, bid)) {
-                        bv = v[i];
-                        bid = e;
-                    }
-                }
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
-                    const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-                    const int oid = __shfl_xor_sync(0xFFFFFFFFu, bid, off);
-                    if (better(ov, oid, bv, bid)) {
-                        bv = ov;
-                        bid = oid;
-                    }
-                }
-                if (bid < E && (bid & 31) == lane)
-                    taken |= 1u << (bid >> 5);
-                if (j == 0)
-                    top = bv;
-                if (lane == j) {
-                    my_val = bv;
-                    my_id = bid;
-                }
-            }
-            const float ex = lane < k ? expf(my_val - top) : 0.f;
-            float z;
-            if (A.renorm) {
-                z = 0.f;
-                for (int j = 0; j < k; ++j)
-                    z += __shfl_sync(0xFFFFFFFFu, ex, j);
-            } else {
-                float part = 0.f;
-#pragma unroll
-                for (int i = 0; i < NPL; ++i)
-                    if (i < npl && i * 32 + lane < E)
-                        part += expf(v[i] - top);
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1)
-                    part += __shfl_xor_sync(0xFFFFFFFFu, part, off);
-                z = part;
-            }
-            my_w = ex / z;
+            topk_warp<32>(A.logits + (size_t)t * E, E, k, A.renorm, lane, my_id, my_w);
         }
         if (lane < k) {
             // an id outside [0, E) (given, or none found among NaN logits) is
@@ -526,84 +542,60 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     const int Nd = nd_routed + (A.has_shared ? 1 : 0);
     const int NP = tk + (A.has_shared ? T : 0);
     DEC_MARK(3);
-    prefetch_experts(A, nd_routed, [&](int d) { return slot_e[d]; });
 
     // ------------------------------------------------ C: gate/up + SwiGLU
     {
-        const float *xs = big;
-        const int F = I / kTileRows, KS = H / kKStep, ngroups = A.wfmt == MOE_WFMT_Q4K ? H / 256 : H / A.G;
-        const int r4 = lane & 3, jp = lane >> 2;
-        const int units = Nd * (I / 4);
-        for (int u = blockIdx.x + gridDim.x * warp; u < units; u += gridDim.x * kWarps) {
-            const int d = u / (I / 4), row0 = (u % (I / 4)) * 4;
-            const int e = slot_e[d], base = slot_base[d], cnt = slot_cnt[d];
-            const size_t tile = (size_t)e * F + row0 / kTileRows;
-            const int r = row0 % kTileRows + r4;
-            const uint8_t *qb = A.gu_q + tile * KS * code_block_bytes(2) + (size_t)r * kChunkBytes;
-            const uint8_t *mb = A.gu_meta + tile * A.gu_meta_bytes;
-            for (int i0 = 0; i0 < cnt; i0 += kDecodeMaxT) {
-                float acc[2][kDecodeMaxT];
-#pragma unroll
-                for (int m = 0; m < 2; ++m)
-#pragma unroll
-                    for (int i = 0; i < kDecodeMaxT; ++i)
-                        acc[m][i] = 0.f;
-                for (int j0 = 0; j0 < nchH; j0 += 32) {
-                    // up to four chunks of this lane, both matrices: loads first
-                    uint4 cd[4][2];
-                    float ca[4][2], cb[4][2];
-#pragma unroll
-                    for (int n = 0; n < 4; ++n) {
-                        const int j = j0 + jp + 8 * n;
-#pragma unroll
-                        for (int m = 0; m < 2; ++m) {
-                            if (j < nchH) {
-                                cd[n][m] = __ldg((const uint4 *)(qb + ((size_t)((j >> 1) * 2 + m) * 2 + (j & 1)) *
-                                                                          kTileRows * kChunkBytes));
-                                chunk_coeffs(A, mb, m, ngroups, r, j * 32, ca[n][m], cb[n][m]);
-                            } else {
-                                cd[n][m] = make_uint4(0, 0, 0, 0);
-                                ca[n][m] = cb[n][m] = 0.f;
-                            }
-                        }
-                    }
+        const int ngroups = WFMT == MOE_WFMT_Q4K ? H / 256 : H >> gshift;
+        const int per_slot = I / kFeat;
+        const int U = Nd * per_slot;
+        float *part = red;   // [warp][token][lane]
+        GuLoad cur, nxt;
+        int u = blockIdx.x;
+        if (u < U)
+            gu_load<WFMT>(A, slot_e[u / per_slot], (u % per_slot) * kFeat, 0, nchH, ngroups, gshift, warp, lane, cur);
+        for (; u < U; u += gridDim.x) {
+            const int d = u / per_slot, f0 = (u % per_slot) * kFeat;
+            const int base = slot_base[d], cnt = slot_cnt[d];
+            for (int i = 0; i < cnt; ++i)
+                part[(warp * kN + i) * 32 + lane] = 0.f;
+            for (int j0 = 0; j0 < nchH; j0 += 4 * kWarps) {
+                // the next chunk group of this unit, or the first of the next unit
+                const int jn = j0 + 4 * kWarps;
+                const int un = u + gridDim.x;
+                if (jn < nchH)
+                    gu_load<WFMT>(A, slot_e[d], f0, jn, nchH, ngroups, gshift, warp, lane, nxt);
+                else if (un < U)
+                    gu_load<WFMT>(A, slot_e[un / per_slot], (un % per_slot) * kFeat, 0, nchH, ngroups, gshift, warp,
+                                  lane, nxt);
+                for (int i = 0; i < cnt; ++i) {
+                    const int t = pair_tok[base + i];
+                    float acc = 0.f;
 #pragma unroll
                     for (int n = 0; n < 4; ++n) {
-                        const int j = j0 + jp + 8 * n;
-                        if (j >= nchH)
-                            continue;
-#pragma unroll
-                        for (int m = 0; m < 2; ++m) {
+                        const int j = j0 + warp + n * kWarps;
+                        if (j < nchH) {
                             float c[32];
-                            decode_codes(cd[n][m], sym, c);
-#pragma unroll
-                            for (int i = 0; i < kDecodeMaxT; ++i) {
-                                if (i0 + i < cnt) {
-                                    const int t = pair_tok[base + i0 + i];
-                                    const float dot = dot32(c, xs + ((size_t)t * nchH + j) * kPad);
-                                    acc[m][i] = fmaf(ca[n][m], dot, fmaf(cb[n][m], sums[t * nchH + j], acc[m][i]));
-                                }
-                            }
+                            decode_codes<kSym>(cur.cd[n], c);
+                            const float dot = dot32(c, big + ((size_t)t * nchH + j) * kPad);
+                            acc = fmaf(cur.ca[n], dot, fmaf(cur.cb[n], sums[t * nchH + j], acc));
                         }
                     }
+                    part[(warp * kN + i) * 32 + lane] += acc;
                 }
-#pragma unroll
-                for (int m = 0; m < 2; ++m)
-#pragma unroll
-                    for (int i = 0; i < kDecodeMaxT; ++i)
-#pragma unroll
-                        for (int o = 4; o < 32; o <<= 1)
-                            acc[m][i] += __shfl_xor_sync(0xFFFFFFFFu, acc[m][i], o);
-                if (jp == 0) {
-#pragma unroll
-                    for (int i = 0; i < kDecodeMaxT; ++i) {
-                        if (i0 + i < cnt) {
-                            const float g = acc[0][i];
-                            A.h[(size_t)(base + i0 + i) * I + row0 + r4] = g / (1.0f + expf(-g)) * acc[1][i];
-                        }
-                    }
-                }
+                cur = nxt;
             }
+            __syncthreads();
+            // feature f of the unit for its token i: gate and up sums over the warps, in order
+            if (tid < kFeat * cnt) {
+                const int i = tid / kFeat, f = tid % kFeat;
+                float g = 0.f, v = 0.f;
+                for (int w = 0; w < kWarps; ++w) {
+                    g += part[(w * kN + i) * 32 + f];
+                    v += part[(w * kN + i) * 32 + kFeat + f];
+                }
+                A.h[(size_t)(base + i) * I + f0 + f] = g / (1.0f + expf(-g)) * v;
+            }
+            __syncthreads();
         }
     }
     DEC_MARK(4);
@@ -611,117 +603,107 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
         return;
     DEC_MARK(5);
 
-    // ------------------------------------------------ D: down
+    // ------------------------------------------------ D: down + combine
     {
         float *hs = big;
-        for (int i = tid; i < NP * I / 4; i += kThreads) {
+        for (int i = tid; i < NP * (I / 4); i += kThreads) {
             const int p = i / (I / 4), kk = (i % (I / 4)) * 4;
             const float4 v = __ldcg((const float4 *)(A.h + (size_t)p * I + kk));
             *(float4 *)(hs + ((size_t)p * nchI + kk / 32) * kPad + kk % 32) = v;
         }
         __syncthreads();
-        for (int i = tid; i < NP * nchI; i += kThreads) {
-            const float *src = hs + (size_t)i * kPad;
-            float s = 0.f;
-            for (int q = 0; q < 32; ++q)
-                s += src[q];
-            sums[i] = s;
-        }
+        for (int i = tid; i < NP * nchI; i += kThreads)
+            sums[i] = chunk_sum(hs + (size_t)i * kPad);
         __syncthreads();
-        const int F = H / kTileRows, KS = I / kKStep, ngroups = A.wfmt == MOE_WFMT_Q4K ? I / 256 : I / A.G;
-        const int r4 = lane & 3, jp = lane >> 2;
-        const int units = Nd * (H / 4);
-        for (int u = blockIdx.x + gridDim.x * warp; u < units; u += gridDim.x * kWarps) {
-            const int d = u / (H / 4), row0 = (u % (H / 4)) * 4;
-            const int e = slot_e[d], base = slot_base[d], cnt = slot_cnt[d];
-            const size_t tile = (size_t)e * F + row0 / kTileRows;
-            const int r = row0 % kTileRows + r4;
-            const uint8_t *qb = A.dn_q + tile * KS * code_block_bytes(1) + (size_t)r * kChunkBytes;
-            const uint8_t *mb = A.dn_meta + tile * A.dn_meta_bytes;
-            for (int i0 = 0; i0 < cnt; i0 += kDecodeMaxT) {
-                float acc[kDecodeMaxT];
+        const int F = H / kTileRows, KS = I / kKStep, ngroups = WFMT == MOE_WFMT_Q4K ? I / 256 : I >> gshift;
+        // lanes per row: the power of two >= I / 32 chunks (at most 32);
+        // a slot pass covers kCols rows of one expert, SP passes side by side
+        int LJ = 1;
+        while (LJ < nchI)
+            LJ <<= 1;
+        const int per_pass = kCols * LJ;                // threads of one slot pass (>= 32: warp-uniform)
+        const int SP = kThreads / per_pass;
+        const int sub = tid / per_pass, cc = (tid / LJ) % kCols, j = tid % LJ;
+        float *o_s = red;   // [pair][column]
+        for (int u = blockIdx.x; u < H / kCols; u += gridDim.x) {
+            const int C = u * kCols + cc;
+            const int r = C % kTileRows;
+            for (int d0 = 0; d0 < Nd; d0 += SP * kDnBatch) {
+                uint4 cd[kDnBatch];
+                float ca[kDnBatch], cb[kDnBatch];
 #pragma unroll
-                for (int i = 0; i < kDecodeMaxT; ++i)
-                    acc[i] = 0.f;
-                for (int j0 = 0; j0 < nchI; j0 += 32) {
-                    uint4 cd[4];
-                    float ca[4], cb[4];
-#pragma unroll
-                    for (int n = 0; n < 4; ++n) {
-                        const int j = j0 + jp + 8 * n;
-                        if (j < nchI) {
-                            cd[n] = __ldg((const uint4 *)(qb + ((size_t)(j >> 1) * 2 + (j & 1)) * kTileRows *
-                                                                   kChunkBytes));
-                            chunk_coeffs(A, mb, 0, ngroups, r, j * 32, ca[n], cb[n]);
-                        } else {
-                            cd[n] = make_uint4(0, 0, 0, 0);
-                            ca[n] = cb[n] = 0.f;
-                        }
-                    }
-#pragma unroll
-                    for (int n = 0; n < 4; ++n) {
-                        const int j = j0 + jp + 8 * n;
-                        if (j >= nchI)
-                            continue;
-                        float c[32];
-                        decode_codes(cd[n], sym, c);
-#pragma unroll
-                        for (int i = 0; i < kDecodeMaxT; ++i) {
-                            if (i0 + i < cnt) {
-                                const int p = base + i0 + i;
-                                const float dot = dot32(c, hs + ((size_t)p * nchI + j) * kPad);
-                                acc[i] = fmaf(ca[n], dot, fmaf(cb[n], sums[p * nchI + j], acc[i]));
-                            }
-                        }
+                for (int b = 0; b < kDnBatch; ++b) {
+                    const int d = d0 + b * SP + sub;
+                    cd[b] = make_uint4(0, 0, 0, 0);
+                    ca[b] = cb[b] = 0.f;
+                    if (d < Nd && j < nchI) {
+                        const size_t tile = (size_t)slot_e[d] * F + C / kTileRows;
+                        cd[b] = __ldg((const uint4 *)(A.dn_q + (tile * KS + (j >> 1)) * code_block_bytes(1) +
+                                                      ((size_t)(j & 1) * kTileRows + r) * kChunkBytes));
+                        chunk_coeffs<WFMT>(A.dn_meta + tile * A.dn_meta_bytes, 0, ngroups, r, j * 32, gshift, ca[b],
+                                           cb[b]);
                     }
                 }
 #pragma unroll
-                for (int i = 0; i < kDecodeMaxT; ++i)
-#pragma unroll
-                    for (int o = 4; o < 32; o <<= 1)
-                        acc[i] += __shfl_xor_sync(0xFFFFFFFFu, acc[i], o);
-                if (jp == 0) {
-#pragma unroll
-                    for (int i = 0; i < kDecodeMaxT; ++i)
-                        if (i0 + i < cnt)
-                            A.o[(size_t)(base + i0 + i) * H + row0 + r4] = acc[i];
+                for (int b = 0; b < kDnBatch; ++b) {
+                    const int d = d0 + b * SP + sub;
+                    if (d >= Nd)
+                        continue;   // uniform over the pass's threads, which span whole warps
+                    const int base = slot_base[d], cnt = slot_cnt[d];
+                    float c[32];
+                    decode_codes<kSym>(cd[b], c);
+                    for (int i = 0; i < cnt; ++i) {
+                        const int p = base + i;
+                        float v = 0.f;
+                        if (j < nchI)
+                            v = fmaf(ca[b], dot32(c, hs + ((size_t)p * nchI + j) * kPad), cb[b] * sums[p * nchI + j]);
+                        for (int o = LJ >> 1; o > 0; o >>= 1)
+                            v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+                        if (j == 0)
+                            o_s[p * kCols + cc] = v;
+                    }
                 }
             }
+            __syncthreads();
+            // the combine of these columns: routed experts in j order, then the shared expert
+            if (tid < T * kCols) {
+                const int t = tid / kCols, c2 = tid % kCols;
+                float acc = 0.f;
+                for (int jj = 0; jj < k; ++jj)
+                    acc = fmaf(w_s[t * k + jj], o_s[pidx[t * k + jj] * kCols + c2], acc);
+                if (A.has_shared)
+                    acc = fmaf(w_s[tk + t], o_s[(tk + t) * kCols + c2], acc);
+                A.y[(size_t)t * H + u * kCols + c2] = (uint16_t)(pack_bf16x2(acc, 0.f) & 0xFFFFu);
+            }
+            __syncthreads();
         }
     }
     DEC_MARK(6);
-    if (!grid_sync(A.bar, A.status, 93, flag))
-        return;
-    DEC_MARK(7);
-
-    // ------------------------------------------------ E: combine
-    for (int i = blockIdx.x * kThreads + tid; i < T * H; i += gridDim.x * kThreads) {
-        const int t = i / H, col = i % H;
-        float acc = 0.f;
-        for (int j = 0; j < k; ++j)
-            acc = fmaf(w_s[t * k + j], __ldcg(A.o + (size_t)pidx[t * k + j] * H + col), acc);
-        if (A.has_shared)
-            acc = fmaf(w_s[tk + t], __ldcg(A.o + (size_t)(tk + t) * H + col), acc);
-        A.y[i] = (uint16_t)(pack_bf16x2(acc, 0.f) & 0xFFFFu);
-    }
-    DEC_MARK(8);
 }
+
+}  // namespace
 
 cudaError_t launch_decode_layer(const DecodeArgs &a, int grid, cudaStream_t st)
 {
     const DecodeSmem L = decode_smem_layout(a.T, a.k, a.H, a.I, a.has_shared);
-    // the opt-in limit once per device (callers never ask for more: see the admission check)
-    static std::atomic<bool> configured[64];
+    void (*kern)(const DecodeArgs, const DecodeSmem) =
+        a.wfmt == MOE_WFMT_Q4K         ? decode_layer_kernel<MOE_WFMT_Q4K>
+        : a.wfmt == MOE_WFMT_INT4_ASYM ? decode_layer_kernel<MOE_WFMT_INT4_ASYM>
+                                       : decode_layer_kernel<MOE_WFMT_INT4_SYM>;
+    // the opt-in limit once per device and format (callers never ask for
+    // more: see the admission check)
+    static std::atomic<bool> configured[64][3];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
-    if (dev < 0 || dev >= 64 || !configured[dev].load(std::memory_order_acquire)) {
-        e = cudaFuncSetAttribute(decode_layer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    const int f = a.wfmt == MOE_WFMT_Q4K ? 1 : a.wfmt == MOE_WFMT_INT4_ASYM ? 2 : 0;
+    if (dev < 0 || dev >= 64 || !configured[dev][f].load(std::memory_order_acquire)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess)
             return e;
         if (dev >= 0 && dev < 64)
-            configured[dev].store(true, std::memory_order_release);
+            configured[dev][f].store(true, std::memory_order_release);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -733,7 +715,7 @@ cudaError_t launch_decode_layer(const DecodeArgs &a, int grid, cudaStream_t st)
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_layer_kernel, a, L);
+    return cudaLaunchKernelEx(&cfg, kern, a, L);
 }
 
 }  // namespace moeq4

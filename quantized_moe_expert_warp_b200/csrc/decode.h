@@ -1,5 +1,5 @@
 // Fused decode layer (decode.cu): the whole layer for T <= kDecodeMaxT tokens
-// in one cooperative launch.
+// (expert intermediate I <= 1024) in one cooperative launch.
 #pragma once
 
 #include <cstddef>
@@ -26,7 +26,6 @@ struct DecodeArgs {
     int32_t *topk_ids;          // [T, k]
     float *topk_w;              // [T, k]
     float *h;                   // [NP, I] gate/up outputs, NP = T k (+ T)
-    float *o;                   // [NP, H] expert outputs before the combine
     uint16_t *y;                // [T, H] bf16
     int *status;                // [code, detail]
     unsigned *bar;              // [count, generation, abort] of the grid barrier

@@ -20,9 +20,9 @@
 // exact in fp32 and accumulate into one fp32 accumulator.
 //
 // Warp roles of one persistent CTA (one per SM, 768 threads):
-//   warp 0      loads token rows of B: gate/up gathers them with cp.async
-//               (zero rows past the tail); down reads contiguous rows of h
-//               with one tiled TMA copy per k-step
+//   warp 0      loads the token rows of B with one tiled TMA copy per k-step:
+//               rows of x in permuted order (gate/up, routed experts), of x
+//               (shared expert, router) or of h (down)
 //   warp 1      issues tcgen05.mma (one thread) and commits stage releases
 //   warp 2      streams code blocks and per-tile scale blocks with bulk copies
 //   warp 3      owns the TMEM allocation; in the router pass it also forms
@@ -159,9 +159,6 @@ struct Geo {
     static constexpr int kAccCols = kAccBufs * kNAcc * BN;
     static constexpr int kTmemCols = 512;
     static_assert(kAccCols + kAStages * kNA * 32 <= kTmemCols, "TMEM budget");
-    static constexpr bool kGather = MODE == MODE_GATE_UP;
-    // the down pass's token rows are contiguous rows of h: one TMA tile per k-step
-    static constexpr bool kTmaB = MODE == MODE_DOWN;
 };
 
 struct Barriers {
@@ -309,7 +306,8 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, int n_issued, int dep
 
 template <int MODE, int WFMT, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ GemmArgs p, const __grid_constant__ CUtensorMap tmap_b)
+    grouped_gemm_kernel(const __grid_constant__ GemmArgs p, const __grid_constant__ CUtensorMap tmap_b,
+                        const __grid_constant__ CUtensorMap tmap_b2)
 {
     using L = Geo<MODE, BN>;
     constexpr int kBN = BN;
@@ -344,9 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->a_empty[s], 1);
         }
         for (int s = 0; s < L::kBStages; ++s) {
-            // gather: one cp.async completion arrival per lane of the B producer;
-            // TMA: one arrival with the stage's byte count
-            mbar_init(&bars->b_full[s], L::kTmaB ? 1 : 32);
+            mbar_init(&bars->b_full[s], 1);   // one arrival with the stage's byte count
             mbar_init(&bars->b_empty[s], 1);
         }
         for (int s = 0; s < NCS; ++s) {
@@ -384,79 +380,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     WaitCtx wc{&bars->abort_flag, p.status, globaltimer_ns(), wait_limit_ns(p.status)};
     CYC_DECL
 
-    if (warp == 0 && L::kTmaB) {
+    if (warp == 0) {
         // ------------------------------------------------ B producer (TMA tiles of contiguous rows)
         // A tile of BN rows from the unit's first row: rows of the next
         // expert only feed MMA columns the epilogue discards, rows past the
-        // end of h arrive as zeros.
-        if (elect_one())
+        // end of the source arrive as zeros.  With a second source (gate/up
+        // with a shared expert) the shared expert's units read x itself.
+        if (elect_one()) {
             tma_prefetch_desc(&tmap_b);
+            if (p.b_src2)
+                tma_prefetch_desc(&tmap_b2);
+        }
         __syncwarp();
         int step = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
             const Unit un = decode_unit<BN>(u, p, sched);
+            const bool second = p.b_src2 && un.e >= p.E;
+            const CUtensorMap *map = second ? &tmap_b2 : &tmap_b;
+            const int y = second ? un.row0 - p.Tk : un.row0;
+            CYC(2);
             for (int ks = un.ks0; ks < un.ks0 + un.nks; ++ks, ++step) {
                 const int s = step % L::kBStages;
                 if (step >= L::kBStages && !warp_wait(&bars->b_empty[s], ((step / L::kBStages) & 1) ^ 1, wc, 1)) {
                     ok = false;
                     break;
                 }
+                CYC(0);
                 if (elect_one()) {
                     mbar_arrive_expect_tx(&bars->b_full[s], (uint32_t)(kBN * 128));
-                    tma_load_2d(sB + s * kBN * 128, &tmap_b, ks * kKStep, un.row0, &bars->b_full[s]);
+                    tma_load_2d(sB + s * kBN * 128, map, ks * kKStep, y, &bars->b_full[s]);
                 }
                 __syncwarp();
-            }
-        }
-        drain_ring(bars->b_full, step, L::kBStages, p.status, 12, &bars->never_abort);
-    } else if (warp == 0) {
-        // ------------------------------------------------ B producer (cp.async row gather)
-        int step = 0;
-        bool ok = true;
-        for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
-            const Unit un = decode_unit<BN>(u, p, sched);
-            const uint16_t *src[kBN / 32];
-            uint32_t bytes[kBN / 32];
-#pragma unroll
-            for (int i = 0; i < kBN / 32; ++i) {
-                const int r = lane + 32 * i;
-                const int prow = un.row0 + r;
-                int srow = 0;
-                if (r < un.nvalid)
-                    srow = L::kGather ? (prow < p.Tk ? p.sorted_slot[prow] / p.topk : prow - p.Tk) : prow;
-                src[i] = p.b_src + (size_t)srow * p.ldb;
-                bytes[i] = r < un.nvalid ? 16u : 0u;
-            }
-            CYC(2);
-            for (int ks = un.ks0; ks < un.ks0 + un.nks; ++ks, ++step) {
-                const int s = step % L::kBStages;
-                if (step >= L::kBStages && !mbar_wait(&bars->b_empty[s], ((step / L::kBStages) & 1) ^ 1, wc, 1)) {
-                    ok = false;
-                    break;
-                }
-                CYC(0);
-                const uint32_t base = smem_u32(sB + s * kBN * 128);
-#pragma unroll
-                for (int i = 0; i < kBN / 32; ++i) {
-                    const int r = lane + 32 * i;
-                    if (r < un.nmma) {
-                        const uint32_t rbase = base + (r >> 3) * 1024 + (r & 7) * 128;
-                        const uint16_t *g = src[i] + ks * kKStep;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            cp_async_16(rbase + ((j ^ (r & 7)) << 4), g + j * 8, bytes[i]);
-                    }
-                }
-                // this lane's copies for the stage arrive on b_full[s] when they land
-                cp_async_arrive_noinc(&bars->b_full[s]);
                 CYC(1);
                 if (lane == 0)
                     TRACE_OTHER(0, step);
             }
         }
-        cp_async_wait_group<0>();
-        __syncwarp();
         drain_ring(bars->b_full, step, L::kBStages, p.status, 12, &bars->never_abort);
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (converged warp, one elected lane)
@@ -490,9 +450,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0)
                     TRACE_OTHER(9, step);
                 tc_fence_after();
-                // the B stage was written by cp.async (generic proxy); the MMA
-                // reads it through the async proxy
-                fence_proxy_async_smem();
                 const uint64_t bdesc0 = sdesc_kmajor_sw128(smem_u32(sB + sb * kBN * 128));
                 const uint32_t a_base = tmem + L::kAccCols + sa * L::kNA * 32;
                 if (elect_one()) {
@@ -532,8 +489,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ code / meta producer (converged warp)
         // A unit's code blocks are contiguous in the kernel layout, so one bulk
         // copy moves CK k-steps: the copy engine's throughput is set by the
-        // number of copies more than by their size.
-        if (MODE != MODE_ROUTER) {
+        // number of copies more than by their size.  (Under the status block's
+        // test knob this CTA issues none, and its dequant waits run out.)
+        if (MODE != MODE_ROUTER && !test_knob_hits_this_cta(p.status)) {
             int cidx = 0, munit = 0, nmeta = 0;   // cidx: code chunks issued; nmeta: meta blocks issued
             bool ok = true;
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++munit) {
@@ -992,18 +950,18 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 // Tensor map of the B rows (bf16 [b_rows, ldb], row-major) in tiles of
 // 64 elements (128 bytes, 128-byte swizzle: the MMA's K-major layout) by
 // BN rows.
-static cudaError_t encode_b_map(CUtensorMap *m, const GemmArgs &a, int bn)
+static cudaError_t encode_b_map(CUtensorMap *m, const uint16_t *src, int ld, int rows, int bn)
 {
     const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc)
         return cudaErrorNotSupported;
-    if ((reinterpret_cast<uintptr_t>(a.b_src) & 15) || a.b_rows < 1 || ((size_t)a.ldb * 2) % 16)
+    if ((reinterpret_cast<uintptr_t>(src) & 15) || rows < 1 || ((size_t)ld * 2) % 16)
         return cudaErrorInvalidValue;
-    const cuuint64_t dims[2] = {(cuuint64_t)a.ldb, (cuuint64_t)a.b_rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)a.ldb * 2};
+    const cuuint64_t dims[2] = {(cuuint64_t)ld, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
     const cuuint32_t box[2] = {(cuuint32_t)kKStep, (cuuint32_t)bn};
     const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(a.b_src), dims, strides,
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(src), dims, strides,
                            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
@@ -1013,12 +971,12 @@ template <int MODE, int WFMT, int BN>
 static cudaError_t launch_one(const GemmArgs &a_in, int num_sms, cudaStream_t st)
 {
     auto kern = grouped_gemm_kernel<MODE, WFMT, BN>;
-    CUtensorMap tmap{};
-    if (Geo<MODE, BN>::kTmaB) {
-        const cudaError_t e = encode_b_map(&tmap, a_in, BN);
-        if (e != cudaSuccess)
-            return e;
-    }
+    CUtensorMap tmap{}, tmap2{};
+    cudaError_t e = encode_b_map(&tmap, a_in.b_src, a_in.ldb, a_in.b_rows, BN);
+    if (e == cudaSuccess && a_in.b_src2)
+        e = encode_b_map(&tmap2, a_in.b_src2, a_in.ldb, a_in.b_rows2, BN);
+    if (e != cudaSuccess)
+        return e;
     GemmArgs a = a_in;
     if (a.ksplit < 1)
         a.ksplit = 1;
@@ -1029,10 +987,10 @@ static cudaError_t launch_one(const GemmArgs &a_in, int num_sms, cudaStream_t st
     const size_t smem = gemm_smem_bytes<MODE, BN>(a.meta_bytes, a.E_total, r);
     if (smem > kSmemLimit)
         return cudaErrorInvalidConfiguration;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
-    return launch_pdl(kern, num_sms, kThreads, smem, st, a, tmap);
+    return launch_pdl(kern, num_sms, kThreads, smem, st, a, tmap, tmap2);
 }
 
 size_t gemm_smem_required(int nmat, int meta_bytes, int E_total)

@@ -43,9 +43,11 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 struct GemmArgs {
     const uint8_t *wq;          // codes, kernel layout
     const uint8_t *wmeta;       // scales / super-block headers, kernel layout
-    const uint16_t *b_src;      // token rows: x [T, H] (gathered) or h [rows, I]
-    int ldb;                    // elements per row of b_src
+    const uint16_t *b_src;      // token rows of the routed experts: x in permuted order [T k, H], or h [rows, I]
+    int ldb;                    // elements per row of b_src (and b_src2)
     int b_rows;                 // rows of b_src
+    const uint16_t *b_src2;     // gate/up with a shared expert: its token rows x [T, H]; else null
+    int b_rows2;                // rows of b_src2
     const int32_t *sorted_slot; // permutation (gather pass)
     int topk;
     int Tk;                     // T * k: rows at or past Tk belong to the shared expert
@@ -102,6 +104,10 @@ cudaError_t launch_permute(const int32_t *ids, int T, int E, int k, int32_t *cou
 int noalloc_max_experts();
 cudaError_t launch_permute_noalloc(const int32_t *ids, int T, int E, int k, int32_t *counts, int32_t *offsets,
                                    int32_t *sorted_slot, int32_t *dest_pos, cudaStream_t st);
+
+// out[p] = x[sorted_slot[p] / k] for p < rows (x, out: bf16 rows of H elements)
+cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *sorted_slot, int rows, int k, int H, uint16_t *out,
+                               int num_sms, cudaStream_t st);
 
 cudaError_t launch_combine(const uint16_t *y_perm, const int32_t *dest_pos, const float *w, const uint16_t *shared_out,
                            const float *gate_logit, int T, int H, int k, uint16_t *y, cudaStream_t st);

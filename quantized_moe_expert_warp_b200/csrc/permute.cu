@@ -245,6 +245,41 @@ cudaError_t launch_permute(const int32_t *ids, int T, int E, int k, int32_t *cou
 
 
 // ------------------------------------------------------------------------
+// Token rows in permuted order: out[p] = x[sorted_slot[p] / k] for the
+// rows p < rows, so that the gate/up GEMM can read each expert's rows as one
+// contiguous block with TMA tiles.  One warp copies one row with 16-byte
+// vectors (H a multiple of 128).
+// ------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t *__restrict__ x,
+                                                          const int32_t *__restrict__ sorted_slot, int rows, int k,
+                                                          int H, uint16_t *__restrict__ out)
+{
+    pdl_wait();
+    pdl_allow_successor();
+    const int lane = threadIdx.x & 31;
+    const int n16 = H / 8;
+    const int warps = gridDim.x * (blockDim.x / 32);
+    for (int p = (blockIdx.x * blockDim.x + threadIdx.x) / 32; p < rows; p += warps) {
+        const int t = sorted_slot[p] / k;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
+        uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)p * H);
+        for (int i = lane; i < n16; i += 32)
+            dst[i] = src[i];
+    }
+}
+
+cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *sorted_slot, int rows, int k, int H, uint16_t *out,
+                               int num_sms, cudaStream_t st)
+{
+    if (rows <= 0)
+        return cudaSuccess;
+    const int need = (rows + 7) / 8;   // eight warps per block
+    const int blocks = need < 4 * num_sms ? need : 4 * num_sms;
+    return launch_pdl(gather_rows_kernel, blocks, 256, 0, st, x, sorted_slot, rows, k, H, out);
+}
+
+// ------------------------------------------------------------------------
 // Allocation-free variant of moe_permute.
 //
 // Some callers cannot allocate device memory at the point where they need a

@@ -162,6 +162,15 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: kernels here take wel
 // Word of a workspace's status block holding the caller's wait budget in
 // microseconds (0: the 2 s default).
 constexpr int kStatusWaitLimitWord = 20;
+// Test knob word: c > 0 makes CTA c - 1 of a launch lose one of its own
+// signals (a grid-barrier arrival in the decode kernel, the weight copies in
+// the grouped GEMMs), so that its waits run out of the budget.  Zero in use.
+constexpr int kStatusTestKnobWord = 21;
+
+__device__ __forceinline__ bool test_knob_hits_this_cta(const int *status)
+{
+    return status && *(const volatile int *)(status + kStatusTestKnobWord) == (int)blockIdx.x + 1;
+}
 
 // The wait budget of a launch: the status block's word, else 2 s.
 __device__ __forceinline__ uint64_t wait_limit_ns(const int *status)
@@ -249,21 +258,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, WaitCt
         return true;
     uint32_t spins = 0;
     while (true) {
-        if (mbar_try_wait(bar, parity, sleep, hint)) {
-            MOEQ4_WAIT_HOOK(where, spins);
-            return true;
-        }
+        // after every failed poll: has another role given up, has the budget run out
         if (lds_volatile_s32(smem_u32((const void *)w.abort_flag)))
             return false;
-        if ((MOEQ4_BACKOFF_SITES >> where) & 1u)
-            __nanosleep(MOEQ4_BACKOFF_NS);
-        if (++spins % kClockEvery == 0) {
+        if (spins++ % kClockEvery == 0) {
             if (globaltimer_ns() - w.t0 > w.limit) {
                 *w.abort_flag = 1;
                 if (w.status && atomicCAS(w.status, 0, MOE_ERR_TIMEOUT) == 0)
                     w.status[1] = where;
                 return false;
             }
+        }
+        if ((MOEQ4_BACKOFF_SITES >> where) & 1u)
+            __nanosleep(MOEQ4_BACKOFF_NS);
+        if (mbar_try_wait(bar, parity, sleep, hint)) {
+            MOEQ4_WAIT_HOOK(where, spins);
+            return true;
         }
     }
 #endif

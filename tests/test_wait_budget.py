@@ -4,10 +4,11 @@ Every wait in the kernels gives up after the workspace's wait budget (word
 20 of its 256-byte status block, in microseconds; 0 means 2 s), records
 MOE_ERR_TIMEOUT in the status word and lets the kernel return, with TMEM
 freed and its own copies landed.  These tests make waits run out on
-purpose without any fault: a fused decode launch in which one CTA (chosen
-through word 21) does not arrive at the first grid barrier, so that every
-CTA's wait on it runs out of a 1 ms budget; and expert GEMMs given a 1 us
-budget, far less than their waits need.  Each time the status must say
+purpose without any fault, through the status block's test knob (word
+21): a fused decode launch in which one CTA does not arrive at the first
+grid barrier, so that every CTA's wait on it runs out of a 1 ms budget; and
+expert GEMMs in which one CTA issues no weight copies, so that its dequant
+warps' waits run out of a 1 ms budget while its other roles wind down.  Each time the status must say
 MOE_ERR_TIMEOUT, the call must come back long before the 2 s default, and
 the next call on the same workspace (status block cleared) must be exact.
 """
@@ -23,7 +24,7 @@ pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 
 WAIT_LIMIT_WORD = 20
-SKIP_ARRIVAL_WORD = 21
+TEST_KNOB_WORD = 21
 
 
 @pytest.fixture(scope="module")
@@ -60,7 +61,7 @@ def test_decode_lost_barrier_arrival_times_out(dev):
 
     words = ws[:256].view(torch.int32)
     words[WAIT_LIMIT_WORD] = 1000     # 1 ms
-    words[SKIP_ARRIVAL_WORD] = 3      # CTA 2 never arrives at the first barrier
+    words[TEST_KNOB_WORD] = 3         # CTA 2 never arrives at the first barrier
     y = torch.empty_like(y_ref)
     torch.cuda.synchronize(dev)
     t0 = time.perf_counter()
@@ -81,8 +82,8 @@ def test_decode_lost_barrier_arrival_times_out(dev):
                                  small_cfg("ffn_budget_wide", T=1200, E=4, k=2)],
                          ids=lambda c: c.name)
 def test_expert_gemms_run_out_of_budget_cleanly(dev, cfg):
-    """Both grouped GEMMs (gathered and TMA-fed token rows) on a valid
-    permutation, first with the default budget, then with 1 us."""
+    """Both grouped GEMMs on a valid permutation, first as they are, then
+    with CTA 0's weight copies withheld under a 1 ms budget."""
     import quantized_moe_expert_warp_b200 as mq
     from quantized_moe_expert_warp_b200.host import upload_layer, x_to_device
     layer = synth.make_layer(cfg)
@@ -110,7 +111,9 @@ def test_expert_gemms_run_out_of_budget_cleanly(dev, cfg):
     mq.moe_expert_ffn_q4(packed, x, T, ss, offsets, yp_ref, sh_ref, ws, n)
     assert mq.moe_read_status(ws) == (0, 0)
 
-    ws[:256].view(torch.int32)[WAIT_LIMIT_WORD] = 1   # 1 us: the first waits already run out
+    words = ws[:256].view(torch.int32)
+    words[WAIT_LIMIT_WORD] = 1000     # 1 ms
+    words[TEST_KNOB_WORD] = 1         # CTA 0 issues no weight copies: its dequant waits run out
     yp, sh = out()
     torch.cuda.synchronize(dev)
     t0 = time.perf_counter()
