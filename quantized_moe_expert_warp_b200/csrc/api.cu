@@ -214,7 +214,8 @@ LayerWs layer_layout(const moe_config_t *c, int T, uint8_t *base)
 struct DecodeWs {
     int *status;
     unsigned *bar;
-    float *logits, *gate_logit, *w, *h;
+    float *logits, *gate_logit, *w;
+    uint16_t *h;
     int32_t *ids;
     size_t bytes;
 };
@@ -236,7 +237,7 @@ DecodeWs decode_layout(const moe_config_t *c, int T, uint8_t *base)
     w.gate_logit = (float *)take(sizeof(float) * (size_t)T);
     w.ids = (int32_t *)take(sizeof(int32_t) * Tk);
     w.w = (float *)take(sizeof(float) * Tk);
-    w.h = (float *)take(sizeof(float) * NP * c->I);
+    w.h = (uint16_t *)take(sizeof(uint16_t) * NP * c->I);
     w.bytes = off;
     return w;
 }
@@ -250,7 +251,7 @@ const char *decode_refusal(const moe_config_t *c, int T)
         return "the fused decode kernel takes at most 8 tokens";
     if (c->I > 1024)
         return "the fused decode kernel takes an expert intermediate of at most 1024";
-    if (decode_smem_layout(T, c->k, c->H, c->I, c->has_shared).bytes > kMaxDynamicSmem)
+    if (decode_smem_layout(T, c->k, c->H, c->I, c->has_shared, c->wfmt).bytes > kMaxDynamicSmem)
         return "x or the expert intermediates of this shape exceed shared memory";
     return nullptr;
 }

@@ -7,28 +7,33 @@
 // per SM runs four phases separated by two grid barriers (bounded waits):
 //
 //   A  router: logits[t, e] = x[t] . Wr[e] (+ bias), gate[t] = x[t] . g;
-//      one warp per router row, rows spread over the CTAs
+//      one warp per router row (fp32 FMAs), rows spread over the CTAs
 //   B  every CTA routes all T tokens itself (top-k as in route.cu) and
 //      groups the (token, expert) pairs by expert
-//   C  gate/up + SwiGLU: a unit is (expert, 16 features), i.e. 16 rows of
-//      Wg and the 16 matching rows of Wu, one row per lane; the 16 warps
-//      split K = H, and the next unit's codes are loaded while the current
-//      one is computed:  h[p, i] = silu(x[t] . Wg_e[i]) * (x[t] . Wu_e[i])
-//   D  down and combine: a unit is 16 output columns of every chosen
-//      expert; lanes split K = I, and the combine of those columns happens
-//      in the same CTA:  y[t, c] = bf16( sum_j w[t,j] (h[p(t,j)] . Wd_e[c])
-//                                         + sigmoid(gate[t]) (h[shared t] . Wd_s[c]) )
+//   C  gate/up + SwiGLU: a unit is (expert, 16 features), i.e. a 16-row tile
+//      of Wg and the matching tile of Wu; the 16 warps split K = H, each
+//      runs warp-level m16n8k16 tensor-core MMAs against the expert's tokens
+//      (up to 8 columns), and the warps' sums are added in a fixed order:
+//          h[p, i] = bf16( silu(x[t] . Wg_e[i]) * (x[t] . Wu_e[i]) )
+//   D  down and combine: a unit is 16 output columns (a 16-row tile of Wd)
+//      of every chosen expert, one warp per expert, MMAs against the
+//      expert's h rows; the combine of those columns happens in the CTA:
+//          y[t, c] = bf16( sum_j w[t,j] (h[p(t,j)] . Wd_e[c])
+//                          + sigmoid(gate[t]) (h[shared t] . Wd_s[c]) )
 //
-// The expert weights stay in the packed 4-bit layout of dequant.cuh.  Each
-// 32-weight chunk is decoded to its integer codes (exact small integers in
-// fp32) and the dot product is taken against the codes; the chunk's scale
-// and offset are applied once per chunk:  sum_i (a u_i + b) x_i =
-// a (sum_i u_i x_i) + b (sum_i x_i).  The weights so used are the exact
-// dequantised values of the format (the GEMM path rounds them to bf16 for
-// the tensor cores), and no intermediate is rounded to bf16 before y.
+// The expert weights stay in the packed 4-bit layout of dequant.cuh and are
+// staged per warp in shared memory with cp.async (a ring of 2 to 4 items,
+// so that later items' codes are in flight during the current one).  An MMA's A operand is
+// built straight from the codes: one shift and one logical op give the bf16
+// pair (128 + u, 128 + u') of two codes, exact.  Each 32-weight chunk's scale
+// and offset are applied to the fp32 MMA result once per chunk,
+//     sum_i (a c_i + b) v_i = a (sum_i (128 + u_i) v_i - o sum_i v_i) + b sum_i v_i,
+// with c_i = u_i - 8, o = 136 (int4-sym) or c_i = u_i, o = 128 (the others),
+// so the weights enter at their exact dequantised values; x is bf16 (exact)
+// and h is rounded to bf16 once, as on the prefill path.
 //
 // Each phase runs its code a few times per launch at most, so instruction
-// fetch is a large share of its time: loops over tokens, chunks and units
+// fetch is a large share of its time: loops over tokens, chunks and items
 // stay rolled, and the kernel is instantiated per weight format.
 //
 // Work is split by output rows and columns with fixed K slices, and every
@@ -65,10 +70,18 @@ namespace {
 constexpr int kThreads = kDecodeThreads;
 constexpr int kWarps = kThreads / 32;
 constexpr int kN = kDecodeMaxT;
-constexpr int kPad = 36;    // floats per 32-element chunk row in shared memory (bank spread)
 constexpr int kFeat = 16;   // features per gate/up unit: 16 gate rows + 16 up rows, one per lane
 constexpr int kCols = 16;   // output columns per down unit
-constexpr int kDnBatch = 8; // down: slot passes whose codes are in flight at once
+constexpr int kCodeBuf = 2048; // staged codes of one warp item
+// bytes of one row's scale entry: bf16 scale (int4-sym), bf16 scale and
+// minimum (int4-asym), 16-byte super-block header (Q4K)
+__host__ __device__ constexpr int meta_row_bytes(int wfmt)
+{
+    return wfmt == MOE_WFMT_Q4K ? 16 : wfmt == MOE_WFMT_INT4_ASYM ? 4 : 2;
+}
+// one warp item: its codes, then the scale entries of its 16 rows for each
+// of its 8 (chunk, matrix) pairs
+__host__ __device__ constexpr int item_buf_bytes(int wfmt) { return kCodeBuf + 8 * 16 * meta_row_bytes(wfmt); }
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned *p)
 {
@@ -142,75 +155,25 @@ __device__ __forceinline__ bool better(float v, int id, float bv, int bid)
 }
 
 // (a, b) of one 32-weight chunk so that weight_i = a * c_i + b, where c_i
-// is the decoded code: q = u - 8 for int4-sym (b = 0), u for the others.
-// gshift: log2 of the int4 group size.
+// is the decoded code (q = u - 8 for int4-sym with b = 0, u for the
+// others), from the row's staged scale entry; kpos is the chunk's first
+// position along K.
 template <int WFMT>
-__device__ __forceinline__ void chunk_coeffs(const uint8_t *mblock, int m, int ngroups, int r, int kpos, int gshift,
-                                             float &a, float &b)
+__device__ __forceinline__ void staged_coeffs(const uint8_t *mrow, int kpos, float &a, float &b)
 {
     if (WFMT == MOE_WFMT_Q4K) {
-        const int sb = kpos >> 8;
-        const uint4 hdr = __ldg((const uint4 *)(mblock + ((size_t)(m * ngroups + sb) * kTileRows + r) * 16));
         float dsc, dm;
-        q4k_subblock_scale(hdr, (kpos & 255) >> 5, dsc, dm);
+        q4k_subblock_scale(*(const uint4 *)mrow, (kpos & 255) >> 5, dsc, dm);
         a = dsc;
         b = -dm;
     } else if (WFMT == MOE_WFMT_INT4_ASYM) {
-        const uint32_t sm =
-            __ldg((const uint32_t *)(mblock + ((size_t)(m * ngroups + (kpos >> gshift)) * kTileRows + r) * 4));
+        const uint32_t sm = *(const uint32_t *)mrow;
         a = __uint_as_float(sm << 16);
         b = __uint_as_float(sm & 0xFFFF0000u);
     } else {
-        const uint16_t s =
-            __ldg((const uint16_t *)(mblock + ((size_t)(m * ngroups + (kpos >> gshift)) * kTileRows + r) * 2));
-        a = __uint_as_float((uint32_t)s << 16);
+        a = __uint_as_float((uint32_t) * (const uint16_t *)mrow << 16);
         b = 0.f;
     }
-}
-
-// 32 codes of a chunk -> their integer values in fp32, element order.
-// Element 8w + 2i sits in nibble i of word w, element 8w + 2i + 1 in
-// nibble i + 4.  Two codes at a time become a bf16 pair 128 + u (exact),
-// minus 136 (int4-sym: q = u - 8) or 128 (the others), both exact.
-template <bool SYM>
-__device__ __forceinline__ void decode_codes(const uint4 codes, float (&c)[32])
-{
-    const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
-    const uint32_t off = SYM ? 0x43084308u : 0x43004300u;
-#pragma unroll
-    for (int wi = 0; wi < 4; ++wi) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t t = bf16x2_sub(((w[wi] >> (4 * i)) & 0x000F000Fu) | 0x43004300u, off);
-            c[8 * wi + 2 * i] = __uint_as_float(t << 16);
-            c[8 * wi + 2 * i + 1] = __uint_as_float(t & 0xFFFF0000u);
-        }
-    }
-}
-
-// sum_i c_i v_i over one padded 32-float row in shared memory, four
-// independent partial sums added in a fixed order
-__device__ __forceinline__ float dot32(const float (&c)[32], const float *v)
-{
-    float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        const float4 x4 = *(const float4 *)(v + 4 * q);
-        p0 = fmaf(c[4 * q], x4.x, p0);
-        p1 = fmaf(c[4 * q + 1], x4.y, p1);
-        p2 = fmaf(c[4 * q + 2], x4.z, p2);
-        p3 = fmaf(c[4 * q + 3], x4.w, p3);
-    }
-    return (p0 + p1) + (p2 + p3);
-}
-
-// sum of the 32 floats of a padded chunk row, in order
-__device__ __forceinline__ float chunk_sum(const float *p)
-{
-    float s = 0.f;
-    for (int q = 0; q < 32; ++q)
-        s += p[q];
-    return s;
 }
 
 // Top-k of one token by one warp (lane l holds logits l, l + 32, ...):
@@ -279,58 +242,83 @@ __device__ __forceinline__ void topk_warp(const float *Lrow, int E, int k, int r
     my_w = ex / z;
 }
 
-// Codes and chunk coefficients of one gate/up unit, this thread's share:
-// lane = row (gate rows 0-15, up rows 16-31 of the unit's 16 features),
-// chunks j = warp + 16 n of K = H (n < 4; H <= 2048 per pass of j0).
-struct GuLoad {
-    uint4 cd[4];
-    float ca[4], cb[4];
-};
-
-template <int WFMT>
-__device__ __forceinline__ void gu_load(const DecodeArgs &A, int e, int f0, int j0, int nchH, int ngroups, int gshift,
-                                        int warp, int lane, GuLoad &g)
+// Warp-level bf16 MMA, m16n8k16, fp32 accumulate: d += A B.  A: 16 x 16
+// (row), B: 16 x 8 (col); lane = 4 gid + tid4 holds A rows gid and gid + 8,
+// B column gid, D rows gid, gid + 8 and columns 2 tid4, 2 tid4 + 1.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1)
 {
-    const int F = A.I / kTileRows, KS = A.H / kKStep;
-    const int m = lane >> 4, R = f0 + (lane & 15);
-    const size_t tile = (size_t)e * F + R / kTileRows;
-    const int r = R % kTileRows;
-    const uint8_t *qb = A.gu_q + tile * KS * code_block_bytes(2) + ((size_t)m * 2 * kTileRows + r) * kChunkBytes;
-    const uint8_t *mb = A.gu_meta + tile * A.gu_meta_bytes;
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The bf16 pair (128 + u_{2i}, 128 + u_{2i+1}) of nibbles i and i + 4 of a
+// code word (exact values): the A-fragment register for columns 2i, 2i + 1.
+__device__ __forceinline__ uint32_t code_pair(uint32_t w, int i)
+{
+    return ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
+{
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// cp.async.wait_group with a run-time count (0 .. 3)
+__device__ __forceinline__ void cp_async_wait_upto(int n)
+{
+    if (n >= 3)
+        cp_async_wait_group<3>();
+    else if (n == 2)
+        cp_async_wait_group<2>();
+    else if (n == 1)
+        cp_async_wait_group<1>();
+    else
+        cp_async_wait_group<0>();
+}
+
+// One 32-element chunk of a 16-row tile against an 8-column B operand: the
+// two k16 slices of the chunk.  lo / hi: this lane's codes of rows gid and
+// gid + 8; brow: this lane's B column (a row of 16-bit values in shared
+// memory) at the chunk's first element.
+__device__ __forceinline__ void chunk_mma(float (&d)[4], const uint4 &lo, const uint4 &hi, const uint16_t *brow,
+                                          int tid4)
+{
 #pragma unroll
-    for (int n = 0; n < 4; ++n) {
-        const int j = j0 + warp + n * kWarps;
-        if (j < nchH) {
-            g.cd[n] = __ldg((const uint4 *)(qb + (size_t)(j >> 1) * code_block_bytes(2) +
-                                            (size_t)(j & 1) * kTileRows * kChunkBytes));
-            chunk_coeffs<WFMT>(mb, m, ngroups, r, j * 32, gshift, g.ca[n], g.cb[n]);
-        } else {
-            g.cd[n] = make_uint4(0, 0, 0, 0);
-            g.ca[n] = g.cb[n] = 0.f;
-        }
+    for (int s = 0; s < 2; ++s) {
+        const uint32_t a0 = code_pair(word_of(lo, 2 * s), tid4), a1 = code_pair(word_of(hi, 2 * s), tid4);
+        const uint32_t a2 = code_pair(word_of(lo, 2 * s + 1), tid4), a3 = code_pair(word_of(hi, 2 * s + 1), tid4);
+        const uint32_t b0 = *(const uint32_t *)(brow + 16 * s + 2 * tid4);
+        const uint32_t b1 = *(const uint32_t *)(brow + 16 * s + 8 + 2 * tid4);
+        mma_16816(d, a0, a1, a2, a3, b0, b1);
     }
 }
 
 }  // namespace
 
-DecodeSmem decode_smem_layout(int T, int k, int H, int I, int has_shared)
+DecodeSmem decode_smem_layout(int T, int k, int H, int I, int has_shared, int wfmt)
 {
     DecodeSmem s{};
     const int tk = T * k;
     const int np = tk + (has_shared ? T : 0);
     const int nd = tk + (has_shared ? 1 : 0);
-    const size_t xrows = (size_t)T * (H / 32), hrows = (size_t)np * (I / 32);
-    const size_t rows = xrows > hrows ? xrows : hrows;
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t o = off;
         off += (bytes + 15) & ~(size_t)15;
         return (int)o;
     };
-    s.big = take(sizeof(float) * kPad * rows);
-    s.sums = take(sizeof(float) * rows);
-    // gate/up partials [warp][token][lane]; reused for the down outputs [pair][column]
-    const size_t red = (size_t)kWarps * kN * 32 > (size_t)np * kCols ? (size_t)kWarps * kN * 32 : (size_t)np * kCols;
+    // phases A-C: x as bf16 rows (kN + 1, the last one zero) and its chunk
+    // sums; phase D reuses the space for h (np + 1 rows) and its chunk sums
+    const size_t xbytes = sizeof(uint16_t) * (size_t)(kN + 1) * (H + 8) + sizeof(float) * (size_t)kN * (H / 32) + 16;
+    const size_t hbytes = sizeof(uint16_t) * (size_t)(np + 1) * (I + 8) + sizeof(float) * (size_t)np * (I / 32) + 16;
+    s.big = take(xbytes > hbytes ? xbytes : hbytes);
+    s.sums = 0;   // placed inside big by the kernel
+    // gate/up partials [warp][matrix][row][token]; reused for the down outputs [pair][column]
+    const size_t red = (size_t)kWarps * 2 * 16 * kN > (size_t)np * kCols ? (size_t)kWarps * 2 * 16 * kN
+                                                                         : (size_t)np * kCols;
     s.red = take(sizeof(float) * red);
     s.ids = take(sizeof(int) * (tk > 0 ? tk : 1));
     s.w = take(sizeof(float) * np);
@@ -343,19 +331,103 @@ DecodeSmem decode_smem_layout(int T, int k, int H, int I, int has_shared)
     s.bitmap = take(sizeof(uint32_t) * 32);
     s.wprefix = take(sizeof(int) * 33);
     s.flag = take(sizeof(int) * 4);
+    // the warps' staging rings take what is left, 2 to 4 items deep (a
+    // shape whose 2-deep rings do not fit is refused by the caller)
+    const size_t ring = (size_t)kWarps * item_buf_bytes(wfmt);
+    const size_t left = off < kDecodeSmemLimit ? kDecodeSmemLimit - off : 0;
+    s.nstage = left / ring >= 4 ? 4 : left / ring >= 3 ? 3 : 2;
+    s.cbuf = take(ring * s.nstage);
     s.bytes = off;
     return s;
 }
 
 namespace {
 
+// Gate/up staging of one unit pass for this warp, with 16-byte cp.async:
+// chunks j = j0 + warp + 16 n (n < 4) of the 16 gate and 16 up rows of the
+// unit, as codes [n][matrix][row][16 bytes] (2 KB), then the rows' scale
+// entries of each (n, matrix) [n][matrix][row][entry].  gsh: log2 of the
+// positions along K that share one entry.
+template <int WFMT>
+__device__ __forceinline__ void gu_stage(const DecodeArgs &A, int e, int f0, int j0, int nchH, int gsh, int warp,
+                                         int lane, uint32_t dst)
+{
+    constexpr int MB = meta_row_bytes(WFMT);
+    const int F = A.I / kTileRows, KS = A.H / kKStep;
+    const int ngroups = A.H >> gsh;
+    const size_t tile = (size_t)e * F + f0 / kTileRows;
+    const int r0 = f0 % kTileRows;
+    const uint8_t *mb = A.gu_meta + tile * A.gu_meta_bytes;
+#pragma unroll
+    for (int q = 0; q < (8 * MB + 31) / 32; ++q) {
+        const int idx = lane + 32 * q;   // 8 MB pieces of 16 bytes
+        if (idx < 8 * MB) {
+            const int nm = idx / MB, pi = idx % MB, n = nm >> 1, m = nm & 1;
+            const int j = j0 + warp + kWarps * n;
+            if (j < nchH) {
+                const uint8_t *src = mb + ((size_t)(m * ngroups + ((j * 32) >> gsh)) * kTileRows + r0) * MB + 16 * pi;
+                cp_async_16(dst + kCodeBuf + idx * 16, src, 16);
+            }
+        }
+    }
+    const uint8_t *base = A.gu_q + tile * KS * code_block_bytes(2);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int idx = lane + 32 * q;    // 128 pieces of 16 bytes
+        const int n = idx >> 5, m = (idx >> 4) & 1, row = idx & 15;
+        const int j = j0 + warp + kWarps * n;
+        if (j < nchH) {
+            const uint8_t *src = base + (size_t)(j >> 1) * code_block_bytes(2) +
+                                 ((size_t)(m * 2 + (j & 1)) * kTileRows + r0 + row) * kChunkBytes;
+            cp_async_16(dst + idx * 16, src, 16);
+        }
+    }
+}
+
+// Down staging of one item for this warp: chunks j = 8 q + n (n < 8) of
+// the 16 rows c0 .. c0 + 15 of expert e's down matrix, as codes
+// [n][row][16 bytes] (2 KB), then the rows' scale entries [n][row][entry].
+template <int WFMT>
+__device__ __forceinline__ void dn_stage(const DecodeArgs &A, int e, int c0, int q, int nchI, int gsh, int lane,
+                                         uint32_t dst)
+{
+    constexpr int MB = meta_row_bytes(WFMT);
+    const int F = A.H / kTileRows, KS = A.I / kKStep;
+    const size_t tile = (size_t)e * F + c0 / kTileRows;
+    const int r0 = c0 % kTileRows;
+    const uint8_t *mb = A.dn_meta + tile * A.dn_meta_bytes;
+#pragma unroll
+    for (int qq = 0; qq < (8 * MB + 31) / 32; ++qq) {
+        const int idx = lane + 32 * qq;
+        if (idx < 8 * MB) {
+            const int n = idx / MB, pi = idx % MB;
+            const int j = 8 * q + n;
+            if (j < nchI) {
+                const uint8_t *src = mb + ((size_t)((j * 32) >> gsh) * kTileRows + r0) * MB + 16 * pi;
+                cp_async_16(dst + kCodeBuf + idx * 16, src, 16);
+            }
+        }
+    }
+    const uint8_t *base = A.dn_q + tile * KS * code_block_bytes(1);
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) {
+        const int idx = lane + 32 * qq;
+        const int n = idx >> 4, row = idx & 15;
+        const int j = 8 * q + n;
+        if (j < nchI) {
+            const uint8_t *src = base + (size_t)(j >> 1) * code_block_bytes(1) +
+                                 ((size_t)(j & 1) * kTileRows + r0 + row) * kChunkBytes;
+            cp_async_16(dst + idx * 16, src, 16);
+        }
+    }
+}
+
 template <int WFMT>
 __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeArgs A, const DecodeSmem L)
 {
     extern __shared__ __align__(16) uint8_t smem[];
-    float *big = (float *)(smem + L.big);
-    float *sums = (float *)(smem + L.sums);
     float *red = (float *)(smem + L.red);
+    uint8_t *cbuf = smem + L.cbuf;
     int *ids_s = (int *)(smem + L.ids);
     float *w_s = (float *)(smem + L.w);
     int *pidx = (int *)(smem + L.pidx);
@@ -368,15 +440,38 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     int *wprefix = (int *)(smem + L.wprefix);
     int *flag = (int *)(smem + L.flag);
 
-    constexpr bool kSym = WFMT == MOE_WFMT_INT4_SYM;
+    constexpr float kOff = WFMT == MOE_WFMT_INT4_SYM ? 136.f : 128.f;   // code pair value minus the code
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tid4 = lane & 3;
     const int T = A.T, H = A.H, I = A.I, E = A.E, k = A.k;
     const int tk = T * k;
     const int nchH = H / 32, nchI = I / 32;
     const int gshift = __ffs(A.G > 0 ? A.G : 1) - 1;
+    // x as bf16 rows of H + 8 elements (row kN is zeros) and fp32 chunk sums
+    const int XS = H + 8;
+    uint16_t *xb = (uint16_t *)(smem + L.big);
+    float *xsum = (float *)(xb + (size_t)(kN + 1) * XS);
+    constexpr int kMB = meta_row_bytes(WFMT), kIB = item_buf_bytes(WFMT);
+    const int NS = L.nstage;   // staging ring depth (items in flight per warp)
+    uint8_t *mybuf = cbuf + (size_t)warp * NS * kIB;
+    const uint32_t mybuf_s = smem_u32(mybuf);
 
+    // the abort flag of a previous launch, and this warp's first router row,
+    // are requested before anything else so that their latencies overlap
+    const unsigned aborted = ld_relaxed(A.bar + 2);
+    const int rows = E + (A.has_shared ? 1 : 0);
+    const int e_first = blockIdx.x + gridDim.x * warp;
+    float4 wv[16];
+    if (e_first < rows) {
+        const float *wrow = e_first < E ? A.router_w + (size_t)e_first * H : A.shared_gate;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const int kk = (q * 32 + lane) * 4;
+            wv[q] = kk < H ? __ldg((const float4 *)(wrow + kk)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
     // a previous launch on this workspace gave up in a barrier: stop before touching it
-    if (ld_relaxed(A.bar + 2)) {
+    if (aborted) {
         if (blockIdx.x == 0 && tid == 0)
             record_error(A.status, MOE_ERR_TIMEOUT, 90);
         return;
@@ -387,44 +482,44 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
 
     // ------------------------------------------------ A: x -> smem, router
     {
-        for (int i = tid; i < T * (H / 8); i += kThreads) {
+        for (int i = tid; i < (kN + 1) * (H / 8); i += kThreads) {
             const int t = i / (H / 8), kk = (i % (H / 8)) * 8;
-            const uint4 v = *(const uint4 *)(A.x + (size_t)t * H + kk);
-            float *dst = big + ((size_t)t * nchH + kk / 32) * kPad + kk % 32;
-            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-            *(float4 *)dst = make_float4(__uint_as_float(u[0] << 16), __uint_as_float(u[0] & 0xFFFF0000u),
-                                         __uint_as_float(u[1] << 16), __uint_as_float(u[1] & 0xFFFF0000u));
-            *(float4 *)(dst + 4) = make_float4(__uint_as_float(u[2] << 16), __uint_as_float(u[2] & 0xFFFF0000u),
-                                               __uint_as_float(u[3] << 16), __uint_as_float(u[3] & 0xFFFF0000u));
+            const uint4 v = t < T ? *(const uint4 *)(A.x + (size_t)t * H + kk) : make_uint4(0, 0, 0, 0);
+            *(uint4 *)(xb + (size_t)t * XS + kk) = v;
         }
         __syncthreads();
-        for (int i = tid; i < T * nchH; i += kThreads)
-            sums[i] = chunk_sum(big + (size_t)i * kPad);
+        for (int i = tid; i < kN * nchH; i += kThreads) {
+            const uint16_t *c = xb + (size_t)(i / nchH) * XS + (i % nchH) * 32;
+            float s = 0.f;
+            for (int q = 0; q < 32; ++q)
+                s += __uint_as_float((uint32_t)c[q] << 16);
+            xsum[i] = s;
+        }
         // one warp per router row (and the shared gate vector); a lane holds
         // 16 float4 of a 2048-wide slice of the row, loaded before any use
         float *racc = red + warp * kN;
-        const int rows = E + (A.has_shared ? 1 : 0);
-        for (int e = blockIdx.x + gridDim.x * warp; e < rows; e += gridDim.x * kWarps) {
+        for (int e = e_first; e < rows; e += gridDim.x * kWarps) {
             const float *wrow = e < E ? A.router_w + (size_t)e * H : A.shared_gate;
             for (int seg = 0; seg < H; seg += 2048) {
-                float4 wv[16];
+                if (e != e_first || seg != 0) {   // the first slice is already in registers
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const int kk = seg + (q * 32 + lane) * 4;
-                    wv[q] = kk < H ? __ldg((const float4 *)(wrow + kk)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int q = 0; q < 16; ++q) {
+                        const int kk = seg + (q * 32 + lane) * 4;
+                        wv[q] = kk < H ? __ldg((const float4 *)(wrow + kk)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
                 }
                 for (int t = 0; t < T; ++t) {
-                    const float *xt = big + (size_t)t * nchH * kPad;
+                    const uint16_t *xt = xb + (size_t)t * XS;
                     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
                         const int kk = seg + (q * 32 + lane) * 4;
                         if (kk < H) {
-                            const float4 xv = *(const float4 *)(xt + (kk / 32) * kPad + kk % 32);
-                            a0 = fmaf(wv[q].x, xv.x, a0);
-                            a1 = fmaf(wv[q].y, xv.y, a1);
-                            a0 = fmaf(wv[q].z, xv.z, a0);
-                            a1 = fmaf(wv[q].w, xv.w, a1);
+                            const uint2 xv = *(const uint2 *)(xt + kk);
+                            a0 = fmaf(wv[q].x, __uint_as_float(xv.x << 16), a0);
+                            a1 = fmaf(wv[q].y, __uint_as_float(xv.x & 0xFFFF0000u), a1);
+                            a0 = fmaf(wv[q].z, __uint_as_float(xv.y << 16), a0);
+                            a1 = fmaf(wv[q].w, __uint_as_float(xv.y & 0xFFFF0000u), a1);
                         }
                     }
                     float v = a0 + a1;
@@ -543,137 +638,200 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     const int NP = tk + (A.has_shared ? T : 0);
     DEC_MARK(3);
 
-    // ------------------------------------------------ C: gate/up + SwiGLU
+    // ------------------------------------------------ C: gate/up + SwiGLU (tensor cores)
     {
-        const int ngroups = WFMT == MOE_WFMT_Q4K ? H / 256 : H >> gshift;
+        const int gsh = WFMT == MOE_WFMT_Q4K ? 8 : gshift;
         const int per_slot = I / kFeat;
         const int U = Nd * per_slot;
-        float *part = red;   // [warp][token][lane]
-        GuLoad cur, nxt;
-        int u = blockIdx.x;
-        if (u < U)
-            gu_load<WFMT>(A, slot_e[u / per_slot], (u % per_slot) * kFeat, 0, nchH, ngroups, gshift, warp, lane, cur);
-        for (; u < U; u += gridDim.x) {
+        const int npass = (nchH + 4 * kWarps - 1) / (4 * kWarps);
+        // this warp's items: (unit u, pass), units u = blockIdx.x + gridDim.x i
+        const int nunits = U > (int)blockIdx.x ? (U - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+        const int nitems = nunits * npass;
+        auto unit_of = [&](int it) { return (int)blockIdx.x + (int)gridDim.x * (it / npass); };
+        auto stage = [&](int it2) {
+            if (it2 < nitems) {
+                const int u2 = unit_of(it2), pass2 = it2 % npass;
+                gu_stage<WFMT>(A, slot_e[u2 / per_slot], (u2 % per_slot) * kFeat, pass2 * 4 * kWarps, nchH, gsh, warp,
+                               lane, mybuf_s + (it2 % NS) * kIB);
+            }
+            cp_async_commit();
+        };
+        for (int it2 = 0; it2 < NS - 1; ++it2)
+            stage(it2);
+        float acc[2][4];
+        for (int it = 0; it < nitems; ++it) {
+            const int u = unit_of(it), pass = it % npass;
             const int d = u / per_slot, f0 = (u % per_slot) * kFeat;
             const int base = slot_base[d], cnt = slot_cnt[d];
-            for (int i = 0; i < cnt; ++i)
-                part[(warp * kN + i) * 32 + lane] = 0.f;
-            for (int j0 = 0; j0 < nchH; j0 += 4 * kWarps) {
-                // the next chunk group of this unit, or the first of the next unit
-                const int jn = j0 + 4 * kWarps;
-                const int un = u + gridDim.x;
-                if (jn < nchH)
-                    gu_load<WFMT>(A, slot_e[d], f0, jn, nchH, ngroups, gshift, warp, lane, nxt);
-                else if (un < U)
-                    gu_load<WFMT>(A, slot_e[un / per_slot], (un % per_slot) * kFeat, 0, nchH, ngroups, gshift, warp,
-                                  lane, nxt);
-                for (int i = 0; i < cnt; ++i) {
-                    const int t = pair_tok[base + i];
-                    float acc = 0.f;
+            stage(it + NS - 1);
+            if (pass == 0) {
 #pragma unroll
-                    for (int n = 0; n < 4; ++n) {
-                        const int j = j0 + warp + n * kWarps;
-                        if (j < nchH) {
-                            float c[32];
-                            decode_codes<kSym>(cur.cd[n], c);
-                            const float dot = dot32(c, big + ((size_t)t * nchH + j) * kPad);
-                            acc = fmaf(cur.ca[n], dot, fmaf(cur.cb[n], sums[t * nchH + j], acc));
-                        }
+                for (int m = 0; m < 2; ++m)
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        acc[m][v] = 0.f;
+            }
+            // this lane's B column: token gid of the unit's expert (zero row past cnt)
+            const int trow = gid < cnt ? pair_tok[base + gid] : kN;
+            const int tA = 2 * tid4 < cnt ? pair_tok[base + 2 * tid4] : -1;
+            const int tB = 2 * tid4 + 1 < cnt ? pair_tok[base + 2 * tid4 + 1] : -1;
+            cp_async_wait_upto(NS - 1);   // item it's copies have landed
+            __syncwarp();
+            const uint8_t *buf = mybuf + (it % NS) * kIB;
+            for (int n = 0; n < 4; ++n) {
+                const int j = pass * 4 * kWarps + warp + kWarps * n;
+                if (j >= nchH)
+                    break;
+                float cs[2][2][2];   // [matrix][row lo/hi][a, b]
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    const uint8_t *mrow = buf + kCodeBuf + ((n * 2 + m) * 16 + gid) * kMB;
+                    staged_coeffs<WFMT>(mrow, j * 32, cs[m][0][0], cs[m][0][1]);
+                    staged_coeffs<WFMT>(mrow + 8 * kMB, j * 32, cs[m][1][0], cs[m][1][1]);
+                }
+                const float sA = tA >= 0 ? xsum[tA * nchH + j] : 0.f;
+                const float sB = tB >= 0 ? xsum[tB * nchH + j] : 0.f;
+                const uint16_t *brow = xb + (size_t)trow * XS + j * 32;
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    const uint4 lo = *(const uint4 *)(buf + ((n * 2 + m) * 16 + gid) * 16);
+                    const uint4 hi = *(const uint4 *)(buf + ((n * 2 + m) * 16 + gid + 8) * 16);
+                    float dd[4] = {0.f, 0.f, 0.f, 0.f};
+                    chunk_mma(dd, lo, hi, brow, tid4);
+                    // rows gid (v = 0, 1) and gid + 8 (v = 2, 3); tokens 2 tid4 + (v & 1)
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const float sx = (v & 1) ? sB : sA;
+                        const float a = cs[m][v >> 1][0], b = cs[m][v >> 1][1];
+                        acc[m][v] = fmaf(a, fmaf(-kOff, sx, dd[v]), fmaf(b, sx, acc[m][v]));
                     }
-                    part[(warp * kN + i) * 32 + lane] += acc;
                 }
-                cur = nxt;
             }
-            __syncthreads();
-            // feature f of the unit for its token i: gate and up sums over the warps, in order
-            if (tid < kFeat * cnt) {
-                const int i = tid / kFeat, f = tid % kFeat;
-                float g = 0.f, v = 0.f;
-                for (int w = 0; w < kWarps; ++w) {
-                    g += part[(w * kN + i) * 32 + f];
-                    v += part[(w * kN + i) * 32 + kFeat + f];
+            __syncwarp();
+            if (pass == npass - 1) {
+                // the unit is complete in every warp: gate and up summed over the warps, in order
+#pragma unroll
+                for (int m = 0; m < 2; ++m)
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        red[((warp * 2 + m) * 16 + gid + 8 * (v >> 1)) * kN + 2 * tid4 + (v & 1)] = acc[m][v];
+                __syncthreads();
+                if (tid < kFeat * cnt) {
+                    const int nn = tid / kFeat, f = tid % kFeat;
+                    float g = 0.f, uu = 0.f;
+                    for (int w = 0; w < kWarps; ++w) {
+                        g += red[((w * 2 + 0) * 16 + f) * kN + nn];
+                        uu += red[((w * 2 + 1) * 16 + f) * kN + nn];
+                    }
+                    const float hv = g / (1.0f + expf(-g)) * uu;
+                    A.h[(size_t)(base + nn) * I + f0 + f] = (uint16_t)(pack_bf16x2(hv, 0.f) & 0xFFFFu);
                 }
-                A.h[(size_t)(base + i) * I + f0 + f] = g / (1.0f + expf(-g)) * v;
+                __syncthreads();
             }
-            __syncthreads();
         }
+        cp_async_wait_group<0>();
+        __syncwarp();
     }
     DEC_MARK(4);
     if (!grid_sync(A.bar, A.status, 92, flag))
         return;
     DEC_MARK(5);
 
-    // ------------------------------------------------ D: down + combine
+    // ------------------------------------------------ D: down + combine (tensor cores)
     {
-        float *hs = big;
-        for (int i = tid; i < NP * (I / 4); i += kThreads) {
-            const int p = i / (I / 4), kk = (i % (I / 4)) * 4;
-            const float4 v = __ldcg((const float4 *)(A.h + (size_t)p * I + kk));
-            *(float4 *)(hs + ((size_t)p * nchI + kk / 32) * kPad + kk % 32) = v;
+        // h as bf16 rows of I + 8 elements (row NP is zeros) and fp32 chunk sums
+        const int HS = I + 8;
+        uint16_t *hb = (uint16_t *)(smem + L.big);
+        float *hsum = (float *)(hb + (size_t)(NP + 1) * HS);
+        for (int i = tid; i < (NP + 1) * (I / 8); i += kThreads) {
+            const int p = i / (I / 8), kk = (i % (I / 8)) * 8;
+            const uint4 v = p < NP ? __ldcg((const uint4 *)(A.h + (size_t)p * I + kk)) : make_uint4(0, 0, 0, 0);
+            *(uint4 *)(hb + (size_t)p * HS + kk) = v;
         }
         __syncthreads();
-        for (int i = tid; i < NP * nchI; i += kThreads)
-            sums[i] = chunk_sum(hs + (size_t)i * kPad);
+        for (int i = tid; i < NP * nchI; i += kThreads) {
+            const uint16_t *c = hb + (size_t)(i / nchI) * HS + (i % nchI) * 32;
+            float s = 0.f;
+            for (int q = 0; q < 32; ++q)
+                s += __uint_as_float((uint32_t)c[q] << 16);
+            hsum[i] = s;
+        }
         __syncthreads();
-        const int F = H / kTileRows, KS = I / kKStep, ngroups = WFMT == MOE_WFMT_Q4K ? I / 256 : I >> gshift;
-        // lanes per row: the power of two >= I / 32 chunks (at most 32);
-        // a slot pass covers kCols rows of one expert, SP passes side by side
-        int LJ = 1;
-        while (LJ < nchI)
-            LJ <<= 1;
-        const int per_pass = kCols * LJ;                // threads of one slot pass (>= 32: warp-uniform)
-        const int SP = kThreads / per_pass;
-        const int sub = tid / per_pass, cc = (tid / LJ) % kCols, j = tid % LJ;
+        const int gsh = WFMT == MOE_WFMT_Q4K ? 8 : gshift;
+        const int nparts = (nchI + 7) / 8;
         float *o_s = red;   // [pair][column]
+        // this warp's slots: d = warp + kWarps i; items (slot, part)
+        const int nslots = Nd > warp ? (Nd - 1 - warp) / kWarps + 1 : 0;
+        const int nitems = nslots * nparts;
         for (int u = blockIdx.x; u < H / kCols; u += gridDim.x) {
-            const int C = u * kCols + cc;
-            const int r = C % kTileRows;
-            for (int d0 = 0; d0 < Nd; d0 += SP * kDnBatch) {
-                uint4 cd[kDnBatch];
-                float ca[kDnBatch], cb[kDnBatch];
+            const int c0 = u * kCols;
+            auto stage = [&](int it2) {
+                if (it2 < nitems)
+                    dn_stage<WFMT>(A, slot_e[warp + kWarps * (it2 / nparts)], c0, it2 % nparts, nchI, gsh, lane,
+                                   mybuf_s + (it2 % NS) * kIB);
+                cp_async_commit();
+            };
+            for (int it2 = 0; it2 < NS - 1; ++it2)
+                stage(it2);
+            float acc[4];
+            for (int it = 0; it < nitems; ++it) {
+                const int d = warp + kWarps * (it / nparts), q = it % nparts;
+                const int base = slot_base[d], cnt = slot_cnt[d];
+                stage(it + NS - 1);
+                if (q == 0) {
 #pragma unroll
-                for (int b = 0; b < kDnBatch; ++b) {
-                    const int d = d0 + b * SP + sub;
-                    cd[b] = make_uint4(0, 0, 0, 0);
-                    ca[b] = cb[b] = 0.f;
-                    if (d < Nd && j < nchI) {
-                        const size_t tile = (size_t)slot_e[d] * F + C / kTileRows;
-                        cd[b] = __ldg((const uint4 *)(A.dn_q + (tile * KS + (j >> 1)) * code_block_bytes(1) +
-                                                      ((size_t)(j & 1) * kTileRows + r) * kChunkBytes));
-                        chunk_coeffs<WFMT>(A.dn_meta + tile * A.dn_meta_bytes, 0, ngroups, r, j * 32, gshift, ca[b],
-                                           cb[b]);
+                    for (int v = 0; v < 4; ++v)
+                        acc[v] = 0.f;
+                }
+                const int prow = gid < cnt ? base + gid : NP;
+                const int pA = 2 * tid4 < cnt ? base + 2 * tid4 : -1;
+                const int pB = 2 * tid4 + 1 < cnt ? base + 2 * tid4 + 1 : -1;
+                cp_async_wait_upto(NS - 1);
+                __syncwarp();
+                const uint8_t *buf = mybuf + (it % NS) * kIB;
+                for (int n = 0; n < 8; ++n) {
+                    const int j = 8 * q + n;
+                    if (j >= nchI)
+                        break;
+                    float clo_a, clo_b, chi_a, chi_b;
+                    const uint8_t *mrow = buf + kCodeBuf + (n * 16 + gid) * kMB;
+                    staged_coeffs<WFMT>(mrow, j * 32, clo_a, clo_b);
+                    staged_coeffs<WFMT>(mrow + 8 * kMB, j * 32, chi_a, chi_b);
+                    const float sA = pA >= 0 ? hsum[pA * nchI + j] : 0.f;
+                    const float sB = pB >= 0 ? hsum[pB * nchI + j] : 0.f;
+                    const uint4 lo = *(const uint4 *)(buf + (n * 16 + gid) * 16);
+                    const uint4 hi = *(const uint4 *)(buf + (n * 16 + gid + 8) * 16);
+                    float dd[4] = {0.f, 0.f, 0.f, 0.f};
+                    chunk_mma(dd, lo, hi, hb + (size_t)prow * HS + j * 32, tid4);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const float sx = (v & 1) ? sB : sA;
+                        const float a = (v >> 1) ? chi_a : clo_a, b = (v >> 1) ? chi_b : clo_b;
+                        acc[v] = fmaf(a, fmaf(-kOff, sx, dd[v]), fmaf(b, sx, acc[v]));
                     }
                 }
+                __syncwarp();
+                if (q == nparts - 1) {
+                    // o[pair][column] for the slot's pairs: rows gid, gid + 8 are columns of y
 #pragma unroll
-                for (int b = 0; b < kDnBatch; ++b) {
-                    const int d = d0 + b * SP + sub;
-                    if (d >= Nd)
-                        continue;   // uniform over the pass's threads, which span whole warps
-                    const int base = slot_base[d], cnt = slot_cnt[d];
-                    float c[32];
-                    decode_codes<kSym>(cd[b], c);
-                    for (int i = 0; i < cnt; ++i) {
-                        const int p = base + i;
-                        float v = 0.f;
-                        if (j < nchI)
-                            v = fmaf(ca[b], dot32(c, hs + ((size_t)p * nchI + j) * kPad), cb[b] * sums[p * nchI + j]);
-                        for (int o = LJ >> 1; o > 0; o >>= 1)
-                            v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-                        if (j == 0)
-                            o_s[p * kCols + cc] = v;
+                    for (int v = 0; v < 4; ++v) {
+                        const int nn = 2 * tid4 + (v & 1);
+                        if (nn < cnt)
+                            o_s[(base + nn) * kCols + gid + 8 * (v >> 1)] = acc[v];
                     }
                 }
             }
+            cp_async_wait_group<0>();
             __syncthreads();
             // the combine of these columns: routed experts in j order, then the shared expert
             if (tid < T * kCols) {
                 const int t = tid / kCols, c2 = tid % kCols;
-                float acc = 0.f;
+                float y = 0.f;
                 for (int jj = 0; jj < k; ++jj)
-                    acc = fmaf(w_s[t * k + jj], o_s[pidx[t * k + jj] * kCols + c2], acc);
+                    y = fmaf(w_s[t * k + jj], o_s[pidx[t * k + jj] * kCols + c2], y);
                 if (A.has_shared)
-                    acc = fmaf(w_s[tk + t], o_s[(tk + t) * kCols + c2], acc);
-                A.y[(size_t)t * H + u * kCols + c2] = (uint16_t)(pack_bf16x2(acc, 0.f) & 0xFFFFu);
+                    y = fmaf(w_s[tk + t], o_s[(tk + t) * kCols + c2], y);
+                A.y[(size_t)t * H + c0 + c2] = (uint16_t)(pack_bf16x2(y, 0.f) & 0xFFFFu);
             }
             __syncthreads();
         }
@@ -685,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
 
 cudaError_t launch_decode_layer(const DecodeArgs &a, int grid, cudaStream_t st)
 {
-    const DecodeSmem L = decode_smem_layout(a.T, a.k, a.H, a.I, a.has_shared);
+    const DecodeSmem L = decode_smem_layout(a.T, a.k, a.H, a.I, a.has_shared, a.wfmt);
     void (*kern)(const DecodeArgs, const DecodeSmem) =
         a.wfmt == MOE_WFMT_Q4K         ? decode_layer_kernel<MOE_WFMT_Q4K>
         : a.wfmt == MOE_WFMT_INT4_ASYM ? decode_layer_kernel<MOE_WFMT_INT4_ASYM>

@@ -10,6 +10,7 @@ namespace moeq4 {
 
 constexpr int kDecodeMaxT = 8;
 constexpr int kDecodeThreads = 512;
+constexpr size_t kDecodeSmemLimit = 227 * 1024;   // dynamic shared memory of one CTA
 
 struct DecodeArgs {
     const uint16_t *x;          // [T, H] bf16
@@ -25,7 +26,7 @@ struct DecodeArgs {
     float *gate_logit;          // [T]
     int32_t *topk_ids;          // [T, k]
     float *topk_w;              // [T, k]
-    float *h;                   // [NP, I] gate/up outputs, NP = T k (+ T)
+    uint16_t *h;                // [NP, I] gate/up outputs (bf16), NP = T k (+ T)
     uint16_t *y;                // [T, H] bf16
     int *status;                // [code, detail]
     unsigned *bar;              // [count, generation, abort] of the grid barrier
@@ -33,10 +34,11 @@ struct DecodeArgs {
 
 // Byte offsets of the decode kernel's dynamic shared memory.
 struct DecodeSmem {
-    int big, sums, red, ids, w, pidx, pair_tok, pair_w, slot_e, slot_base, slot_cnt, bitmap, wprefix, flag;
+    int big, sums, red, cbuf, ids, w, pidx, pair_tok, pair_w, slot_e, slot_base, slot_cnt, bitmap, wprefix, flag;
+    int nstage;   // depth of each warp's staging ring
     size_t bytes;
 };
-DecodeSmem decode_smem_layout(int T, int k, int H, int I, int has_shared);
+DecodeSmem decode_smem_layout(int T, int k, int H, int I, int has_shared, int wfmt);
 cudaError_t launch_decode_layer(const DecodeArgs &a, int grid, cudaStream_t st);
 
 }  // namespace moeq4

@@ -193,8 +193,8 @@ def test_decode_admission_and_workspace(L):
     # a3b shape: T = 1..8 admitted, 9 and more go through moe_layer_forward
     sizes = [L.moe_layer_decode_workspace_size(C.byref(c), t) for t in (1, 2, 8)]
     assert 0 < sizes[0] < sizes[1] < sizes[2]
-    # h in fp32 for T k + T pairs (the expert outputs never leave shared memory)
-    assert sizes[2] >= (8 * 8 + 8) * 512 * 4
+    # h in bf16 for T k + T pairs (the expert outputs never leave shared memory)
+    assert sizes[2] >= (8 * 8 + 8) * 512 * 2
     assert L.moe_layer_decode_workspace_size(C.byref(c), 9) == 0
     layer = mq.Layer(c, 0x1000, None, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000)
     rc = L.moe_layer_decode(C.byref(layer), 0x1000, 9, 0x1000, 0x1000, 1 << 30, None, None)
