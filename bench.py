@@ -57,7 +57,7 @@ def expert_bytes(cfg) -> tuple:
     return gu, dn
 
 
-WFMT_NAMES = {0: "int4-sym", 1: "q4k", 2: "int4-asym"}
+WFMT_NAMES = {0: "int4-sym", 1: "q4k", 2: "int4-asym", 3: "int4-sym, fp16 operands"}
 L2_BYTES = 126e6   # B200 L2
 
 
@@ -443,7 +443,8 @@ def extra_config(name, dev, stream, steps, warmup, decode):
     return out
 
 
-DEFAULT_EXTRAS = ("a3b_t512", "a3b_t4096_q4k", "a3b_decode_t1", "a3b_decode_t8", "a3b_decode_t32")
+DEFAULT_EXTRAS = ("a3b_t512", "a3b_t4096_q4k", "a3b_t8192_zipf_f16", "a3b_decode_t1", "a3b_decode_t8",
+                  "a3b_decode_t32")
 
 
 def main():

@@ -56,6 +56,18 @@ extern "C" {
 #define MOE_WFMT_INT4_SYM 0 /* int4 two's complement, one bf16 scale per G weights along K */
 #define MOE_WFMT_Q4K 1      /* Q4_K-style 256-weight super-blocks (see moe_pack_weights)   */
 #define MOE_WFMT_INT4_ASYM 2 /* unsigned int4, a bf16 scale and a bf16 minimum per G weights */
+/* The int4-sym weights above (same canonical input), computed with fp16
+ * tensor-core operands: q*s has at most 11 significant bits, so every
+ * dequantised weight is exact in fp16 (scales in [2^-17, 8188], checked
+ * by moe_pack_weights); the activations x enter as fp16 (exact for bf16
+ * values with 2^-17 <= |x| <= 65504; smaller ones are rounded, within
+ * 2^-25; larger ones are refused at run time), and the SwiGLU output h
+ * is kept in fp16.  This is the library's own exact-weight route for the
+ * symmetric experts (the pages' late-prefill steps on the mq4rs file keep
+ * their routes byte-exact: hipfire 0.4.3 benchmarks, "Late prefill steps
+ * on mq4rs"; an F16 operand route appears there for another model's 6-bit
+ * file, in the Flash-Next prefill table). */
+#define MOE_WFMT_INT4_SYM_F16 3
 
 /* Shapes of one layer.  Admitted: H % 128 == 0, I % 128 == 0, 1 <= k <= E <= 1024,
  * int4-sym / int4-asym: G a power of two, G >= 32, G divides H and I; Q4K: H % 256 == 0,
@@ -131,6 +143,11 @@ int moe_packed_sizes(const moe_config_t *cfg, size_t *gu_q_bytes, size_t *gu_met
  *             uint16 [rows, K/G, 2]; w = q*s + m (the pages' asymmetric
  *             mq4r file; the recipe is this library's reading);
  *   gu_scale / dn_scale are ignored (may be NULL) for Q4K.
+ *   int4-sym-f16: the int4-sym input; the scales are stored as fp16.
+ *             The call then synchronises `stream` and returns
+ *             MOE_ERR_UNSUPPORTED if a scale lies outside [2^-17, 8188]
+ *             (or is not finite), where q*s would not be exact in fp16;
+ *             zero scales are accepted.
  * Outputs go to caller buffers of the sizes moe_packed_sizes() returns.
  * Source: hipfire 0.4.3 benchmarks, "Read this before comparing columns"
  * (symmetric-expert mq4rs file); hipEngine post, "GGUF" (Q4_K).  The bit
@@ -248,6 +265,7 @@ int moe_expert_ffn_q4(const moe_layer_t *L, const uint16_t *x, int T, const int3
  * The two passes of moe_expert_ffn_q4, for callers that want them apart
  * (same kernels, same results):
  *   gate/up:  h[p] = bf16( silu(x[t] Wg_e^T) * (x[t] Wu_e^T) ),  h [T k (+ T), I]
+ *             (fp16 instead of bf16 in the fp16-operand mode, MOE_WFMT_INT4_SYM_F16)
  *             (rows T k .. T k + T - 1 are the shared expert's, token t = p - T k)
  *   down:     y_perm[p] = bf16( h[p] Wd_e^T ), shared_out[t] = bf16( h[T k + t] Wd_s^T )
  * ws: moe_expert_ffn_workspace_size (the h buffer inside it is not used).

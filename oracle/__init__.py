@@ -27,6 +27,7 @@ _lib = None
 WFMT_INT4_SYM = 0
 WFMT_Q4K = 1
 WFMT_INT4_ASYM = 2
+WFMT_INT4_SYM_F16 = 3   # a GPU operand precision of the int4-sym layer: the same layer here
 
 
 def build(force: bool = False) -> str:
@@ -178,12 +179,13 @@ def layer_forward(layer: dict, sample=None, override_ids=None, override_w=None):
 
     A = _LayerArgs()
     A.T, A.H, A.E, A.k, A.I = T, H, E, k, I
-    A.has_shared, A.wfmt, A.G, A.renorm = int(cfg.has_shared), cfg.wfmt, cfg.G, int(cfg.renorm)
+    wfmt = WFMT_INT4_SYM if cfg.wfmt == WFMT_INT4_SYM_F16 else cfg.wfmt
+    A.has_shared, A.wfmt, A.G, A.renorm = int(cfg.has_shared), wfmt, cfg.G, int(cfg.renorm)
     A.x = arr("x", layer["x"], np.uint16)
     A.router_w = arr("wr", layer["router_w"], np.float32)
     A.router_bias = arr("rb", layer.get("router_bias"), np.float32)
     A.shared_gate = arr("sg", layer.get("shared_gate"), np.float32)
-    if cfg.wfmt in (WFMT_INT4_SYM, WFMT_INT4_ASYM):
+    if wfmt in (WFMT_INT4_SYM, WFMT_INT4_ASYM):
         A.gu_q = arr("guq", layer["gu_nib"], np.uint8)
         A.gu_scale = arr("gus", layer["gu_scale"], np.uint16)
         A.dn_q = arr("dnq", layer["dn_nib"], np.uint8)

@@ -17,7 +17,8 @@ __all__ = [
     "moe_dequant_export", "moe_router_workspace_size", "moe_router_logits", "moe_route", "moe_permute_workspace_size", "moe_permute",
     "moe_expert_ffn_workspace_size", "moe_expert_ffn_q4", "moe_combine", "moe_layer_workspace_size",
     "moe_layer_forward", "moe_layer_forward_chunked", "moe_layer_decode_workspace_size", "moe_layer_decode", "moe_read_status", "moe_kernel_launches", "moe_expert_gate_up_q4", "moe_expert_down_q4",
-    "moe_permute_noalloc", "PackedLayer", "WFMT_INT4_SYM", "WFMT_Q4K", "WFMT_INT4_ASYM", "LIB_PATH",
+    "moe_permute_noalloc", "PackedLayer", "WFMT_INT4_SYM", "WFMT_Q4K", "WFMT_INT4_ASYM", "WFMT_INT4_SYM_F16",
+    "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoeq4.so")
@@ -31,6 +32,7 @@ MOE_ERR_WORKSPACE = -5
 WFMT_INT4_SYM = 0
 WFMT_Q4K = 1
 WFMT_INT4_ASYM = 2
+WFMT_INT4_SYM_F16 = 3
 
 _NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_CUDA",
           -4: "MOE_ERR_TIMEOUT", -5: "MOE_ERR_WORKSPACE"}

@@ -121,13 +121,14 @@ int check_config(const moe_config_t *c)
         return fail(MOE_ERR_INVALID_ARG, "cfg: null pointer");
     if (c->H <= 0 || c->I <= 0 || c->E <= 0 || c->k <= 0)
         return fail(MOE_ERR_INVALID_ARG, "cfg: H, I, E, k must be positive");
-    if (c->wfmt != MOE_WFMT_INT4_SYM && c->wfmt != MOE_WFMT_Q4K && c->wfmt != MOE_WFMT_INT4_ASYM)
+    if (c->wfmt != MOE_WFMT_INT4_SYM && c->wfmt != MOE_WFMT_Q4K && c->wfmt != MOE_WFMT_INT4_ASYM &&
+        c->wfmt != MOE_WFMT_INT4_SYM_F16)
         return fail(MOE_ERR_UNSUPPORTED, "cfg: unknown weight format %d", c->wfmt);
     if (c->H % 128 || c->I % 128)
         return fail(MOE_ERR_UNSUPPORTED, "cfg: H (%d) and I (%d) must be multiples of 128", c->H, c->I);
     if (c->E > 1024 || c->k > 32 || c->k > c->E)
         return fail(MOE_ERR_UNSUPPORTED, "cfg: need k <= min(E, 32) and E <= 1024 (E=%d k=%d)", c->E, c->k);
-    if (c->wfmt == MOE_WFMT_INT4_SYM || c->wfmt == MOE_WFMT_INT4_ASYM) {
+    if (c->wfmt != MOE_WFMT_Q4K) {
         if (c->G < 32 || (c->G & (c->G - 1)) || c->H % c->G || c->I % c->G)
             return fail(MOE_ERR_UNSUPPORTED, "cfg: int4 group G=%d must be a power of two >= 32 dividing H and I",
                         c->G);
@@ -155,7 +156,8 @@ struct FfnWs {
 };
 
 // with_xperm = false: the caller lends the permuted-row buffer (the fused
-// layer lends y_perm, which is dead until the down pass writes it).
+// layer lends y_perm and the shared_out buffer right after it, both dead
+// until the down pass writes them).
 FfnWs ffn_layout(const moe_config_t *c, int T, uint8_t *base, bool with_xperm = true)
 {
     FfnWs w{};
@@ -163,8 +165,9 @@ FfnWs ffn_layout(const moe_config_t *c, int T, uint8_t *base, bool with_xperm = 
     w.h = (uint16_t *)(base + off);
     off += align256(sizeof(uint16_t) * ((size_t)T * c->k + (c->has_shared ? T : 0)) * c->I);
     if (with_xperm) {
+        // the routed rows, and in the fp16-operand mode the shared expert's rows after them
         w.x_perm = (uint16_t *)(base + off);
-        off += align256(sizeof(uint16_t) * (size_t)T * c->k * c->H);
+        off += align256(sizeof(uint16_t) * ((size_t)T * c->k + (c->has_shared ? T : 0)) * c->H);
     }
     w.bytes = off;
     return w;
@@ -300,17 +303,21 @@ int run_expert_ffn(const moe_layer_t *L, const uint16_t *x, int T, const int32_t
     a.E_total = Et;
     a.G = c.G;
     a.status = status;
+    const bool f16 = c.wfmt == MOE_WFMT_INT4_SYM_F16;
     if (pass & 1) {
-        // the routed experts' token rows, permuted into contiguous blocks
-        CUDA_TRY(launch_gather_rows(x, sorted_slot, Tk, c.k, c.H, x_perm, num_sms(), st), "gather rows");
+        // the routed experts' token rows, permuted into contiguous blocks (in
+        // the fp16-operand mode as fp16, the shared expert's rows appended)
+        const int shared_rows = f16 && c.has_shared ? T : 0;
+        CUDA_TRY(launch_gather_rows(x, sorted_slot, Tk, c.k, c.H, x_perm, num_sms(), st, shared_rows, f16, status),
+                 "gather rows");
         g_launches += 1;
         // gate/up + SwiGLU -> h [Tk + T, I]
         a.wq = (const uint8_t *)L->gu_q;
         a.wmeta = (const uint8_t *)L->gu_meta;
         a.b_src = x_perm;
         a.ldb = c.H;
-        a.b_rows = Tk;
-        a.b_src2 = c.has_shared ? x : nullptr;
+        a.b_rows = Tk + shared_rows;
+        a.b_src2 = c.has_shared && !f16 ? x : nullptr;
         a.b_rows2 = T;
         a.K = c.H;
         a.F = c.I / kTileRows;
@@ -382,7 +389,7 @@ int moe_pack_weights(const moe_config_t *cfg, const void *gu_canon, const void *
     if (rc)
         return rc;
     REQUIRE(gu_canon && dn_canon, "canonical weights: null pointer");
-    if (cfg->wfmt == MOE_WFMT_INT4_SYM || cfg->wfmt == MOE_WFMT_INT4_ASYM)
+    if (cfg->wfmt != MOE_WFMT_Q4K)
         REQUIRE(gu_scale && dn_scale, "int4 scales: null pointer");
     REQUIRE_PTR(gu_q);
     REQUIRE_PTR(gu_meta);
@@ -391,10 +398,16 @@ int moe_pack_weights(const moe_config_t *cfg, const void *gu_canon, const void *
     cudaStream_t st = (cudaStream_t)stream;
     CUDA_TRY(launch_pack_codes(*cfg, 0, (const uint8_t *)gu_canon, (uint8_t *)gu_q, st), "pack gate/up codes");
     CUDA_TRY(launch_pack_codes(*cfg, 1, (const uint8_t *)dn_canon, (uint8_t *)dn_q, st), "pack down codes");
-    CUDA_TRY(launch_pack_meta(*cfg, 0, (const uint8_t *)gu_canon, (const uint16_t *)gu_scale, (uint8_t *)gu_meta, st),
+    unsigned misfits = 0;
+    CUDA_TRY(launch_pack_meta(*cfg, 0, (const uint8_t *)gu_canon, (const uint16_t *)gu_scale, (uint8_t *)gu_meta, st,
+                              &misfits),
              "pack gate/up scales");
-    CUDA_TRY(launch_pack_meta(*cfg, 1, (const uint8_t *)dn_canon, (const uint16_t *)dn_scale, (uint8_t *)dn_meta, st),
+    CUDA_TRY(launch_pack_meta(*cfg, 1, (const uint8_t *)dn_canon, (const uint16_t *)dn_scale, (uint8_t *)dn_meta, st,
+                              &misfits),
              "pack down scales");
+    if (misfits)
+        return fail(MOE_ERR_UNSUPPORTED,
+                    "fp16-operand mode: %u scales lie outside [2^-17, 8188], where q*s is not exact in fp16", misfits);
     return ok();
 }
 

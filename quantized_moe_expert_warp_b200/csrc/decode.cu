@@ -170,6 +170,9 @@ __device__ __forceinline__ void staged_coeffs(const uint8_t *mrow, int kpos, flo
         const uint32_t sm = *(const uint32_t *)mrow;
         a = __uint_as_float(sm << 16);
         b = __uint_as_float(sm & 0xFFFF0000u);
+    } else if (WFMT == MOE_WFMT_INT4_SYM_F16) {
+        a = __half2float(__ushort_as_half(*(const uint16_t *)mrow));
+        b = 0.f;
     } else {
         a = __uint_as_float((uint32_t) * (const uint16_t *)mrow << 16);
         b = 0.f;
@@ -440,7 +443,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     int *wprefix = (int *)(smem + L.wprefix);
     int *flag = (int *)(smem + L.flag);
 
-    constexpr float kOff = WFMT == MOE_WFMT_INT4_SYM ? 136.f : 128.f;   // code pair value minus the code
+    // code pair value minus the code
+    constexpr float kOff = WFMT == MOE_WFMT_INT4_SYM || WFMT == MOE_WFMT_INT4_SYM_F16 ? 136.f : 128.f;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tid4 = lane & 3;
     const int T = A.T, H = A.H, I = A.I, E = A.E, k = A.k;
@@ -845,17 +849,18 @@ cudaError_t launch_decode_layer(const DecodeArgs &a, int grid, cudaStream_t st)
 {
     const DecodeSmem L = decode_smem_layout(a.T, a.k, a.H, a.I, a.has_shared, a.wfmt);
     void (*kern)(const DecodeArgs, const DecodeSmem) =
-        a.wfmt == MOE_WFMT_Q4K         ? decode_layer_kernel<MOE_WFMT_Q4K>
-        : a.wfmt == MOE_WFMT_INT4_ASYM ? decode_layer_kernel<MOE_WFMT_INT4_ASYM>
-                                       : decode_layer_kernel<MOE_WFMT_INT4_SYM>;
+        a.wfmt == MOE_WFMT_Q4K             ? decode_layer_kernel<MOE_WFMT_Q4K>
+        : a.wfmt == MOE_WFMT_INT4_ASYM     ? decode_layer_kernel<MOE_WFMT_INT4_ASYM>
+        : a.wfmt == MOE_WFMT_INT4_SYM_F16 ? decode_layer_kernel<MOE_WFMT_INT4_SYM_F16>
+                                           : decode_layer_kernel<MOE_WFMT_INT4_SYM>;
     // the opt-in limit once per device and format (callers never ask for
     // more: see the admission check)
-    static std::atomic<bool> configured[64][3];
+    static std::atomic<bool> configured[64][4];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
-    const int f = a.wfmt == MOE_WFMT_Q4K ? 1 : a.wfmt == MOE_WFMT_INT4_ASYM ? 2 : 0;
+    const int f = a.wfmt >= 0 && a.wfmt < 4 ? a.wfmt : 0;
     if (dev < 0 || dev >= 64 || !configured[dev][f].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess)

@@ -12,7 +12,8 @@
 //          are stored offset-binary (q + 8), Q4K and int4-asym codes as they
 //          are (0..15).
 //   meta:  per (expert, tile f) a contiguous block, ordered [m][group][row]:
-//          int4-sym: bf16 scale of group g (K/G groups);
+//          int4-sym: bf16 scale of group g (K/G groups; fp16 for the
+//                    fp16-operand mode);
 //          int4-asym: bf16 scale (low half) and bf16 minimum (high half);
 //          Q4K:      the 16-byte super-block header (fp16 d, fp16 dmin,
 //                    12 bytes of 6-bit sc/m fields) of super-block g.
@@ -38,7 +39,7 @@ __host__ __device__ inline int meta_block_bytes(int nmat, int wfmt, int K, int G
 {
     return wfmt == MOE_WFMT_Q4K        ? nmat * (K / 256) * kTileRows * 16
            : wfmt == MOE_WFMT_INT4_ASYM ? nmat * (K / G) * kTileRows * 4
-                                        : nmat * (K / G) * kTileRows * 2;
+                                        : nmat * (K / G) * kTileRows * 2;   // int4-sym, bf16 or fp16 scale
 }
 
 __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b)
@@ -78,6 +79,47 @@ __device__ __forceinline__ void dequant_int4sym_chunk(const uint4 codes, uint16_
             out[wi * 4 + i] = bf16x2_mul(bf16x2_sub(t, off), s2);
         }
     }
+}
+
+__device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// int4-sym with an fp16 scale: 32 codes (offset-binary) -> 16 words of fp16
+// pairs.  (1024 + u) - 1032 = q exactly, and q * s (at most 11 significant
+// bits) is exact in fp16, so no step rounds.
+__device__ __forceinline__ void dequant_int4sym_f16_chunk(const uint4 codes, uint16_t scale_bits, uint32_t (&out)[16])
+{
+    const uint32_t s2 = (uint32_t)scale_bits | ((uint32_t)scale_bits << 16);
+    const uint32_t off = 0x64086408u;   // fp16 1032.0 in both halves
+    const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t t = ((w[wi] >> (4 * i)) & 0x000F000Fu) | 0x64006400u;   // fp16 pair (1024+u_lo, 1024+u_hi)
+            out[wi * 4 + i] = f16x2_mul(f16x2_sub(t, off), s2);
+        }
+    }
+}
+
+__device__ __forceinline__ float int4sym_f16_value(const uint4 codes, uint16_t scale_bits, int e)
+{
+    const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+    const int wi = e / 8, j = e % 8;
+    const int nib = (j & 1) ? (j >> 1) + 4 : (j >> 1);
+    const int u = (w[wi] >> (4 * nib)) & 0xF;
+    return (float)(u - 8) * __half2float(__ushort_as_half(scale_bits));
 }
 
 __device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c)

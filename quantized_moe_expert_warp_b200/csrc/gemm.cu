@@ -33,6 +33,7 @@
 // Every wait is bounded; on timeout the CTA records MOE_ERR_TIMEOUT and
 // unwinds.
 #include <cstdint>
+#include <cuda_fp16.h>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -424,7 +425,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++uidx) {
             const Unit un = decode_unit<BN>(u, p, sched);
-            const uint32_t idesc = idesc_bf16_f32(128, un.nmma);
+            // fp16-operand mode: fp16 weights and tokens (the router stays bf16)
+            const uint32_t idesc = WFMT == MOE_WFMT_INT4_SYM_F16 && MODE != MODE_ROUTER ? idesc_f16_f32(128, un.nmma)
+                                                                                        : idesc_bf16_f32(128, un.nmma);
             const int ab = uidx % L::kAccBufs;
             const uint32_t acc = tmem + ab * L::kNAcc * kBN;
             CYC(4);
@@ -715,6 +718,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 const int g = kpos >> gshift;
                                 const uint32_t sm = lds32(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 4);
                                 dequant_int4asym_chunk(codes, sm, words[m]);
+                            } else if (WFMT == MOE_WFMT_INT4_SYM_F16) {
+                                const int g = kpos >> gshift;
+                                const uint16_t sbits = lds16(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 2);
+                                dequant_int4sym_f16_chunk(codes, sbits, words[m]);
                             } else {
                                 const int g = kpos >> gshift;
                                 const uint16_t sbits = lds16(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 2);
@@ -839,7 +846,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         } else {
                             o = __uint_as_float(g[j]);
                         }
-                        *(__nv_bfloat16 *)(stage + j * kEpiStride + lane * 2) = __float2bfloat16_rn(o);
+                        // h is fp16 in the fp16-operand mode (the down pass's operand); Y is bf16
+                        if (MODE == MODE_GATE_UP && WFMT == MOE_WFMT_INT4_SYM_F16)
+                            *(__half *)(stage + j * kEpiStride + lane * 2) = __float2half_rn(o);
+                        else
+                            *(__nv_bfloat16 *)(stage + j * kEpiStride + lane * 2) = __float2bfloat16_rn(o);
                     }
                     __syncwarp();
                     // lane: token n0 + (lane & 15), 32-byte half (lane >> 4) of the warp's 64-byte row slice
@@ -1036,9 +1047,10 @@ int gemm_down_tile_tokens(int T, int E, int k)
 template <int MODE, int BN>
 static cudaError_t launch_fmt(const GemmArgs &a, int wfmt, int num_sms, cudaStream_t st)
 {
-    return wfmt == MOE_WFMT_Q4K         ? launch_one<MODE, MOE_WFMT_Q4K, BN>(a, num_sms, st)
-           : wfmt == MOE_WFMT_INT4_ASYM ? launch_one<MODE, MOE_WFMT_INT4_ASYM, BN>(a, num_sms, st)
-                                        : launch_one<MODE, MOE_WFMT_INT4_SYM, BN>(a, num_sms, st);
+    return wfmt == MOE_WFMT_Q4K             ? launch_one<MODE, MOE_WFMT_Q4K, BN>(a, num_sms, st)
+           : wfmt == MOE_WFMT_INT4_ASYM     ? launch_one<MODE, MOE_WFMT_INT4_ASYM, BN>(a, num_sms, st)
+           : wfmt == MOE_WFMT_INT4_SYM_F16 ? launch_one<MODE, MOE_WFMT_INT4_SYM_F16, BN>(a, num_sms, st)
+                                            : launch_one<MODE, MOE_WFMT_INT4_SYM, BN>(a, num_sms, st);
 }
 
 cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int tile_tokens, int num_sms, cudaStream_t st)

@@ -105,17 +105,23 @@ int noalloc_max_experts();
 cudaError_t launch_permute_noalloc(const int32_t *ids, int T, int E, int k, int32_t *counts, int32_t *offsets,
                                    int32_t *sorted_slot, int32_t *dest_pos, cudaStream_t st);
 
-// out[p] = x[sorted_slot[p] / k] for p < rows (x, out: bf16 rows of H elements)
+// out[p] = x[sorted_slot[p] / k] for p < rows, then out[rows + t] = x[t] for
+// t < shared_rows (x, out: rows of H 16-bit elements).  to_f16: bf16 x is
+// written as fp16, and a value beyond fp16's range records
+// MOE_ERR_UNSUPPORTED (detail 40) in status.
 cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *sorted_slot, int rows, int k, int H, uint16_t *out,
-                               int num_sms, cudaStream_t st);
+                               int num_sms, cudaStream_t st, int shared_rows = 0, bool to_f16 = false,
+                               int *status = nullptr);
 
 cudaError_t launch_combine(const uint16_t *y_perm, const int32_t *dest_pos, const float *w, const uint16_t *shared_out,
                            const float *gate_logit, int T, int H, int k, uint16_t *y, cudaStream_t st);
 
 cudaError_t launch_pack_codes(const moe_config_t &cfg, int which, const uint8_t *canon, uint8_t *out,
                               cudaStream_t st);
+// fp16-operand mode: synchronises st and adds to *misfits the scales for
+// which q * s would not be exact in fp16
 cudaError_t launch_pack_meta(const moe_config_t &cfg, int which, const uint8_t *canon, const uint16_t *scale,
-                             uint8_t *out, cudaStream_t st);
+                             uint8_t *out, cudaStream_t st, unsigned *misfits = nullptr);
 cudaError_t launch_dequant_export(const moe_config_t &cfg, int which, int expert, const uint8_t *q,
                                   const uint8_t *meta, float *out_f32, uint16_t *out_bf16, cudaStream_t st);
 

@@ -11,6 +11,7 @@
 // codes); the load-time "symmetry scan" of the benchmarks page ("Other
 // measured changes") corresponds to the format check done by the caller.
 #include <cstdint>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "dequant.cuh"
@@ -62,7 +63,8 @@ __global__ void pack_codes_kernel(const uint8_t *__restrict__ canon, uint8_t *__
         src += (size_t)(k0 / 256) * 144 + 16 + (k0 % 256) / 2;
     else
         src += k0 / 2;
-    const uint32_t flip = wfmt == MOE_WFMT_INT4_SYM ? 8u : 0u;   // int4-sym codes become offset-binary
+    // int4-sym codes (either operand mode) become offset-binary
+    const uint32_t flip = wfmt == MOE_WFMT_INT4_SYM || wfmt == MOE_WFMT_INT4_SYM_F16 ? 8u : 0u;
     uint32_t words[4];
 #pragma unroll
     for (int wi = 0; wi < 4; ++wi) {
@@ -78,8 +80,22 @@ __global__ void pack_codes_kernel(const uint8_t *__restrict__ canon, uint8_t *__
     *(uint4 *)(out + idx * kChunkBytes) = make_uint4(words[0], words[1], words[2], words[3]);
 }
 
-// int4-sym: one thread per bf16 scale; int4-asym: per (scale, minimum) pair;
-// Q4K: one thread per 16-byte header
+// Scales of the fp16-operand mode that q * s would not be exact for, counted
+// by pack_meta_kernel; read back by launch_pack_meta.
+static __device__ unsigned int g_f16_scale_misfits;
+
+// A bf16 scale as fp16 bits; *fits = false where q * s (q in [-8, 7]) would
+// not be exact in fp16: s outside [2^-17, 8188] (zero allowed) or not finite.
+__device__ __forceinline__ uint16_t scale_to_f16(uint16_t b, bool *fits)
+{
+    const float s = __uint_as_float((uint32_t)b << 16);
+    const float a = fabsf(s);
+    *fits = s == 0.f || (a >= 0x1p-17f && a <= 8188.f);
+    return __half_as_ushort(__float2half_rn(s));
+}
+
+// int4-sym: one thread per bf16 scale (stored as fp16 in the fp16-operand
+// mode); int4-asym: per (scale, minimum) pair; Q4K: per 16-byte header
 __global__ void pack_meta_kernel(const uint8_t *__restrict__ canon, const uint16_t *__restrict__ scale,
                                  uint8_t *__restrict__ out, size_t n, int wfmt, int G, MatGeom g)
 {
@@ -104,6 +120,11 @@ __global__ void pack_meta_kernel(const uint8_t *__restrict__ canon, const uint16
     } else if (wfmt == MOE_WFMT_INT4_ASYM) {
         const size_t i = ((e * g.rows_total + row) * (size_t)(g.K / G) + grp) * 2;
         ((uint32_t *)out)[idx] = (uint32_t)scale[i] | ((uint32_t)scale[i + 1] << 16);
+    } else if (wfmt == MOE_WFMT_INT4_SYM_F16) {
+        bool fits;
+        ((uint16_t *)out)[idx] = scale_to_f16(scale[(e * g.rows_total + row) * (size_t)(g.K / G) + grp], &fits);
+        if (!fits)
+            atomicAdd(&g_f16_scale_misfits, 1u);
     } else {
         ((uint16_t *)out)[idx] = scale[(e * g.rows_total + row) * (size_t)(g.K / G) + grp];
     }
@@ -120,13 +141,33 @@ cudaError_t launch_pack_codes(const moe_config_t &cfg, int which, const uint8_t 
 }
 
 cudaError_t launch_pack_meta(const moe_config_t &cfg, int which, const uint8_t *canon, const uint16_t *scale,
-                             uint8_t *out, cudaStream_t st)
+                             uint8_t *out, cudaStream_t st, unsigned *misfits)
 {
     const MatGeom g = geom(cfg, which);
     const size_t E_total = (size_t)cfg.E + (cfg.has_shared ? 1 : 0);
     const size_t n = E_total * g.F * g.nmat * g.ngroups * kTileRows;
+    void *counter = nullptr;
+    cudaError_t e = cudaSuccess;
+    if (cfg.wfmt == MOE_WFMT_INT4_SYM_F16) {
+        // the count lives in this library's device memory: its address is
+        // looked up on the current device (set-up path, not stream work)
+        e = cudaGetSymbolAddress(&counter, g_f16_scale_misfits);
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(counter, 0, sizeof(unsigned), st);
+        if (e != cudaSuccess)
+            return e;
+    }
     pack_meta_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(canon, scale, out, n, cfg.wfmt, cfg.G, g);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e == cudaSuccess && counter) {
+        unsigned host = 0;
+        e = cudaMemcpyAsync(&host, counter, sizeof(unsigned), cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess)
+            e = cudaStreamSynchronize(st);
+        if (misfits)
+            *misfits += host;
+    }
+    return e;
 }
 
 // one thread per (row, 32-element chunk) of one expert matrix
@@ -162,6 +203,12 @@ __global__ void dequant_export_kernel(const uint8_t *__restrict__ q, const uint8
         dequant_int4asym_chunk(codes, sm, words);
         for (int i = 0; i < 32; ++i)
             vals[i] = int4asym_value(codes, sm, i);
+    } else if (wfmt == MOE_WFMT_INT4_SYM_F16) {
+        const int grp = kpos / G;
+        const uint16_t sbits = *(const uint16_t *)(mb + ((m * g.ngroups + grp) * kTileRows + r) * 2);
+        dequant_int4sym_f16_chunk(codes, sbits, words);
+        for (int i = 0; i < 32; ++i)
+            vals[i] = int4sym_f16_value(codes, sbits, i);
     } else {
         const int grp = kpos / G;
         const uint16_t sbits = *(const uint16_t *)(mb + ((m * g.ngroups + grp) * kTileRows + r) * 2);

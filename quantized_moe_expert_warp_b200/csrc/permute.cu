@@ -11,6 +11,7 @@
 // No floating point and no atomics on the outputs: the result is unique.
 #include <cstdint>
 #include <mutex>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "kernels.h"
@@ -246,37 +247,62 @@ cudaError_t launch_permute(const int32_t *ids, int T, int E, int k, int32_t *cou
 
 // ------------------------------------------------------------------------
 // Token rows in permuted order: out[p] = x[sorted_slot[p] / k] for the
-// rows p < rows, so that the gate/up GEMM can read each expert's rows as one
-// contiguous block with TMA tiles.  One warp copies one row with 16-byte
-// vectors (H a multiple of 128).
+// rows p < rows, then the shared expert's rows out[rows + t] = x[t] for
+// t < shared_rows, so that the gate/up GEMM can read each expert's rows as
+// one contiguous block with TMA tiles.  One warp copies one row with
+// 16-byte vectors (H a multiple of 128).  In the fp16-operand mode each
+// bf16 value is written as fp16 (exact for 2^-17 <= |x| <= 65504, rounded
+// below); a value beyond fp16's range records MOE_ERR_UNSUPPORTED.
 // ------------------------------------------------------------------------
 
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v, bool &bad)
+{
+    const float lo = __uint_as_float(v << 16), hi = __uint_as_float(v & 0xFFFF0000u);
+    bad |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t *__restrict__ x,
-                                                          const int32_t *__restrict__ sorted_slot, int rows, int k,
-                                                          int H, uint16_t *__restrict__ out)
+                                                          const int32_t *__restrict__ sorted_slot, int rows,
+                                                          int shared_rows, int k, int H, int to_f16,
+                                                          uint16_t *__restrict__ out, int *status)
 {
     pdl_wait();
     pdl_allow_successor();
     const int lane = threadIdx.x & 31;
     const int n16 = H / 8;
     const int warps = gridDim.x * (blockDim.x / 32);
-    for (int p = (blockIdx.x * blockDim.x + threadIdx.x) / 32; p < rows; p += warps) {
-        const int t = sorted_slot[p] / k;
+    bool bad = false;
+    for (int p = (blockIdx.x * blockDim.x + threadIdx.x) / 32; p < rows + shared_rows; p += warps) {
+        const int t = p < rows ? sorted_slot[p] / k : p - rows;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
         uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)p * H);
-        for (int i = lane; i < n16; i += 32)
-            dst[i] = src[i];
+        for (int i = lane; i < n16; i += 32) {
+            uint4 v = src[i];
+            if (to_f16) {
+                v.x = bf16x2_to_f16x2(v.x, bad);
+                v.y = bf16x2_to_f16x2(v.y, bad);
+                v.z = bf16x2_to_f16x2(v.z, bad);
+                v.w = bf16x2_to_f16x2(v.w, bad);
+            }
+            dst[i] = v;
+        }
     }
+    if (bad)
+        record_error(status, MOE_ERR_UNSUPPORTED, 40);
 }
 
 cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *sorted_slot, int rows, int k, int H, uint16_t *out,
-                               int num_sms, cudaStream_t st)
+                               int num_sms, cudaStream_t st, int shared_rows, bool to_f16, int *status)
 {
-    if (rows <= 0)
+    const int total = rows + shared_rows;
+    if (total <= 0)
         return cudaSuccess;
-    const int need = (rows + 7) / 8;   // eight warps per block
+    const int need = (total + 7) / 8;   // eight warps per block
     const int blocks = need < 4 * num_sms ? need : 4 * num_sms;
-    return launch_pdl(gather_rows_kernel, blocks, 256, 0, st, x, sorted_slot, rows, k, H, out);
+    return launch_pdl(gather_rows_kernel, blocks, 256, 0, st, x, sorted_slot, rows, shared_rows, k, H,
+                      to_f16 ? 1 : 0, out, status);
 }
 
 // ------------------------------------------------------------------------

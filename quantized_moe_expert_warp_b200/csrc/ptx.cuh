@@ -435,6 +435,14 @@ __device__ __forceinline__ uint32_t idesc_bf16_f32(uint32_t m, uint32_t n)
            | ((m >> 4) << 24);       // M >> 4
 }
 
+// The same for fp16 A and B operands (format code 0)
+__device__ __forceinline__ uint32_t idesc_f16_f32(uint32_t m, uint32_t n)
+{
+    return (1u << 4)                 // D format: fp32
+           | ((n >> 3) << 17)        // N >> 3
+           | ((m >> 4) << 24);       // M >> 4
+}
+
 // Shared-memory matrix descriptor: K-major operand in the 128-byte
 // swizzled layout (rows of 64 bf16 = 128 B, 8-row atoms of 1024 B).
 __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr)

@@ -51,6 +51,8 @@ GENERATOR_VERSION = 3
 WFMT_INT4_SYM = 0
 WFMT_Q4K = 1
 WFMT_INT4_ASYM = 2
+# the int4-sym weights computed with fp16 operands: same canonical arrays
+WFMT_INT4_SYM_F16 = 3
 
 
 @dataclass(frozen=True)
@@ -62,7 +64,7 @@ class LayerConfig:
     k: int            # experts per token
     I: int            # expert intermediate size
     has_shared: bool  # one always-on shared expert of intermediate I
-    wfmt: int         # WFMT_INT4_SYM, WFMT_Q4K or WFMT_INT4_ASYM
+    wfmt: int         # WFMT_INT4_SYM, WFMT_Q4K, WFMT_INT4_ASYM or WFMT_INT4_SYM_F16
     G: int            # int4-sym group size along K (256 for Q4K: super-block)
     wr_std: float     # router weight std
     zipf_s: float     # 0: no router bias; else Zipf exponent of the bias
@@ -104,6 +106,9 @@ CONFIGS = {
     "a3b_t4096_q4k": _a3b("a3b_t4096_q4k", 4096, seed=3, wfmt=WFMT_Q4K, G=256),
     # asymmetric int4 (scale and minimum per group of 128), 512 tokens
     "a3b_t512_asym": _a3b("a3b_t512_asym", 512, seed=5, wfmt=WFMT_INT4_ASYM),
+    # the 512-token and 8192-token layers with fp16 tensor-core operands (exact weights)
+    "a3b_t512_f16": _a3b("a3b_t512_f16", 512, seed=1, wfmt=WFMT_INT4_SYM_F16),
+    "a3b_t8192_zipf_f16": _a3b("a3b_t8192_zipf_f16", 8192, seed=2, zipf_s=1.1, wfmt=WFMT_INT4_SYM_F16),
     # decode-shaped batches
     "a3b_decode_t1": _a3b("a3b_decode_t1", 1, seed=4, x_stream=1),
     "a3b_decode_t8": _a3b("a3b_decode_t8", 8, seed=4, x_stream=8),
@@ -318,7 +323,7 @@ def make_expert(cfg: LayerConfig, e: int):
     H, I = cfg.H, cfg.I
     wgu = _normal(cfg.seed, _T_GU, e, (2 * I, H), 0.02)
     wdn = _normal(cfg.seed, _T_DN, e, (H, I), 0.02)
-    if cfg.wfmt == WFMT_INT4_SYM:
+    if cfg.wfmt in (WFMT_INT4_SYM, WFMT_INT4_SYM_F16):
         return quantize_int4_sym(wgu, cfg.G) + quantize_int4_sym(wdn, cfg.G)
     if cfg.wfmt == WFMT_INT4_ASYM:
         return quantize_int4_asym(wgu, cfg.G) + quantize_int4_asym(wdn, cfg.G)
@@ -360,7 +365,7 @@ def make_layer(cfg: LayerConfig, experts: Optional[list] = None) -> dict:
     # deterministic; numpy releases the GIL in the bulk fills and ufuncs
     with ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as ex:
         drawn = list(ex.map(lambda e: make_expert(cfg, e), sel))
-    if cfg.wfmt == WFMT_INT4_SYM:
+    if cfg.wfmt in (WFMT_INT4_SYM, WFMT_INT4_SYM_F16):
         gu_nib = np.zeros((Et, 2 * I, H // 2), np.uint8)
         gu_sc = np.zeros((Et, 2 * I, H // cfg.G), np.uint16)
         dn_nib = np.zeros((Et, H, I // 2), np.uint8)
