@@ -286,6 +286,18 @@ int moe_expert_down_q4(const moe_layer_t *L, const uint16_t *h, int T, const int
 int moe_combine(const uint16_t *y_perm, const int32_t *dest_pos, const float *topk_w, const uint16_t *shared_out,
                 const float *shared_gate_logit, int T, int H, int k, uint16_t *y, void *stream);
 
+/*
+ * Rows in a given order: out[p] = x[index[p] / k] for p < rows (x, out:
+ * rows of H 16-bit values, H % 8 == 0; index values must lie in
+ * [0, k * rows_of_x)).  With index = sorted_slot and k the top-k this is
+ * the permuted copy of the tokens that the gate/up pass reads; with k = 1
+ * it is a plain row gather (the expert-parallel layer uses it to order the
+ * rows it receives by expert, and to put its results back in order).
+ * Source: hipfire 0.4.3 benchmarks, "Read this before comparing columns"
+ * table, row "MoE prefill route" (per-expert buffers of token rows).
+ */
+int moe_gather_rows(const uint16_t *x, const int32_t *index, int rows, int k, int H, uint16_t *out, void *stream);
+
 /* --------------------------------------------------------- fused layer */
 
 /* Workspace bytes of moe_layer_forward for up to T_max tokens. */

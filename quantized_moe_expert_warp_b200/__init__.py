@@ -15,7 +15,7 @@ import os
 __all__ = [
     "MoeError", "Config", "lib", "moe_version", "moe_last_error", "moe_packed_sizes", "moe_pack_weights",
     "moe_dequant_export", "moe_router_workspace_size", "moe_router_logits", "moe_route", "moe_permute_workspace_size", "moe_permute",
-    "moe_expert_ffn_workspace_size", "moe_expert_ffn_q4", "moe_combine", "moe_layer_workspace_size",
+    "moe_expert_ffn_workspace_size", "moe_expert_ffn_q4", "moe_combine", "moe_gather_rows", "moe_layer_workspace_size",
     "moe_layer_forward", "moe_layer_forward_chunked", "moe_layer_decode_workspace_size", "moe_layer_decode", "moe_read_status", "moe_kernel_launches", "moe_expert_gate_up_q4", "moe_expert_down_q4",
     "moe_permute_noalloc", "PackedLayer", "WFMT_INT4_SYM", "WFMT_Q4K", "WFMT_INT4_ASYM", "WFMT_INT4_SYM_F16",
     "LIB_PATH",
@@ -96,6 +96,7 @@ def lib():
             "moe_expert_ffn_workspace_size": (sz, [vp, i32]),
             "moe_expert_ffn_q4": (i32, [vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]),
             "moe_combine": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, vp, vp]),
+            "moe_gather_rows": (i32, [vp, vp, i32, i32, i32, vp, vp]),
             "moe_layer_workspace_size": (sz, [vp, i32]),
             "moe_layer_forward": (i32, [vp, vp, i32, vp, vp, sz, vp, vp]),
             "moe_layer_forward_chunked": (i32, [vp, vp, i32, vp, i32, vp, sz, vp]),
@@ -228,6 +229,10 @@ def moe_expert_ffn_q4(layer: "PackedLayer", x, T, sorted_slot, offsets, y_perm, 
 def moe_combine(y_perm, dest_pos, topk_w, shared_out, shared_gate_logit, T, H, k, y, stream=None):
     _call("moe_combine", _ptr(y_perm), _ptr(dest_pos), _ptr(topk_w), _ptr(shared_out),
           _ptr(shared_gate_logit), T, H, k, _ptr(y), _stream(stream))
+
+
+def moe_gather_rows(x, index, rows, k, H, out, stream=None):
+    _call("moe_gather_rows", _ptr(x), _ptr(index), rows, k, H, _ptr(out), _stream(stream))
 
 
 def moe_layer_workspace_size(cfg, T_max) -> int:

@@ -648,6 +648,21 @@ int moe_combine(const uint16_t *y_perm, const int32_t *dest_pos, const float *to
     return ok();
 }
 
+int moe_gather_rows(const uint16_t *x, const int32_t *index, int rows, int k, int H, uint16_t *out, void *stream)
+{
+    REQUIRE(rows >= 0, "rows must be >= 0");
+    REQUIRE(k >= 1, "k must be >= 1");
+    REQUIRE(H > 0 && H % 8 == 0, "H must be a positive multiple of 8");
+    if (rows == 0)
+        return ok();
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(index);
+    REQUIRE_PTR(out);
+    CUDA_TRY(launch_gather_rows(x, index, rows, k, H, out, num_sms(), (cudaStream_t)stream), "gather rows");
+    g_launches += 1;
+    return ok();
+}
+
 size_t moe_layer_workspace_size(const moe_config_t *cfg, int T_max)
 {
     if (check_config(cfg) || T_max < 0)
