@@ -176,6 +176,7 @@ FfnWs ffn_layout(const moe_config_t *c, int T, uint8_t *base, bool with_xperm = 
 struct LayerWs {
     int *status;
     float *logits, *gate_logit, *w, *router_part;
+    uint16_t *router_split;
     int32_t *ids, *counts, *offsets, *sorted_slot, *dest_pos;
     void *perm_scratch;
     uint8_t *ffn;
@@ -196,6 +197,7 @@ LayerWs layer_layout(const moe_config_t *c, int T, uint8_t *base)
     w.status = (int *)take(256);
     w.logits = (float *)take(sizeof(float) * (size_t)T * c->E);
     w.router_part = (float *)take(router_part_bytes(c, T));
+    w.router_split = (uint16_t *)take(router_split_bytes(c->E, c->H));
     w.gate_logit = (float *)take(sizeof(float) * (size_t)T);
     w.ids = (int32_t *)take(sizeof(int32_t) * Tk);
     w.w = (float *)take(sizeof(float) * Tk);
@@ -432,7 +434,7 @@ size_t moe_router_workspace_size(const moe_config_t *cfg, int T)
 {
     if (!cfg || T < 0 || check_config(cfg))
         return 0;
-    return align256(router_part_bytes(cfg, T)) + 256;
+    return align256(router_part_bytes(cfg, T)) + align256(router_split_bytes(cfg->E, cfg->H)) + 256;
 }
 
 int moe_router_logits(const moe_layer_t *L, const uint16_t *x, int T, float *logits, float *gate_logit, void *ws,
@@ -456,10 +458,11 @@ int moe_router_logits(const moe_layer_t *L, const uint16_t *x, int T, float *log
     cudaStream_t st = (cudaStream_t)stream;
     const int S = router_slices(&L->cfg, T);
     float *part = S > 1 ? (float *)ws : logits;
+    uint16_t *wsplit = (uint16_t *)((uint8_t *)ws + align256(router_part_bytes(&L->cfg, T)));
     CUDA_TRY(launch_router_gemm(x, T, L->cfg.H, L->router_w, L->router_bias, L->cfg.E, g, part,
-                                g ? gate_logit : nullptr, S, nullptr, num_sms(), st),
+                                g ? gate_logit : nullptr, S, wsplit, nullptr, num_sms(), st),
              "router logits");
-    g_launches += 1;
+    g_launches += 2;
     if (S > 1) {
         CUDA_TRY(launch_router_reduce(part, S, T, L->cfg.E, L->router_bias, logits, st), "router reduce");
         g_launches += 1;
@@ -698,9 +701,9 @@ int moe_layer_forward(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *
     const float *g = c.has_shared ? L->shared_gate : nullptr;
     const int S = router_slices(&c, T);
     CUDA_TRY(launch_router_gemm(x, T, c.H, L->router_w, L->router_bias, c.E, g, S > 1 ? w.router_part : w.logits,
-                                g ? w.gate_logit : nullptr, S, w.status, num_sms(), st),
+                                g ? w.gate_logit : nullptr, S, w.router_split, w.status, num_sms(), st),
              "router logits");
-    g_launches += 1;
+    g_launches += 2;
     const int32_t *ids = w.ids;
     const float *tw = w.w;
     if (override_route) {

@@ -11,22 +11,15 @@
 // dequant warps write them straight into tensor memory (TMEM), where the
 // MMA reads its A operand, and the tokens are gathered into swizzled
 // shared memory as the B operand.  The accumulator stays in TMEM until the
-// epilogue warps apply SwiGLU (gate/up pass), round to bf16 (down pass) or
-// add the router bias (router pass).
-//
-// The router pass uses the same engine: its fp32 weights are split into two
-// bf16 parts (hi + lo carry 16 significand bits, the rest is below the fp32
-// accumulation error of the tensor cores over K = 2048), both products are
-// exact in fp32 and accumulate into one fp32 accumulator.
+// epilogue warps apply SwiGLU (gate/up pass) or round to bf16 (down pass).
 //
 // Warp roles of one persistent CTA (one per SM, 768 threads):
 //   warp 0      loads the token rows of B with one tiled TMA copy per k-step:
 //               rows of x in permuted order (gate/up, routed experts), of x
-//               (shared expert, router) or of h (down)
+//               (shared expert) or of h (down)
 //   warp 1      issues tcgen05.mma (one thread) and commits stage releases
 //   warp 2      streams code blocks and per-tile scale blocks with bulk copies
-//   warp 3      owns the TMEM allocation; in the router pass it also forms
-//               the shared expert's gate logits x . g
+//   warp 3      owns the TMEM allocation
 //   warps 4-19  dequantise, in two groups of eight taking alternate k-steps:
 //               row r = 32*(warp%4) + lane, half c of the k-step = ((warp-4)%8)/4
 //   warps 20-23 epilogue (TMEM -> registers -> global)
@@ -121,7 +114,7 @@ constexpr int kEpiBytes = 4 * kEpiTok * kEpiStride;              // staging for 
 constexpr int kDeqWarps = MOEQ4_DEQ_WARPS;     // dequant warps (warps 4 .. 3 + kDeqWarps), a multiple of 8
 constexpr int kThreads = (8 + kDeqWarps) * 32;
 
-enum { MODE_GATE_UP = 0, MODE_DOWN = 1, MODE_ROUTER = 2 };
+enum { MODE_GATE_UP = 0, MODE_DOWN = 1 };
 
 template <int MODE, int BN>
 struct Geo {
@@ -133,22 +126,22 @@ struct Geo {
     // accumulator buffers (up to 2) as fit; with two, the epilogue of one
     // tile overlaps the MMAs of the next.  The requested A-stage count is cut
     // to leave room for one accumulator buffer.
-    static constexpr int kAStagesReq = MODE == MODE_GATE_UP ? MOEQ4_A_STAGES_GU : MODE == MODE_DOWN ? MOEQ4_A_STAGES_DN : 4;
+    static constexpr int kAStagesReq = MODE == MODE_GATE_UP ? MOEQ4_A_STAGES_GU : MOEQ4_A_STAGES_DN;
     static constexpr int kAStagesFit = (512 - kNAcc_ * BN) / (kNA * 32);
     static constexpr int kAStages = kAStagesReq < kAStagesFit ? kAStagesReq : kAStagesFit;
     static_assert(kAStages >= 2 && kAStages <= kMaxAStages, "TMEM A stages");
     static constexpr int kAccBufs = (512 - kAStages * kNA * 32) / (kNAcc_ * BN) >= 2 ? 2 : 1;
-    static constexpr int kNCode = MODE == MODE_GATE_UP ? 2 : MODE == MODE_DOWN ? 1 : 0; // code matrices
+    static constexpr int kNCode = MODE == MODE_GATE_UP ? 2 : 1;   // code matrices
     // dequant warp groups: groups of four warps, each warp a full k-step of
-    // its 32 rows, or groups of eight, each warp one half of a k-step (the
-    // router, and any warp count that would give more groups than TMEM A
-    // stages: a group must not reuse a stage whose previous MMAs it has not
-    // waited for, so that no mbarrier waiter runs two phases ahead)
-    static constexpr int kGroupWarps = MODE == MODE_ROUTER || kDeqWarps / 4 > kAStages ? 8 : 4;
+    // its 32 rows, or groups of eight, each warp one half of a k-step (any
+    // warp count that would give more groups than TMEM A stages: a group must
+    // not reuse a stage whose previous MMAs it has not waited for, so that no
+    // mbarrier waiter runs two phases ahead)
+    static constexpr int kGroupWarps = kDeqWarps / 4 > kAStages ? 8 : 4;
     static constexpr int kGroups = kDeqWarps / kGroupWarps;
     static_assert(kGroups <= kAStages, "dequant groups must not outnumber the TMEM A stages");
     static constexpr int kHalves = kGroupWarps == 8 ? 1 : 2;
-    static constexpr int kCodeBlock = kNCode ? code_block_bytes(kNCode) : 0;
+    static constexpr int kCodeBlock = code_block_bytes(kNCode);
     // the gathered token rows wait on L2 / HBM latency, so their shared-memory
     // ring is deeper than the TMEM ring
     static constexpr int kBStages = BN == 64 ? MOEQ4_B_STAGES_64 : BN == 128 ? MOEQ4_B_STAGES_128 : 4;
@@ -181,7 +174,6 @@ struct Barriers {
 
 struct Unit {
     int e, f, row0, nvalid, nmma;
-    int split, ks0, nks;   // K slice of the unit (router split-K; otherwise the whole K)
 };
 
 struct Sched {
@@ -194,14 +186,6 @@ template <int BN>
 __device__ __forceinline__ Unit decode_unit(int u, const GemmArgs &p, const Sched &sc)
 {
     Unit r;
-    const int ks_all = p.K / kKStep;
-    r.split = 0;
-    if (p.ksplit > 1) {
-        r.split = u % p.ksplit;
-        u /= p.ksplit;
-    }
-    r.nks = ks_all / p.ksplit;
-    r.ks0 = r.split * r.nks;
     const int tile = u / p.F;
     r.f = u - tile * p.F;
     int lo = 0, hi = p.E_total - 1;   // largest e with tile_start[e] <= tile (a non-empty expert)
@@ -223,7 +207,6 @@ __device__ __forceinline__ Unit decode_unit(int u, const GemmArgs &p, const Sche
 // Every CTA derives the tile schedule from the permutation offsets: rows of
 // expert e are [offsets[e], offsets[e+1]); the shared expert (if any) is
 // expert E with rows [T k, T k + T); expert e owns ceil(rows / BN) tiles.
-// Without offsets (router pass) the T token rows form a single group.
 template <int BN>
 __device__ void build_schedule(const GemmArgs &p, int *s_tile_start, int *s_row_start, int *s_row_count,
                                int *s_part)
@@ -234,10 +217,7 @@ __device__ void build_schedule(const GemmArgs &p, int *s_tile_start, int *s_row_
     int local = 0;
     for (int e = e0; e < min(n, e0 + per); ++e) {
         int start, cnt;
-        if (!p.offsets) {
-            start = 0;
-            cnt = p.T;
-        } else if (e < p.E) {
+        if (e < p.E) {
             start = p.offsets[e];
             cnt = p.offsets[e + 1] - p.offsets[e];
         } else {
@@ -279,30 +259,6 @@ __device__ void build_schedule(const GemmArgs &p, int *s_tile_start, int *s_row_
     }
     if (threadIdx.x == kThreads - 1)
         s_tile_start[n] = s_part[32 + kThreads / 32 - 1];
-}
-
-// fp32 -> two bf16 parts (hi, lo): w - hi is exact in fp32, so hi + lo
-// matches w to about 2^-17 relative.
-__device__ __forceinline__ void split2(float w0, float w1, uint32_t &hi, uint32_t &lo)
-{
-    hi = pack_bf16x2(w0, w1);
-    const float r0 = w0 - __uint_as_float(hi << 16);
-    const float r1 = w1 - __uint_as_float(hi & 0xFFFF0000u);
-    lo = pack_bf16x2(r0, r1);
-}
-
-// A producer that stops early (a wait ran out, or another role gave up)
-// still waits, with a fresh bounded budget, until the copies it issued have
-// landed, so that none writes into this CTA's shared memory after it exits:
-// the last `depth` of the n_issued ring slots it filled.  On the normal path
-// every such phase has completed already.
-__device__ __forceinline__ void drain_ring(uint64_t *full, int n_issued, int depth, int *status, int where,
-                                           int *never_abort)
-{
-    WaitCtx wd{never_abort, status, globaltimer_ns(), kWaitLimitNs};
-    for (int i = max(0, n_issued - depth); i < n_issued; ++i)
-        if (!warp_wait(&full[i % depth], (i / depth) & 1, wd, where))
-            break;
 }
 
 template <int MODE, int WFMT, int BN>
@@ -376,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    const int total_units = s_tile_start[p.E_total] * p.F * p.ksplit;
+    const int total_units = s_tile_start[p.E_total] * p.F;
     const int KS = p.K / kKStep;
     WaitCtx wc{&bars->abort_flag, p.status, globaltimer_ns(), wait_limit_ns(p.status)};
     CYC_DECL
@@ -401,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const CUtensorMap *map = second ? &tmap_b2 : &tmap_b;
             const int y = second ? un.row0 - p.Tk : un.row0;
             CYC(2);
-            for (int ks = un.ks0; ks < un.ks0 + un.nks; ++ks, ++step) {
+            for (int ks = 0; ks < KS; ++ks, ++step) {
                 const int s = step % L::kBStages;
                 if (step >= L::kBStages && !warp_wait(&bars->b_empty[s], ((step / L::kBStages) & 1) ^ 1, wc, 1)) {
                     ok = false;
@@ -425,9 +381,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++uidx) {
             const Unit un = decode_unit<BN>(u, p, sched);
-            // fp16-operand mode: fp16 weights and tokens (the router stays bf16)
-            const uint32_t idesc = WFMT == MOE_WFMT_INT4_SYM_F16 && MODE != MODE_ROUTER ? idesc_f16_f32(128, un.nmma)
-                                                                                        : idesc_bf16_f32(128, un.nmma);
+            // fp16-operand mode: fp16 weights and tokens
+            const uint32_t idesc = WFMT == MOE_WFMT_INT4_SYM_F16 ? idesc_f16_f32(128, un.nmma)
+                                                                 : idesc_bf16_f32(128, un.nmma);
             const int ab = uidx % L::kAccBufs;
             const uint32_t acc = tmem + ab * L::kNAcc * kBN;
             CYC(4);
@@ -437,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
             }
             CYC(0);
-            for (int ks = 0; ks < un.nks; ++ks, ++step) {
+            for (int ks = 0; ks < KS; ++ks, ++step) {
                 const int sa = step % L::kAStages, sb = step % L::kBStages;
                 // every lane polls the same barriers, so the outcome is warp-uniform
                 if (!mbar_wait(&bars->a_full[sa], (step / L::kAStages) & 1, wc, 3)) {
@@ -461,11 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint64_t bdesc = bdesc0 + (uint64_t)(kk * 2);   // +32 bytes along K
 #pragma unroll
                         for (int m = 0; m < L::kNA; ++m) {
-                            const uint32_t a_t = a_base + m * 32 + kk * 8;
-                            if (MODE == MODE_ROUTER)   // both parts into one accumulator
-                                mma_ts_f16(acc, a_t, bdesc, idesc, (ks | kk | m) != 0);
-                            else
-                                mma_ts_f16(acc + m * kBN, a_t, bdesc, idesc, (ks | kk) != 0);
+                            mma_ts_f16(acc + m * kBN, a_base + m * 32 + kk * 8, bdesc, idesc, (ks | kk) != 0);
                         }
                     }
                     mma_commit(&bars->a_empty[sa]);
@@ -494,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // copy moves CK k-steps: the copy engine's throughput is set by the
         // number of copies more than by their size.  (Under the status block's
         // test knob this CTA issues none, and its dequant waits run out.)
-        if (MODE != MODE_ROUTER && !test_knob_hits_this_cta(p.status)) {
+        if (!test_knob_hits_this_cta(p.status)) {
             int cidx = 0, munit = 0, nmeta = 0;   // cidx: code chunks issued; nmeta: meta blocks issued
             bool ok = true;
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++munit) {
@@ -535,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // instrumented builds, first CTAs: record when each code chunk lands
         // (event 14, by chunk), each B stage lands (event 8, by step) and each
         // A stage is complete in TMEM (event 10, by step)
-        if (MODE != MODE_ROUTER && blockIdx.x < 4 && lane == 0) {
+        if (blockIdx.x < 4 && lane == 0) {
             int n_units = 0;
             for (int u = blockIdx.x; u < total_units; u += gridDim.x)
                 ++n_units;
@@ -569,31 +521,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
 #endif
-        // ------------------------------------------------ shared-expert gate logits
-        if (MODE == MODE_ROUTER && p.gate_w) {
-            for (int t = blockIdx.x; t < p.T; t += gridDim.x) {
-                const uint16_t *xr = p.b_src + (size_t)t * p.ldb;
-                float acc = 0.f;
-                for (int c0 = lane * 8; c0 < p.K; c0 += 256) {
-                    const uint4 v = *(const uint4 *)(xr + c0);
-                    const float4 g0 = *(const float4 *)(p.gate_w + c0);
-                    const float4 g1 = *(const float4 *)(p.gate_w + c0 + 4);
-                    acc = fmaf(__uint_as_float(v.x << 16), g0.x, acc);
-                    acc = fmaf(__uint_as_float(v.x & 0xFFFF0000u), g0.y, acc);
-                    acc = fmaf(__uint_as_float(v.y << 16), g0.z, acc);
-                    acc = fmaf(__uint_as_float(v.y & 0xFFFF0000u), g0.w, acc);
-                    acc = fmaf(__uint_as_float(v.z << 16), g1.x, acc);
-                    acc = fmaf(__uint_as_float(v.z & 0xFFFF0000u), g1.y, acc);
-                    acc = fmaf(__uint_as_float(v.w << 16), g1.z, acc);
-                    acc = fmaf(__uint_as_float(v.w & 0xFFFF0000u), g1.w, acc);
-                }
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1)
-                    acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-                if (lane == 0)
-                    p.gate_out[t] = acc;
-            }
-        }
     } else if (warp >= 4 && warp < 4 + kDeqWarps) {
         // ------------------------------------------------ dequant into TMEM
         // Groups of L::kGroupWarps warps take k-steps round-robin; a warp owns
@@ -610,156 +537,109 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++munit) {
             const int mb = munit & (NMETA - 1);
             const uint8_t *meta = sMeta + mb * meta_al;
-            float4 pre[8];                                // router: this row's next k-step, prefetched
-            const float *wrow = nullptr;
-            int kbeg = 0, kend = KS;                      // k-steps of the unit
-            if (MODE == MODE_ROUTER) {
-                const Unit un = decode_unit<BN>(u, p, sched);
-                kbeg = un.ks0;
-                kend = un.ks0 + un.nks;
-                const int e = un.f * kTileRows + r;
-                wrow = e < p.E ? p.a_f32 + (size_t)e * p.K + c0 * 32 : nullptr;
-                // first k-step of this group in the unit
-                const int kfirst = kbeg + ((grp - step) % L::kGroups + L::kGroups) % L::kGroups;
-                if (kfirst >= kend)
-                    wrow = nullptr;
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    pre[i] = wrow ? *(const float4 *)(wrow + kfirst * kKStep + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
-            } else if (!mbar_wait(&bars->meta_full[mb], (munit >> p.nmeta_log2) & 1, wc, 8)) {
+            if (!mbar_wait(&bars->meta_full[mb], (munit >> p.nmeta_log2) & 1, wc, 8))
                 break;
-            }
             CYC(7);
             const int ngroups = WFMT == MOE_WFMT_Q4K ? p.K / 256 : p.K >> gshift;
             // This warp's k-steps of the unit: those with step % kGroups == grp.
             // Every dequant warp frees every code chunk of the unit exactly
             // once: right after its last k-step in the chunk, or, for chunks
             // where it has none, as it passes them.
-            const int step0 = step;                       // global step of k-step kbeg
-            const int nchunks = MODE == MODE_ROUTER ? 0 : (KS + CK - 1) >> p.ck_log2;
+            const int step0 = step;                       // global step of k-step 0
+            const int nchunks = (KS + CK - 1) >> p.ck_log2;
             int released = 0;                             // chunks of this unit already freed
-            for (int ks = kbeg + ((grp - step0) % L::kGroups + L::kGroups) % L::kGroups; ks < kend;
-                 ks += L::kGroups) {
-                step = step0 + (ks - kbeg);
+            for (int ks = ((grp - step0) % L::kGroups + L::kGroups) % L::kGroups; ks < KS; ks += L::kGroups) {
+                step = step0 + ks;
                 const int sa = step % L::kAStages;
                 const uint32_t a_col = tmem + lane_off + L::kAccCols + sa * L::kNA * 32;
                 CYC(6);
-                if (MODE == MODE_ROUTER) {
+                const int my_chunk = ks >> p.ck_log2;
+                const int cidx = cbase + my_chunk;
+                const int sc = cidx & (NCS - 1);
+                // chunks passed without a k-step of this warp are freed before it
+                // waits for a later one (a warp never holds one chunk while
+                // waiting for another)
+                if (my_chunk > released) {
+                    __syncwarp();
+                    if (lane == 0)
+                        for (int cc = released; cc < my_chunk; ++cc)
+                            mbar_arrive(&bars->code_empty[(cbase + cc) & (NCS - 1)]);
+                    released = my_chunk;
+                }
+                if (lane == 0 && warp == 4)
+                    TRACE_OTHER(15, step);
+                if (!mbar_wait(&bars->code_full[sc], (cidx >> p.ncs_log2) & 1, wc, 9)) {
+                    ok = false;
+                    break;
+                }
+                CYC(0);
+#ifdef MOEQ4_TRACE_WARPS
+                if (lane == 0)
+                    TRACE_EVENT((warp - 4) * 2, step);
+#else
+                if (lane == 0 && warp == 4)
+                    TRACE_EVENT(2, step);
+#endif
+                const uint32_t cblk = smem_u32(sCode) + sc * chunk_bytes + (ks & (CK - 1)) * L::kCodeBlock;
+#pragma unroll 1
+                for (int h = 0; h < L::kHalves; ++h) {
+                    const int c = c0 + h;
+                    const int kpos = ks * kKStep + c * 32;
                     uint32_t words[L::kNA][16];
-                    float v[32];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        v[4 * i] = pre[i].x;
-                        v[4 * i + 1] = pre[i].y;
-                        v[4 * i + 2] = pre[i].z;
-                        v[4 * i + 3] = pre[i].w;
+                    for (int m = 0; m < L::kNA; ++m) {
+                        const uint4 codes = lds128(cblk + ((m * 2 + c) * kTileRows + r) * kChunkBytes);
+                        if (WFMT == MOE_WFMT_Q4K) {
+                            const int g = kpos / 256;
+                            const uint4 hdr = lds128(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 16);
+                            float dsc, dm;
+                            q4k_subblock_scale(hdr, (kpos % 256) / 32, dsc, dm);
+                            dequant_q4k_chunk(codes, dsc, dm, words[m]);
+                        } else if (WFMT == MOE_WFMT_INT4_ASYM) {
+                            const int g = kpos >> gshift;
+                            const uint32_t sm = lds32(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 4);
+                            dequant_int4asym_chunk(codes, sm, words[m]);
+                        } else if (WFMT == MOE_WFMT_INT4_SYM_F16) {
+                            const int g = kpos >> gshift;
+                            const uint16_t sbits = lds16(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 2);
+                            dequant_int4sym_f16_chunk(codes, sbits, words[m]);
+                        } else {
+                            const int g = kpos >> gshift;
+                            const uint16_t sbits = lds16(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 2);
+                            dequant_int4sym_chunk(codes, sbits, words[m]);
+                        }
                     }
-                    if (wrow && ks + L::kGroups < kend) {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            pre[i] = *(const float4 *)(wrow + (ks + L::kGroups) * kKStep + 4 * i);
+                    if (h == 0) {
+                        CYC(1);
+                        if (lane == 0 && warp == 4)
+                            TRACE_EVENT(11, step);
+                        // the MMAs that read this TMEM stage kAStages k-steps ago have finished
+                        if (step >= L::kAStages &&
+                            !mbar_wait(&bars->a_empty[sa], ((step / L::kAStages) & 1) ^ 1, wc, 10)) {
+                            ok = false;
+                            break;
+                        }
+                        if (lane == 0 && warp == 4)
+                            TRACE_OTHER(12, step);
+                        tc_fence_after();
+                        CYC(2);
                     }
-#pragma unroll
-                    for (int jj = 0; jj < 16; ++jj)
-                        split2(v[2 * jj], v[2 * jj + 1], words[0][jj], words[1 % L::kNA][jj]);
-                    if (step >= L::kAStages &&
-                        !mbar_wait(&bars->a_empty[sa], ((step / L::kAStages) & 1) ^ 1, wc, 10)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
 #pragma unroll
                     for (int m = 0; m < L::kNA; ++m)
-                        tmem_st16(a_col + m * 32 + c0 * 16, words[m]);
-                } else {
-                    const int my_chunk = ks >> p.ck_log2;
-                    const int cidx = cbase + my_chunk;
-                    const int sc = cidx & (NCS - 1);
-                    // chunks passed without a k-step of this warp are freed before it
-                    // waits for a later one (a warp never holds one chunk while
-                    // waiting for another)
-                    if (my_chunk > released) {
-                        __syncwarp();
-                        if (lane == 0)
-                            for (int cc = released; cc < my_chunk; ++cc)
-                                mbar_arrive(&bars->code_empty[(cbase + cc) & (NCS - 1)]);
-                        released = my_chunk;
-                    }
-                    if (lane == 0 && warp == 4)
-                        TRACE_OTHER(15, step);
-                    if (!mbar_wait(&bars->code_full[sc], (cidx >> p.ncs_log2) & 1, wc, 9)) {
-                        ok = false;
-                        break;
-                    }
-                    CYC(0);
-#ifdef MOEQ4_TRACE_WARPS
-                    if (lane == 0)
-                        TRACE_EVENT((warp - 4) * 2, step);
-#else
-                    if (lane == 0 && warp == 4)
-                        TRACE_EVENT(2, step);
-#endif
-                    const uint32_t cblk = smem_u32(sCode) + sc * chunk_bytes + (ks & (CK - 1)) * L::kCodeBlock;
-#pragma unroll 1
-                    for (int h = 0; h < L::kHalves; ++h) {
-                        const int c = c0 + h;
-                        const int kpos = ks * kKStep + c * 32;
-                        uint32_t words[L::kNA][16];
-#pragma unroll
-                        for (int m = 0; m < L::kNA; ++m) {
-                            const uint4 codes = lds128(cblk + ((m * 2 + c) * kTileRows + r) * kChunkBytes);
-                            if (WFMT == MOE_WFMT_Q4K) {
-                                const int g = kpos / 256;
-                                const uint4 hdr = lds128(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 16);
-                                float dsc, dm;
-                                q4k_subblock_scale(hdr, (kpos % 256) / 32, dsc, dm);
-                                dequant_q4k_chunk(codes, dsc, dm, words[m]);
-                            } else if (WFMT == MOE_WFMT_INT4_ASYM) {
-                                const int g = kpos >> gshift;
-                                const uint32_t sm = lds32(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 4);
-                                dequant_int4asym_chunk(codes, sm, words[m]);
-                            } else if (WFMT == MOE_WFMT_INT4_SYM_F16) {
-                                const int g = kpos >> gshift;
-                                const uint16_t sbits = lds16(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 2);
-                                dequant_int4sym_f16_chunk(codes, sbits, words[m]);
-                            } else {
-                                const int g = kpos >> gshift;
-                                const uint16_t sbits = lds16(smem_u32(meta) + ((m * ngroups + g) * kTileRows + r) * 2);
-                                dequant_int4sym_chunk(codes, sbits, words[m]);
-                            }
-                        }
-                        if (h == 0) {
-                            CYC(1);
-                            if (lane == 0 && warp == 4)
-                                TRACE_EVENT(11, step);
-                            // the MMAs that read this TMEM stage kAStages k-steps ago have finished
-                            if (step >= L::kAStages &&
-                                !mbar_wait(&bars->a_empty[sa], ((step / L::kAStages) & 1) ^ 1, wc, 10)) {
-                                ok = false;
-                                break;
-                            }
-                            if (lane == 0 && warp == 4)
-                                TRACE_OTHER(12, step);
-                            tc_fence_after();
-                            CYC(2);
-                        }
-#pragma unroll
-                        for (int m = 0; m < L::kNA; ++m)
-                            tmem_st16(a_col + m * 32 + c * 16, words[m]);
-                        CYC(h == 0 ? 3 : 4);
-                    }
-                    if (!ok)
-                        break;
-                    // after its last k-step in the chunk the warp frees it
-                    const int chunk_end = min((my_chunk + 1) << p.ck_log2, KS);
-                    if (ks + L::kGroups >= chunk_end) {
-                        __syncwarp();
-                        if (lane == 0)
-                            mbar_arrive(&bars->code_empty[sc]);
-                        released = my_chunk + 1;
-                    }
-                    CYC(11);
+                        tmem_st16(a_col + m * 32 + c * 16, words[m]);
+                    CYC(h == 0 ? 3 : 4);
                 }
+                if (!ok)
+                    break;
+                // after its last k-step in the chunk the warp frees it
+                const int chunk_end = min((my_chunk + 1) << p.ck_log2, KS);
+                if (ks + L::kGroups >= chunk_end) {
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&bars->code_empty[sc]);
+                    released = my_chunk + 1;
+                }
+                CYC(11);
                 tmem_wait_st();
                 CYC(5);
                 if (lane == 0 && warp == 4)
@@ -778,14 +658,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok)
                 break;
-            step = step0 + (kend - kbeg);
-            if (MODE != MODE_ROUTER) {
-                __syncwarp();
-                if (lane == 0) {
-                    for (int cc = released; cc < nchunks; ++cc)
-                        mbar_arrive(&bars->code_empty[(cbase + cc) & (NCS - 1)]);
-                    mbar_arrive(&bars->meta_empty[mb]);
-                }
+            step = step0 + KS;
+            __syncwarp();
+            if (lane == 0) {
+                for (int cc = released; cc < nchunks; ++cc)
+                    mbar_arrive(&bars->code_empty[(cbase + cc) & (NCS - 1)]);
+                mbar_arrive(&bars->meta_empty[mb]);
             }
             cbase += (KS + CK - 1) >> p.ck_log2;
         }
@@ -823,50 +701,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_arrive(&bars->acc_empty[ab]);
                     released = true;
                 }
-                if (MODE == MODE_ROUTER) {
-                    // split-K: one partial [T, E] per K slice, the bias is added when they are summed
-                    if (col < p.E) {
-                        const float b = p.ksplit == 1 && p.bias ? p.bias[col] : 0.f;
-                        float *out = p.out_f32 + (size_t)un.split * p.T * p.E;
+                // this lane's feature for 16 tokens -> staging [token][feature] (bf16)
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int n = n0 + j;
-                            if (n < un.nvalid)
-                                out[(size_t)(un.row0 + n) * p.E + col] = __uint_as_float(g[j]) + b;
-                        }
+                for (int j = 0; j < 16; ++j) {
+                    float o;
+                    if (MODE == MODE_GATE_UP) {
+                        const float a = __uint_as_float(g[j]);
+                        o = __fdividef(a, 1.0f + __expf(-a)) * __uint_as_float(v[j]);   // silu(a) * u
+                    } else {
+                        o = __uint_as_float(g[j]);
                     }
-                } else {
-                    // this lane's feature for 16 tokens -> staging [token][feature] (bf16)
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        float o;
-                        if (MODE == MODE_GATE_UP) {
-                            const float a = __uint_as_float(g[j]);
-                            o = __fdividef(a, 1.0f + __expf(-a)) * __uint_as_float(v[j]);   // silu(a) * u
-                        } else {
-                            o = __uint_as_float(g[j]);
-                        }
-                        // h is fp16 in the fp16-operand mode (the down pass's operand); Y is bf16
-                        if (MODE == MODE_GATE_UP && WFMT == MOE_WFMT_INT4_SYM_F16)
-                            *(__half *)(stage + j * kEpiStride + lane * 2) = __float2half_rn(o);
-                        else
-                            *(__nv_bfloat16 *)(stage + j * kEpiStride + lane * 2) = __float2bfloat16_rn(o);
-                    }
-                    __syncwarp();
-                    // lane: token n0 + (lane & 15), 32-byte half (lane >> 4) of the warp's 64-byte row slice
-                    const int t = lane & 15, hh = lane >> 4;
-                    const int n = n0 + t;
-                    if (n < un.nvalid) {
-                        const int prow = un.row0 + n;
-                        uint16_t *dst = prow < p.Tk ? p.out + (size_t)prow * p.ldo
-                                                    : p.out_shared + (size_t)(prow - p.Tk) * p.ldo;
-                        uint4 *d4 = (uint4 *)(dst + un.f * kTileRows + q * 32 + hh * 16);
-                        const uint4 *s4 = (const uint4 *)(stage + t * kEpiStride + hh * 32);
-                        d4[0] = s4[0];
-                        d4[1] = s4[1];
-                    }
-                    __syncwarp();
+                    // h is fp16 in the fp16-operand mode (the down pass's operand); Y is bf16
+                    if (MODE == MODE_GATE_UP && WFMT == MOE_WFMT_INT4_SYM_F16)
+                        *(__half *)(stage + j * kEpiStride + lane * 2) = __float2half_rn(o);
+                    else
+                        *(__nv_bfloat16 *)(stage + j * kEpiStride + lane * 2) = __float2bfloat16_rn(o);
                 }
+                __syncwarp();
+                // lane: token n0 + (lane & 15), 32-byte half (lane >> 4) of the warp's 64-byte row slice
+                const int t = lane & 15, hh = lane >> 4;
+                const int n = n0 + t;
+                if (n < un.nvalid) {
+                    const int prow = un.row0 + n;
+                    uint16_t *dst = prow < p.Tk ? p.out + (size_t)prow * p.ldo
+                                                : p.out_shared + (size_t)(prow - p.Tk) * p.ldo;
+                    uint4 *d4 = (uint4 *)(dst + un.f * kTileRows + q * 32 + hh * 16);
+                    const uint4 *s4 = (const uint4 *)(stage + t * kEpiStride + hh * 32);
+                    d4[0] = s4[0];
+                    d4[1] = s4[1];
+                }
+                __syncwarp();
             }
             if (!released) {
                 tc_fence_before();
@@ -926,8 +790,6 @@ static Rings gemm_rings(int meta_bytes, int E_total, int KS)
 {
     using L = Geo<MODE, BN>;
     Rings r{0, 0, 1};
-    if (MODE == MODE_ROUTER)
-        return r;
     r.nmeta_log2 = meta_bytes <= 4096 ? 2 : 1;
     r.ck_log2 = 1;
     while ((L::kCodeBlock << (r.ck_log2 + 1)) <= 32768 && (1 << (r.ck_log2 + 1)) <= KS)
@@ -961,7 +823,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 // Tensor map of the B rows (bf16 [b_rows, ldb], row-major) in tiles of
 // 64 elements (128 bytes, 128-byte swizzle: the MMA's K-major layout) by
 // BN rows.
-static cudaError_t encode_b_map(CUtensorMap *m, const uint16_t *src, int ld, int rows, int bn)
+cudaError_t encode_b_map(CUtensorMap *m, const uint16_t *src, int ld, int rows, int bn)
 {
     const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc)
@@ -989,8 +851,6 @@ static cudaError_t launch_one(const GemmArgs &a_in, int num_sms, cudaStream_t st
     if (e != cudaSuccess)
         return e;
     GemmArgs a = a_in;
-    if (a.ksplit < 1)
-        a.ksplit = 1;
     const Rings r = gemm_rings<MODE, BN>(a.meta_bytes, a.E_total, a.K / kKStep);
     a.ck_log2 = r.ck_log2;
     a.ncs_log2 = r.ncs_log2;
@@ -1013,22 +873,6 @@ size_t gemm_smem_required(int nmat, int meta_bytes, int E_total)
     const size_t b = nmat == 2 ? gemm_smem_bytes<MODE_GATE_UP, 128>(meta_bytes, E_total, r)
                                : gemm_smem_bytes<MODE_DOWN, 256>(meta_bytes, E_total, r);
     return a > b ? a : b;
-}
-
-// K slices of the router GEMM: enough work units (128 experts x 128 tokens x
-// K slice) to cover the SMs, at most 32 slices, each a whole number of
-// k-steps, and at most 4 MB of partial logits (they are written and read
-// back once more).
-int router_ksplit(int T, int E, int H, int sms)
-{
-    const int units = ((E + kTileRows - 1) / kTileRows) * ((T + 127) / 128);
-    const int ks = H / kKStep;
-    const size_t part_cap = (size_t)4 << 20;
-    int s = 1;
-    while (2 * s <= 32 && ks % (2 * s) == 0 && units * 2 * s <= sms &&
-           (size_t)2 * s * T * E * sizeof(float) <= part_cap)
-        s *= 2;
-    return s;
 }
 
 int gemm_tile_tokens(int T, int E, int k) { return (long long)T * k <= 64LL * E ? 64 : 128; }
@@ -1061,33 +905,6 @@ cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int tile_
     return tile_tokens == 64    ? launch_fmt<MODE_DOWN, 64>(a, wfmt, num_sms, st)
            : tile_tokens == 128 ? launch_fmt<MODE_DOWN, 128>(a, wfmt, num_sms, st)
                                 : launch_fmt<MODE_DOWN, 256>(a, wfmt, num_sms, st);
-}
-
-// Router logits on tensor cores: logits[t, e] = x[t] . Wr[e] (+ bias[e]),
-// and gate_out[t] = x[t] . g when g is given.
-cudaError_t launch_router_gemm(const uint16_t *x, int T, int H, const float *wr, const float *bias, int E,
-                               const float *gate_w, float *logits, float *gate_out, int ksplit, int *status,
-                               int num_sms, cudaStream_t st)
-{
-    if (T == 0)
-        return cudaSuccess;
-    GemmArgs a{};
-    a.b_src = x;
-    a.ldb = H;
-    a.b_rows = T;
-    a.T = T;
-    a.E = E;
-    a.E_total = 1;
-    a.K = H;
-    a.F = (E + kTileRows - 1) / kTileRows;
-    a.a_f32 = wr;
-    a.bias = bias;
-    a.gate_w = gate_w;
-    a.gate_out = gate_out;
-    a.out_f32 = logits;
-    a.ksplit = ksplit;
-    a.status = status;
-    return launch_one<MODE_ROUTER, 0, 128>(a, num_sms, st);
 }
 
 }  // namespace moeq4

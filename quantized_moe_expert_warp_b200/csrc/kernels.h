@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <utility>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "moeq4.h"
@@ -56,18 +57,12 @@ struct GemmArgs {
     int T;                      // tokens (rows of the shared expert)
     int E_total;                // E (+ 1 with a shared expert)
     int K;                      // reduction length (H for gate/up, I for down)
-    int ksplit;                 // router: K slices (partials out_f32 + slice * T * E); 1 otherwise
     int F;                      // 128-row tiles per expert matrix
     int G;                      // int4-sym group size
     int meta_bytes;             // per (expert, tile) meta block
     int ck_log2;                // k-steps per code chunk (set by the launcher)
     int ncs_log2;               // code chunks in the ring (set by the launcher)
     int nmeta_log2;             // meta blocks in the ring (set by the launcher)
-    const float *a_f32;         // router pass: fp32 A rows [E, K]
-    const float *bias;          // router pass: bias [E] or null
-    const float *gate_w;        // router pass: shared-expert gate vector [K] or null
-    float *gate_out;            // router pass: gate logits [T]
-    float *out_f32;             // router pass: logits [T, E]
     uint16_t *out;              // routed rows: out + p * ldo
     uint16_t *out_shared;       // shared rows: out_shared + (p - Tk) * ldo
     int ldo;
@@ -82,9 +77,18 @@ int gemm_down_tile_tokens(int T, int E, int k);
 cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int tile_tokens, int num_sms, cudaStream_t st);
 size_t gemm_smem_required(int nmat, int meta_bytes, int E_total);
 
+// Tensor map of a row-major 16-bit matrix [rows, ld] in boxes of 64
+// elements (128 bytes, 128-byte swizzle: the MMA's K-major layout) by
+// box_rows rows.
+cudaError_t encode_b_map(CUtensorMap *m, const uint16_t *src, int ld, int rows, int box_rows);
+
+// Router logits (or their K-slice partials) and the shared expert's gate
+// logits; wsplit: router_split_bytes(E, H) of scratch for the bf16 hi/lo
+// copies of the weights.  Two launches.
 cudaError_t launch_router_gemm(const uint16_t *x, int T, int H, const float *wr, const float *bias, int E,
-                               const float *gate_w, float *logits, float *gate_out, int ksplit, int *status,
-                               int num_sms, cudaStream_t st);
+                               const float *gate_w, float *logits, float *gate_out, int ksplit, uint16_t *wsplit,
+                               int *status, int num_sms, cudaStream_t st);
+size_t router_split_bytes(int E, int H);
 int router_ksplit(int T, int E, int H, int sms);
 // Top-k routing on logits [T, E], or on the sum of `nsplit` partials
 // part[s][T][E] (summed in slice order, bias added last); with partials the

@@ -288,6 +288,20 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, WaitCt
     return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
 }
 
+// A producer that stops early (a wait ran out, or another role gave up)
+// still waits, with a fresh bounded budget, until the copies it issued have
+// landed, so that none writes into this CTA's shared memory after it exits:
+// the last `depth` of the n_issued ring slots it filled.  On the normal path
+// every such phase has completed already.
+__device__ __forceinline__ void drain_ring(uint64_t *full, int n_issued, int depth, int *status, int where,
+                                           int *never_abort)
+{
+    WaitCtx wd{never_abort, status, globaltimer_ns(), kWaitLimitNs};
+    for (int i = max(0, n_issued - depth); i < n_issued; ++i)
+        if (!warp_wait(&full[i % depth], (i / depth) & 1, wd, where))
+            break;
+}
+
 // True on exactly one lane of a converged warp.  Single-thread tcgen05 and
 // bulk-copy instructions are issued under this predicate from a converged
 // warp: issuing them from a lone divergent lane costs several times longer.
