@@ -345,7 +345,11 @@ int run_expert_ffn(const moe_layer_t *L, const uint16_t *x, int T, const int32_t
         a.out = y_perm;
         a.out_shared = shared_out;
         a.ldo = c.H;
-        CUDA_TRY(launch_grouped_gemm(a, 1, c.wfmt, gemm_down_tile_tokens(T, c.E, c.k), num_sms(), st), "down GEMM");
+        if (down_resident_fits(c.I, a.meta_bytes, Et))
+            CUDA_TRY(launch_down_resident(a, c.wfmt, num_sms(), st), "down GEMM");
+        else
+            CUDA_TRY(launch_grouped_gemm(a, 1, c.wfmt, gemm_down_tile_tokens(T, c.E, c.k), num_sms(), st),
+                     "down GEMM");
         g_launches += 1;
     }
     return MOE_OK;

@@ -669,7 +669,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------ epilogue (last four warps)
-        const int r = (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         int uidx = 0;
         for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++uidx) {
@@ -683,7 +682,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0 && warp == 4 + kDeqWarps)
                 TRACE_OTHER(6, uidx);
             const uint32_t acc = tmem + lane_off + ab * L::kNAcc * kBN;
-            const int col = un.f * kTileRows + r;
             const int q = warp & 3;
             uint8_t *stage = s_epi + q * kEpiTok * kEpiStride;
             bool released = false;
@@ -836,6 +834,24 @@ cudaError_t encode_b_map(CUtensorMap *m, const uint16_t *src, int ld, int rows, 
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(src), dims, strides,
                            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t encode_kstep_map(CUtensorMap *m, const uint16_t *src, int ld, int rows, int box_rows, int box_ksteps)
+{
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc)
+        return cudaErrorNotSupported;
+    if ((reinterpret_cast<uintptr_t>(src) & 15) || rows < 1 || ld % kKStep || box_ksteps < 1 ||
+        box_ksteps > ld / kKStep || box_rows < 8 || box_rows > 256)
+        return cudaErrorInvalidValue;
+    const cuuint64_t dims[3] = {(cuuint64_t)kKStep, (cuuint64_t)rows, (cuuint64_t)(ld / kKStep)};
+    const cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)kKStep * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)kKStep, (cuuint32_t)box_rows, (cuuint32_t)box_ksteps};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t *>(src), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }

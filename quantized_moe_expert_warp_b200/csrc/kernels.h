@@ -63,6 +63,9 @@ struct GemmArgs {
     int ck_log2;                // k-steps per code chunk (set by the launcher)
     int ncs_log2;               // code chunks in the ring (set by the launcher)
     int nmeta_log2;             // meta blocks in the ring (set by the launcher)
+    int item_tiles;             // resident down pass: token tiles per work item (set by the launcher)
+    int b_stages, b_sk;         // resident down pass: B stages and k-steps per stage (set by the launcher)
+    int ncs, nmeta;             // resident down pass: code and scale ring depths (set by the launcher)
     uint16_t *out;              // routed rows: out + p * ldo
     uint16_t *out_shared;       // shared rows: out_shared + (p - Tk) * ldo
     int ldo;
@@ -75,12 +78,21 @@ int gemm_tile_tokens(int T, int E, int k);
 // Token-tile width of the down pass: 256 when experts average >= 128 rows, else as above.
 int gemm_down_tile_tokens(int T, int E, int k);
 cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int tile_tokens, int num_sms, cudaStream_t st);
+// Down pass with each dequantised 128-row weight tile resident in TMEM
+// (K <= 512) for up to eight token tiles of 128; down_resident_fits tells
+// whether a configuration can take it.
+bool down_resident_fits(int K, int meta_bytes, int E_total);
+cudaError_t launch_down_resident(const GemmArgs &a, int wfmt, int num_sms, cudaStream_t st);
 size_t gemm_smem_required(int nmat, int meta_bytes, int E_total);
 
 // Tensor map of a row-major 16-bit matrix [rows, ld] in boxes of 64
 // elements (128 bytes, 128-byte swizzle: the MMA's K-major layout) by
 // box_rows rows.
 cudaError_t encode_b_map(CUtensorMap *m, const uint16_t *src, int ld, int rows, int box_rows);
+// The same rows as a 3D map (64 elements, rows, ld / 64 k-steps; the third
+// dimension steps 128 bytes) in boxes of box_rows rows by box_ksteps
+// k-steps: one copy lands box_ksteps swizzled [box_rows x 64] slabs.
+cudaError_t encode_kstep_map(CUtensorMap *m, const uint16_t *src, int ld, int rows, int box_rows, int box_ksteps);
 
 // Router logits (or their K-slice partials) and the shared expert's gate
 // logits; wsplit: router_split_bytes(E, H) of scratch for the bf16 hi/lo
