@@ -134,28 +134,6 @@ __device__ __forceinline__ int mma_width(int nvalid) { return max(16, (nvalid + 
 // TMA box (index into the kernel's maps: 32, 64, 128 rows) for an MMA width
 __device__ __forceinline__ int box_index(int nmma) { return nmma <= 32 ? 0 : nmma <= 64 ? 1 : 2; }
 
-// One TMA copy of a 3D box: (64 elements of K, rows, k-steps) of a map whose
-// third dimension steps 128 bytes along a row, so the box lands as one
-// 128-byte-swizzled [rows x 64] slab per k-step.
-__device__ __forceinline__ void tma_load_3d(void *dst, const void *tmap, int x, int y, int z, uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-        "[%5];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// The last `depth` phases of a ring that one thread filled, waited for by that thread.
-__device__ __forceinline__ void drain_ring_lane(uint64_t *full, int n_issued, int depth, int *status, int where,
-                                                int *never_abort)
-{
-    WaitCtx wd{never_abort, status, globaltimer_ns(), kWaitLimitNs};
-    for (int i = max(0, n_issued - depth); i < n_issued; ++i)
-        if (!mbar_wait(&full[i % depth], (i / depth) & 1, wd, where))
-            break;
-}
-
 // Builds the schedule.  Rows of expert e are [offsets[e], offsets[e+1]);
 // the shared expert (if any) is expert E with rows [T k, T k + T).  Expert
 // e has t = ceil(rows / BN) token tiles: t / NT full items and, when t % NT

@@ -302,6 +302,16 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, int n_issued, int dep
             break;
 }
 
+// The last `depth` phases of a ring that one thread filled, waited for by that thread.
+__device__ __forceinline__ void drain_ring_lane(uint64_t *full, int n_issued, int depth, int *status, int where,
+                                                int *never_abort)
+{
+    WaitCtx wd{never_abort, status, globaltimer_ns(), kWaitLimitNs};
+    for (int i = max(0, n_issued - depth); i < n_issued; ++i)
+        if (!mbar_wait(&full[i % depth], (i / depth) & 1, wd, where))
+            break;
+}
+
 // True on exactly one lane of a converged warp.  Single-thread tcgen05 and
 // bulk-copy instructions are issued under this predicate from a converged
 // warp: issuing them from a lone divergent lane costs several times longer.
@@ -375,6 +385,18 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int x, 
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
         "[%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// One TMA copy of a 3D box: (64 elements of K, rows, k-steps) of a map whose
+// third dimension steps 128 bytes along a row, so the box lands as one
+// 128-byte-swizzled [rows x 64] slab per k-step.
+__device__ __forceinline__ void tma_load_3d(void *dst, const void *tmap, int x, int y, int z, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
         : "memory");
 }
 

@@ -215,6 +215,10 @@ SMALL_LAYERS = [
     # asymmetric int4 (scale and minimum per group of 64), shared expert
     small_cfg("asym_shared", T=150, H=512, E=8, k=2, I=256, has_shared=True, G=64, wr_std=0.03,
               wfmt=synth.WFMT_INT4_ASYM),
+    # K = I > 512: the down pass cannot keep a weight tile in TMEM and streams it (10 k-steps)
+    small_cfg("wide_down", T=300, H=256, E=8, k=2, I=640, has_shared=True, G=128, wr_std=0.03),
+    # the same with Q4K super-blocks (12 k-steps)
+    small_cfg("wide_down_q4k", T=200, H=512, E=4, k=2, I=768, G=256, wfmt=synth.WFMT_Q4K),
 ]
 
 
@@ -271,7 +275,7 @@ def test_fused_equals_composed_bitwise(dev, cfg):
     assert torch.equal(y.view(torch.int16), fused["y_bf16"].view(torch.int16))
 
 
-@pytest.mark.parametrize("cfg", [SMALL_LAYERS[5], SMALL_LAYERS[3], SMALL_LAYERS[1], SMALL_LAYERS[7]],
+@pytest.mark.parametrize("cfg", [SMALL_LAYERS[5], SMALL_LAYERS[3], SMALL_LAYERS[1], SMALL_LAYERS[7], SMALL_LAYERS[8]],
                          ids=lambda c: c.name)
 @pytest.mark.parametrize("ctas", [1, 3])
 def test_layer_on_few_ctas_is_bitwise_equal(dev, cfg, ctas, monkeypatch):
