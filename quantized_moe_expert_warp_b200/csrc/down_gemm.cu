@@ -28,9 +28,11 @@
 //   warp 1      MMA issuer (one elected thread)
 //   warp 2      code and scale blocks of each item, one bulk copy each
 //   warp 3      TMEM allocation
-//   warps 4-19  dequant: four groups of four warps; group g expands k-steps
-//               g, g + 4, ...; warp % 4 is the TMEM lane quadrant (32 rows)
-//   warps 20-23 epilogue (TMEM -> bf16 -> y rows)
+//   warps 4-15  dequant: three groups of four warps; group g expands k-steps
+//               g, g + 3, ...; warp % 4 is the TMEM lane quadrant (32 rows)
+//   warps 16-23 epilogue (TMEM -> bf16 -> y rows): two warps per lane
+//               quadrant take alternate 16-column chunks of a token tile, so
+//               that draining a tile takes no longer than its MMAs
 // Every wait is bounded; on timeout the CTA records MOE_ERR_TIMEOUT and
 // unwinds.
 //
@@ -57,15 +59,17 @@ namespace moeq4 {
 namespace {
 
 constexpr int kDnThreads = 768;
-constexpr int kDnDeqWarps = 16;
-constexpr int kDnGroups = 4;
+constexpr int kDnDeqWarps = 12;
+constexpr int kDnGroups = 3;
+constexpr int kDnEpiWarps = 8;
+static_assert(4 + kDnDeqWarps + kDnEpiWarps == kDnThreads / 32, "warp roles");
 constexpr int kDnMaxKS = 8;          // A slots: K <= 512
 constexpr int kDnMaxBStages = 4;
 constexpr int kDnMaxNCS = 2;         // code blocks of items in flight
 constexpr int kDnMaxMeta = 4;
 constexpr int kDnEpiTok = 16;
 constexpr int kDnEpiStride = 80;
-constexpr int kDnEpiBytes = 4 * kDnEpiTok * kDnEpiStride;
+constexpr int kDnEpiBytes = kDnEpiWarps * kDnEpiTok * kDnEpiStride;
 constexpr int kDnCodeStep = code_block_bytes(1);   // 4 KB: one k-step of a 128-row tile
 
 struct DnBars {
@@ -208,7 +212,7 @@ __device__ void dn_build_schedule(const GemmArgs &p, const DnSched &s, DnBars *b
     __syncthreads();
 }
 
-template <int WFMT, int BN>
+template <int WFMT, int BN, int SK>
 __global__ void __launch_bounds__(kDnThreads, 1)
     down_resident_kernel(const __grid_constant__ GemmArgs p, const __grid_constant__ CUtensorMap tmap32,
                          const __grid_constant__ CUtensorMap tmap64, const __grid_constant__ CUtensorMap tmap128)
@@ -218,7 +222,6 @@ __global__ void __launch_bounds__(kDnThreads, 1)
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int KS = p.K / kKStep;
     const int NB = p.b_stages;                // B ring depth
-    const int SK = p.b_sk;                    // k-steps per B stage
     const int stage_bytes = BN * 128 * SK;
     const int NCS = p.ncs;                    // code ring depth (items)
     const int NMETA = p.nmeta;
@@ -260,7 +263,7 @@ __global__ void __launch_bounds__(kDnThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->acc_full[s], 1);
-            mbar_init(&bars->acc_empty[s], 4);
+            mbar_init(&bars->acc_empty[s], kDnEpiWarps);
         }
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
@@ -313,7 +316,9 @@ __global__ void __launch_bounds__(kDnThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        int step = 0, tidx = 0, iidx = 0;
+        int tidx = 0, iidx = 0;
+        int sb = 0;            // B ring slot of the next stage
+        uint32_t bpar = 0;     // and the parity of its phase
         bool ok = true;
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x, ++iidx) {
             const DnItem it = dn_item<BN>(u, p, sched, n_full);
@@ -331,31 +336,60 @@ __global__ void __launch_bounds__(kDnThreads, 1)
                 }
                 const bool last = j == it.ntiles - 1;
                 const int box_rows = 32 << box_index(nmma);   // rows per k-step slab of the stage
-                for (int k0 = 0; k0 < KS && ok; k0 += SK, ++step) {
-                    const int sb = step % NB;
-                    if (!mbar_wait(&bars->b_full[sb], (step / NB) & 1, wc, 45)) {
+                for (int k0 = 0; k0 < KS && ok; k0 += SK) {
+                    if (!mbar_wait(&bars->b_full[sb], bpar, wc, 45)) {
                         ok = false;
                         break;
                     }
-                    for (int ks = k0; ks < k0 + SK; ++ks) {
-                        if (j == 0 && !mbar_wait(&bars->a_full[ks], iidx & 1, wc, 44)) {
-                            ok = false;
-                            break;
-                        }
+                    const uint32_t sbase = smem_u32(sB + sb * stage_bytes);
+                    if (j > 0) {
+                        // weights already in TMEM: the stage's SK x 4 MMAs straight from one
+                        // elected lane (issue cost, not the tensor pipe, bounds a loop with
+                        // per-k-step bookkeeping at N = 128)
                         tc_fence_after();
-                        const uint64_t bdesc0 =
-                            sdesc_kmajor_sw128(smem_u32(sB + sb * stage_bytes + (ks - k0) * box_rows * 128));
-                        const uint32_t a_base = tmem + kAccCols + ks * 32;
                         if (elect_one()) {
+                            const uint64_t d0 = sdesc_kmajor_sw128(sbase);
+                            const uint32_t a0 = tmem + kAccCols + k0 * 32;
+                            const uint32_t slab = (uint32_t)(box_rows * 8);   // descriptor units of a k-step slab
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma_ts_f16(acc, a_base + kk * 8, bdesc0 + (uint64_t)(kk * 2), idesc, (ks | kk) != 0);
-                            if (ks == k0 + SK - 1)
-                                mma_commit(&bars->b_empty[sb]);
-                            if (last)   // the item's weights in this slot are no longer needed
-                                mma_commit(&bars->a_empty[ks]);
+                            for (int t = 0; t < SK; ++t)
+#pragma unroll
+                                for (int kk = 0; kk < 4; ++kk)
+                                    mma_ts_f16(acc, a0 + t * 32 + kk * 8, d0 + (uint64_t)(t * slab + kk * 2), idesc,
+                                               (t | kk) ? 1u : (uint32_t)k0);
+                            if (last) {   // the item's weights in these slots are no longer needed
+#pragma unroll
+                                for (int t = 0; t < SK; ++t)
+                                    mma_commit(&bars->a_empty[k0 + t]);
+                            }
+                            mma_commit(&bars->b_empty[sb]);
                         }
                         __syncwarp();
+                    } else {
+                        // first tile of the item: each k-step waits for its slot's weights
+                        for (int ks = k0; ks < k0 + SK; ++ks) {
+                            if (!mbar_wait(&bars->a_full[ks], iidx & 1, wc, 44)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint64_t bdesc0 = sdesc_kmajor_sw128(sbase + (ks - k0) * box_rows * 128);
+                            const uint32_t a_base = tmem + kAccCols + ks * 32;
+                            if (elect_one()) {
+#pragma unroll
+                                for (int kk = 0; kk < 4; ++kk)
+                                    mma_ts_f16(acc, a_base + kk * 8, bdesc0 + (uint64_t)(kk * 2), idesc, ks | kk);
+                                if (ks == k0 + SK - 1)
+                                    mma_commit(&bars->b_empty[sb]);
+                                if (last)
+                                    mma_commit(&bars->a_empty[ks]);
+                            }
+                            __syncwarp();
+                        }
+                    }
+                    if (++sb == NB) {
+                        sb = 0;
+                        bpar ^= 1u;
                     }
                 }
                 if (ok) {
@@ -464,9 +498,10 @@ __global__ void __launch_bounds__(kDnThreads, 1)
         }
     } else if (warp >= 4 + kDnDeqWarps) {
         // ------------------------------------------------ epilogue (one token tile at a time)
-        const int q = warp & 3;
+        const int q = warp & 3;                        // TMEM lane quadrant
+        const int half = (warp - 4 - kDnDeqWarps) >> 2;   // chunks half, half + 2, ...
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        uint8_t *stage = s_epi + q * kDnEpiTok * kDnEpiStride;
+        uint8_t *stage = s_epi + (warp - 4 - kDnDeqWarps) * kDnEpiTok * kDnEpiStride;
         int tidx = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
@@ -482,12 +517,19 @@ __global__ void __launch_bounds__(kDnThreads, 1)
                 const int nmma = mma_width(nvalid);
                 const int row0 = it.row0 + j * BN;
                 const uint32_t acc = tmem + lane_off + ab * BN;
-                for (int n0 = 0; n0 < nmma; n0 += kDnEpiTok) {
-                    uint32_t g[16];
+                int n0 = half * kDnEpiTok;
+                uint32_t g[16], nx[16];
+                if (n0 < nmma) {
                     tmem_ld16(acc + n0, g);
                     tmem_wait_ld();
-                    if (n0 + kDnEpiTok >= nmma) {
-                        // every column is in registers: hand the accumulator back
+                }
+                for (; n0 < nmma; n0 += 2 * kDnEpiTok) {
+                    // the next chunk's columns load while this one is stored
+                    const bool more = n0 + 2 * kDnEpiTok < nmma;
+                    if (more)
+                        tmem_ld16(acc + n0 + 2 * kDnEpiTok, nx);
+                    else {
+                        // every column of this warp is in registers: hand the accumulator back
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0)
@@ -512,6 +554,19 @@ __global__ void __launch_bounds__(kDnThreads, 1)
                         d4[1] = s4[1];
                     }
                     __syncwarp();
+                    if (more) {
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj)
+                            g[jj] = nx[jj];
+                    }
+                }
+                if (half * kDnEpiTok >= nmma) {
+                    // no chunk of this tile for this warp
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&bars->acc_empty[ab]);
                 }
             }
         }
@@ -538,27 +593,27 @@ size_t dn_smem_bytes(int BN, int KS, int meta_bytes, int E_total, const DnRings 
 constexpr size_t kDnSmemLimit = 227 * 1024;
 
 // B stages of four k-steps (two or one when K/64 is not a multiple of four),
-// three stages where they fit, else two; two code blocks, up to four scale
-// blocks.
+// three stages where they fit, else two; two code blocks; four scale blocks
+// where they fit, else two.
 bool dn_rings(int BN, int KS, int meta_bytes, int E_total, DnRings &r)
 {
-    r.b_sk = KS % 4 == 0 ? 4 : KS % 2 == 0 ? 2 : 1;
+    r.b_sk = KS % 4 == 0 ? 4 : 2;
     r.ncs = 2;
-    r.nmeta = meta_bytes <= 4096 ? 4 : 2;
-    for (r.b_stages = kDnMaxBStages - 1; r.b_stages >= 2; --r.b_stages)
-        if (dn_smem_bytes(BN, KS, meta_bytes, E_total, r) <= kDnSmemLimit)
-            return true;
+    for (r.nmeta = meta_bytes <= 4096 ? 4 : 2; r.nmeta >= 2; r.nmeta /= 2)
+        for (r.b_stages = kDnMaxBStages - 1; r.b_stages >= 2; --r.b_stages)
+            if (dn_smem_bytes(BN, KS, meta_bytes, E_total, r) <= kDnSmemLimit)
+                return true;
     return false;
 }
 
-template <int WFMT, int BN>
+template <int WFMT, int BN, int SK>
 cudaError_t launch_dn(const GemmArgs &a_in, int num_sms, cudaStream_t st)
 {
-    auto kern = down_resident_kernel<WFMT, BN>;
+    auto kern = down_resident_kernel<WFMT, BN, SK>;
     GemmArgs a = a_in;
     const int KS = a.K / kKStep;
     DnRings r{};
-    if (!dn_rings(BN, KS, a.meta_bytes, a.E_total, r))
+    if (!dn_rings(BN, KS, a.meta_bytes, a.E_total, r) || r.b_sk != SK)
         return cudaErrorInvalidConfiguration;
     CUtensorMap m32{}, m64{}, m128{};
     cudaError_t e = encode_kstep_map(&m32, a_in.b_src, a_in.ldb, a_in.b_rows, 32, r.b_sk);
@@ -584,23 +639,32 @@ cudaError_t launch_dn(const GemmArgs &a_in, int num_sms, cudaStream_t st)
 bool down_resident_fits(int K, int meta_bytes, int E_total)
 {
     DnRings r{};
-    return K % kKStep == 0 && K / kKStep <= kDnMaxKS && dn_rings(128, K / kKStep, meta_bytes, E_total, r);
+    return K % kKStep == 0 && K / kKStep <= kDnMaxKS && (K / kKStep) % 2 == 0 &&
+           dn_rings(128, K / kKStep, meta_bytes, E_total, r);
 }
 
 #ifndef MOEQ4_DOWN_ITEM_TILES
 #define MOEQ4_DOWN_ITEM_TILES 8
 #endif
 
+template <int SK>
+cudaError_t launch_dn_fmt(const GemmArgs &a, int wfmt, int num_sms, cudaStream_t st)
+{
+    return wfmt == MOE_WFMT_Q4K           ? launch_dn<MOE_WFMT_Q4K, 128, SK>(a, num_sms, st)
+           : wfmt == MOE_WFMT_INT4_ASYM   ? launch_dn<MOE_WFMT_INT4_ASYM, 128, SK>(a, num_sms, st)
+           : wfmt == MOE_WFMT_INT4_SYM_F16 ? launch_dn<MOE_WFMT_INT4_SYM_F16, 128, SK>(a, num_sms, st)
+                                           : launch_dn<MOE_WFMT_INT4_SYM, 128, SK>(a, num_sms, st);
+}
+
 cudaError_t launch_down_resident(const GemmArgs &a_in, int wfmt, int num_sms, cudaStream_t st)
 {
     GemmArgs a = a_in;
     a.item_tiles = MOEQ4_DOWN_ITEM_TILES;
-    if (a.item_tiles < 1 || a.item_tiles > 16 || a.K / kKStep > kDnMaxKS || a.K % kKStep)
+    const int KS = a.K / kKStep;
+    if (a.item_tiles < 1 || a.item_tiles > 16 || KS > kDnMaxKS || a.K % kKStep || KS % 2)
         return cudaErrorInvalidValue;
-    return wfmt == MOE_WFMT_Q4K           ? launch_dn<MOE_WFMT_Q4K, 128>(a, num_sms, st)
-           : wfmt == MOE_WFMT_INT4_ASYM   ? launch_dn<MOE_WFMT_INT4_ASYM, 128>(a, num_sms, st)
-           : wfmt == MOE_WFMT_INT4_SYM_F16 ? launch_dn<MOE_WFMT_INT4_SYM_F16, 128>(a, num_sms, st)
-                                           : launch_dn<MOE_WFMT_INT4_SYM, 128>(a, num_sms, st);
+    // k-steps per B stage: four, or two when K / 64 is not a multiple of four
+    return KS % 4 == 0 ? launch_dn_fmt<4>(a, wfmt, num_sms, st) : launch_dn_fmt<2>(a, wfmt, num_sms, st);
 }
 
 }  // namespace moeq4
