@@ -342,51 +342,36 @@ __global__ void __launch_bounds__(kDnThreads, 1)
                         break;
                     }
                     const uint32_t sbase = smem_u32(sB + sb * stage_bytes);
-                    if (j > 0) {
-                        // weights already in TMEM: the stage's SK x 4 MMAs straight from one
-                        // elected lane (issue cost, not the tensor pipe, bounds a loop with
-                        // per-k-step bookkeeping at N = 128)
-                        tc_fence_after();
-                        if (elect_one()) {
-                            const uint64_t d0 = sdesc_kmajor_sw128(sbase);
-                            const uint32_t a0 = tmem + kAccCols + k0 * 32;
-                            const uint32_t slab = (uint32_t)(box_rows * 8);   // descriptor units of a k-step slab
+                    if (j == 0) {
+                        // first tile of the item: the stage's weight slots must be filled
+#pragma unroll
+                        for (int t = 0; t < SK; ++t)
+                            if (ok && !mbar_wait(&bars->a_full[k0 + t], iidx & 1, wc, 44))
+                                ok = false;
+                        if (!ok)
+                            break;
+                    }
+                    // the stage's SK x 4 MMAs straight from one elected lane (issue cost,
+                    // not the tensor pipe, bounds a loop with per-k-step bookkeeping at N = 128)
+                    tc_fence_after();
+                    if (elect_one()) {
+                        const uint64_t d0 = sdesc_kmajor_sw128(sbase);
+                        const uint32_t a0 = tmem + kAccCols + k0 * 32;
+                        const uint32_t slab = (uint32_t)(box_rows * 8);   // descriptor units of a k-step slab
+#pragma unroll
+                        for (int t = 0; t < SK; ++t)
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_ts_f16(acc, a0 + t * 32 + kk * 8, d0 + (uint64_t)(t * slab + kk * 2), idesc,
+                                           (t | kk) ? 1u : (uint32_t)k0);
+                        if (last) {   // the item's weights in these slots are no longer needed
 #pragma unroll
                             for (int t = 0; t < SK; ++t)
-#pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    mma_ts_f16(acc, a0 + t * 32 + kk * 8, d0 + (uint64_t)(t * slab + kk * 2), idesc,
-                                               (t | kk) ? 1u : (uint32_t)k0);
-                            if (last) {   // the item's weights in these slots are no longer needed
-#pragma unroll
-                                for (int t = 0; t < SK; ++t)
-                                    mma_commit(&bars->a_empty[k0 + t]);
-                            }
-                            mma_commit(&bars->b_empty[sb]);
+                                mma_commit(&bars->a_empty[k0 + t]);
                         }
-                        __syncwarp();
-                    } else {
-                        // first tile of the item: each k-step waits for its slot's weights
-                        for (int ks = k0; ks < k0 + SK; ++ks) {
-                            if (!mbar_wait(&bars->a_full[ks], iidx & 1, wc, 44)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            const uint64_t bdesc0 = sdesc_kmajor_sw128(sbase + (ks - k0) * box_rows * 128);
-                            const uint32_t a_base = tmem + kAccCols + ks * 32;
-                            if (elect_one()) {
-#pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    mma_ts_f16(acc, a_base + kk * 8, bdesc0 + (uint64_t)(kk * 2), idesc, ks | kk);
-                                if (ks == k0 + SK - 1)
-                                    mma_commit(&bars->b_empty[sb]);
-                                if (last)
-                                    mma_commit(&bars->a_empty[ks]);
-                            }
-                            __syncwarp();
-                        }
+                        mma_commit(&bars->b_empty[sb]);
                     }
+                    __syncwarp();
                     if (++sb == NB) {
                         sb = 0;
                         bpar ^= 1u;
