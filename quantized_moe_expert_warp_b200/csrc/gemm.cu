@@ -886,12 +886,24 @@ size_t gemm_smem_required(int nmat, int meta_bytes, int E_total)
     const Rings r{1, 1, 1};
     const size_t a = nmat == 2 ? gemm_smem_bytes<MODE_GATE_UP, 64>(meta_bytes, E_total, r)
                                : gemm_smem_bytes<MODE_DOWN, 64>(meta_bytes, E_total, r);
-    const size_t b = nmat == 2 ? gemm_smem_bytes<MODE_GATE_UP, 128>(meta_bytes, E_total, r)
+    const size_t b = nmat == 2 ? gemm_smem_bytes<MODE_GATE_UP, 192>(meta_bytes, E_total, r)
                                : gemm_smem_bytes<MODE_DOWN, 256>(meta_bytes, E_total, r);
-    return a > b ? a : b;
+    const size_t c = nmat == 2 ? gemm_smem_bytes<MODE_GATE_UP, 128>(meta_bytes, E_total, r) : 0;
+    return a > b ? (a > c ? a : c) : (b > c ? b : c);
 }
 
-int gemm_tile_tokens(int T, int E, int k) { return (long long)T * k <= 64LL * E ? 64 : 128; }
+// Gate/up token tiles: 64 when experts average at most 64 rows, 192 when
+// they average at least 128 (one accumulator of 2 x 192 columns and two A
+// stages fill TMEM: half again the MMA work per dequantised k-step), else 128.
+#ifndef MOEQ4_GU_TILE_MAX
+#define MOEQ4_GU_TILE_MAX 192
+#endif
+int gemm_tile_tokens(int T, int E, int k)
+{
+    if ((long long)T * k <= 64LL * E)
+        return 64;
+    return MOEQ4_GU_TILE_MAX >= 192 && (long long)T * k >= 128LL * E ? 192 : 128;
+}
 
 // The down pass reads its token rows with TMA and has a single matrix, so
 // when experts average at least 128 rows it takes 256-token tiles: twice the
@@ -901,7 +913,9 @@ int gemm_tile_tokens(int T, int E, int k) { return (long long)T * k <= 64LL * E 
 #endif
 int gemm_down_tile_tokens(int T, int E, int k)
 {
-    return MOEQ4_DOWN_TILE_MAX >= 256 && (long long)T * k >= 128LL * E ? 256 : gemm_tile_tokens(T, E, k);
+    if (MOEQ4_DOWN_TILE_MAX >= 256 && (long long)T * k >= 128LL * E)
+        return 256;
+    return (long long)T * k <= 64LL * E ? 64 : 128;
 }
 
 template <int MODE, int BN>
@@ -916,8 +930,9 @@ static cudaError_t launch_fmt(const GemmArgs &a, int wfmt, int num_sms, cudaStre
 cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int tile_tokens, int num_sms, cudaStream_t st)
 {
     if (nmat == 2)
-        return tile_tokens == 64 ? launch_fmt<MODE_GATE_UP, 64>(a, wfmt, num_sms, st)
-                                 : launch_fmt<MODE_GATE_UP, 128>(a, wfmt, num_sms, st);
+        return tile_tokens == 64    ? launch_fmt<MODE_GATE_UP, 64>(a, wfmt, num_sms, st)
+               : tile_tokens == 192 ? launch_fmt<MODE_GATE_UP, 192>(a, wfmt, num_sms, st)
+                                    : launch_fmt<MODE_GATE_UP, 128>(a, wfmt, num_sms, st);
     return tile_tokens == 64    ? launch_fmt<MODE_DOWN, 64>(a, wfmt, num_sms, st)
            : tile_tokens == 128 ? launch_fmt<MODE_DOWN, 128>(a, wfmt, num_sms, st)
                                 : launch_fmt<MODE_DOWN, 256>(a, wfmt, num_sms, st);
