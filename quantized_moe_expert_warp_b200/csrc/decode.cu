@@ -48,6 +48,7 @@
 #include "dequant.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
+#include "topk.cuh"
 
 #ifdef MOEQ4_TRACE
 // phase timestamps (%globaltimer) of the first four CTAs, thread 0
@@ -149,10 +150,6 @@ __device__ bool grid_sync(unsigned *bar, int *status, int where, int *s_flag)
     return *s_flag != 0;
 }
 
-__device__ __forceinline__ bool better(float v, int id, float bv, int bid)
-{
-    return v > bv || (v == bv && id < bid);
-}
 
 // (a, b) of one 32-weight chunk so that weight_i = a * c_i + b, where c_i
 // is the decoded code (q = u - 8 for int4-sym with b = 0, u for the
@@ -193,38 +190,10 @@ __device__ __forceinline__ void topk_warp(const float *Lrow, int E, int k, int r
         const int e = i * 32 + lane;
         v[i] = e < E ? __ldcg(Lrow + e) : -CUDART_INF_F;
     }
-    uint32_t taken = 0;
-    float top = 0.f, my_val = 0.f;
-    my_id = -1;
-    for (int j = 0; j < k; ++j) {
-        float bv = -CUDART_INF_F;
-        int bid = 0x7FFFFFFF;
-#pragma unroll
-        for (int i = 0; i < NPL; ++i) {
-            const int e = i * 32 + lane;
-            if (e < E && !((taken >> i) & 1u) && better(v[i], e, bv, bid)) {
-                bv = v[i];
-                bid = e;
-            }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-            const int oid = __shfl_xor_sync(0xFFFFFFFFu, bid, off);
-            if (better(ov, oid, bv, bid)) {
-                bv = ov;
-                bid = oid;
-            }
-        }
-        if (bid != 0x7FFFFFFF && (bid & 31) == lane)
-            taken |= 1u << (bid >> 5);
-        if (j == 0)
-            top = bv;
-        if (lane == j) {
-            my_val = bv;
-            my_id = bid == 0x7FFFFFFF ? -1 : bid;
-        }
-    }
+    float top, my_val;
+    warp_topk<NPL>(v, E, k, lane, my_val, my_id, top);
+    if (my_id == 0x7FFFFFFF)
+        my_id = -1;
     const float ex = lane < k ? expf(my_val - top) : 0.f;
     float z;
     if (renorm) {

@@ -11,16 +11,12 @@
 
 #include "kernels.h"
 #include "ptx.cuh"
+#include "topk.cuh"
 
 namespace moeq4 {
 
 // ------------------------------------------------------------------ top-k
-// One warp per token; lane l holds logits l, l+32, ... in registers.
-
-__device__ __forceinline__ bool better(float v, int id, float bv, int bid)
-{
-    return v > bv || (v == bv && id < bid);
-}
+// One warp per token (warp_topk in topk.cuh).
 
 // Router logit of (t, e) from split-K partials: slices summed in order,
 // then the bias.  Shared by the route and reduce kernels so that both give
@@ -87,39 +83,9 @@ __global__ void __launch_bounds__(128) route_kernel(const float *__restrict__ lo
             v[i] = e < E ? L[e] : -CUDART_INF_F;
         }
     }
-    uint32_t taken = 0;
-    float top = 0.f, my_val = 0.f;
-    int my_id = 0;
-    for (int j = 0; j < k; ++j) {
-        float bv = -CUDART_INF_F;
-        int bid = 0x7FFFFFFF;
-#pragma unroll
-        for (int i = 0; i < NPL; ++i) {
-            const int e = i * 32 + lane;
-            if (e < E && !((taken >> i) & 1u) && better(v[i], e, bv, bid)) {
-                bv = v[i];
-                bid = e;
-            }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-            const int oid = __shfl_xor_sync(0xFFFFFFFFu, bid, off);
-            if (better(ov, oid, bv, bid)) {
-                bv = ov;
-                bid = oid;
-            }
-        }
-        // bid stays 0x7FFFFFFF only when every remaining logit is NaN
-        if (bid != 0x7FFFFFFF && (bid & 31) == lane)
-            taken |= 1u << (bid >> 5);
-        if (j == 0)
-            top = bv;
-        if (lane == j) {
-            my_val = bv;
-            my_id = bid;
-        }
-    }
+    float top, my_val;
+    int my_id;
+    warp_topk<NPL>(v, E, k, lane, my_val, my_id, top);
     const float ex = lane < k ? expf(my_val - top) : 0.f;
     float z;
     if (renorm) {
