@@ -64,7 +64,7 @@ L2_BYTES = 126e6   # B200 L2
 # The profiled kernels (router, gate/up and down GEMMs) are compiled from
 # these files alone; other translation units and the public header's
 # declarations do not change their code.
-GEMM_SOURCES = ("dequant.cuh", "gemm.cu", "kernels.h", "ptx.cuh")
+GEMM_SOURCES = ("dequant.cuh", "gemm.cu", "down_gemm.cu", "kernels.h", "ptx.cuh")
 
 
 def kernel_source_hash() -> str:

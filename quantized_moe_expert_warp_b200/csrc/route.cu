@@ -53,15 +53,26 @@ __global__ void __launch_bounds__(128) route_kernel(const float *__restrict__ lo
             const int e = i * 32 + lane;
             v[i] = e < E ? row[e] : 0.f;
         }
-#pragma unroll 2
-        for (int sl = 1; sl < nsplit; ++sl) {
-            const float *r = row + (size_t)sl * TE;
+        // slices 1, 2, ... in groups (four while the values fit in registers):
+        // a group's loads are issued together, then added in slice order
+        constexpr int G = NPL <= 8 ? 4 : 1;
+        for (int sl = 1; sl < nsplit; sl += G) {
+            float g[G][NPL];
 #pragma unroll
-            for (int i = 0; i < NPL; ++i) {
-                const int e = i * 32 + lane;
-                if (e < E)
-                    v[i] += r[e];
+            for (int q = 0; q < G; ++q) {
+                const float *r = row + (size_t)(sl + q) * TE;
+#pragma unroll
+                for (int i = 0; i < NPL; ++i) {
+                    const int e = i * 32 + lane;
+                    g[q][i] = sl + q < nsplit && e < E ? r[e] : 0.f;
+                }
             }
+#pragma unroll
+            for (int q = 0; q < G; ++q)
+#pragma unroll
+                for (int i = 0; i < NPL; ++i)
+                    if (sl + q < nsplit && i * 32 + lane < E)
+                        v[i] += g[q][i];
         }
 #pragma unroll
         for (int i = 0; i < NPL; ++i) {

@@ -23,17 +23,22 @@ __device__ __forceinline__ uint32_t order_key(float v)
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Lane j < k gets the j-th largest logit (val) and its expert id (id;
-// 0x7FFFFFFF and val = -inf where every remaining logit is NaN); every lane
-// gets the largest logit (top).
+// The logit of an order key (not 0).
+__device__ __forceinline__ float key_value(uint32_t key)
+{
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// Lane j < k gets the j-th largest logit (my_val; a -0 logit as +0) and its
+// expert id (my_id; 0x7FFFFFFF and my_val = -inf where every remaining
+// logit is NaN); every lane gets the largest logit (top).  The selection
+// carries no per-lane value array: the owner lane marks its logit taken in
+// a bit mask, and the value is recovered from the winning key.
 template <int NPL>
 __device__ __forceinline__ void warp_topk(const float (&v)[NPL], int E, int k, int lane, float &my_val, int &my_id,
                                           float &top)
 {
-    uint32_t key[NPL];
-#pragma unroll
-    for (int i = 0; i < NPL; ++i)
-        key[i] = i * 32 + lane < E ? order_key(v[i]) : 0u;
+    uint32_t taken = 0u;   // bit i: logit i * 32 + lane already chosen
     top = 0.f;
     my_val = -CUDART_INF_F;
     my_id = 0x7FFFFFFF;
@@ -42,25 +47,23 @@ __device__ __forceinline__ void warp_topk(const float (&v)[NPL], int E, int k, i
         uint32_t bk = 0u;
         int bi = 0;
 #pragma unroll
-        for (int i = 0; i < NPL; ++i)
-            if (key[i] > bk) {
-                bk = key[i];
+        for (int i = 0; i < NPL; ++i) {
+            const uint32_t ki = i * 32 + lane < E && !((taken >> i) & 1u) ? order_key(v[i]) : 0u;
+            if (ki > bk) {
+                bk = ki;
                 bi = i;
             }
+        }
         const uint32_t wk = __reduce_max_sync(0xFFFFFFFFu, bk);
         const int bid = (int)__reduce_min_sync(0xFFFFFFFFu, (wk != 0u && bk == wk) ? (uint32_t)(bi * 32 + lane)
                                                                                    : 0x7FFFFFFFu);
-        float val = -CUDART_INF_F;   // an unfilled position adds nothing to the softmax sums
-        if (bid != 0x7FFFFFFF) {     // warp-uniform
-            float mine = 0.f;
-#pragma unroll
-            for (int i = 0; i < NPL; ++i)
-                if (i == (bid >> 5)) {
-                    mine = v[i];
-                    if ((bid & 31) == lane)
-                        key[i] = 0u;   // taken
-                }
-            val = __shfl_sync(0xFFFFFFFFu, mine, bid & 31);
+        // the chosen logit is the key's inverse (a -0 logit comes back as +0, which
+        // changes no softmax term); an unfilled position adds nothing to the sums
+        float val = -CUDART_INF_F;
+        if (bid != 0x7FFFFFFF) {   // warp-uniform
+            val = key_value(wk);
+            if ((bid & 31) == lane)
+                taken |= 1u << (bid >> 5);
         }
         if (j == 0)
             top = val;
