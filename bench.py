@@ -61,17 +61,19 @@ WFMT_NAMES = {0: "int4-sym", 1: "q4k", 2: "int4-asym", 3: "int4-sym, fp16 operan
 L2_BYTES = 126e6   # B200 L2
 
 
-# The profiled kernels (router, gate/up and down GEMMs) are compiled from
-# these files alone; other translation units and the public header's
-# declarations do not change their code.
+# The profiled kernels are compiled from these files alone (other
+# translation units and the public header's declarations do not change
+# their code): the grouped GEMMs, and the fused decode kernel.
 GEMM_SOURCES = ("dequant.cuh", "gemm.cu", "down_gemm.cu", "kernels.h", "ptx.cuh")
+DECODE_SOURCES = ("decode.cu", "decode.h", "dequant.cuh", "kernels.h", "ptx.cuh", "topk.cuh")
 
 
-def kernel_source_hash() -> str:
-    """Hash of the sources of the profiled GEMM kernels (GEMM_SOURCES under
-    csrc/): a committed ncu figure counts only while it matches."""
+def kernel_source_hash(kernel_tag: str = "gate_up") -> str:
+    """Hash of the sources of a profiled kernel (GEMM_SOURCES, or
+    DECODE_SOURCES for the fused decode kernel, under csrc/): a committed
+    ncu figure counts only while it matches."""
     h = hashlib.sha256()
-    for name in GEMM_SOURCES:
+    for name in DECODE_SOURCES if kernel_tag == "decode" else GEMM_SOURCES:
         with open(os.path.join(ROOT, "quantized_moe_expert_warp_b200", "csrc", name), "rb") as fh:
             h.update(name.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -88,7 +90,7 @@ def ncu_traffic(kernel_tag: str, workload: str):
         if ":" in line:
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
-    if vals.get("source_sha256") != kernel_source_hash():
+    if vals.get("source_sha256") != kernel_source_hash(kernel_tag):
         return None
     try:
         return int(float(vals["dram_bytes_per_launch"]))

@@ -278,15 +278,25 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t *__rest
         const int t = p < rows ? sorted_slot[p] / k : p - rows;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
         uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)p * H);
-        for (int i = lane; i < n16; i += 32) {
-            uint4 v = src[i];
-            if (to_f16) {
-                v.x = bf16x2_to_f16x2(v.x, bad);
-                v.y = bf16x2_to_f16x2(v.y, bad);
-                v.z = bf16x2_to_f16x2(v.z, bad);
-                v.w = bf16x2_to_f16x2(v.w, bad);
+        // four 16-byte loads per lane in flight before their stores
+        for (int i0 = lane; i0 < n16; i0 += 4 * 32) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (i0 + 32 * u < n16)
+                    v[u] = src[i0 + 32 * u];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (i0 + 32 * u >= n16)
+                    break;
+                if (to_f16) {
+                    v[u].x = bf16x2_to_f16x2(v[u].x, bad);
+                    v[u].y = bf16x2_to_f16x2(v[u].y, bad);
+                    v[u].z = bf16x2_to_f16x2(v[u].z, bad);
+                    v[u].w = bf16x2_to_f16x2(v[u].w, bad);
+                }
+                dst[i0 + 32 * u] = v[u];
             }
-            dst[i] = v;
         }
     }
     if (bad)
