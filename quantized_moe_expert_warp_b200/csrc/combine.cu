@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict
     for (int c = threadIdx.x % chunks; c < chunks; c += blockDim.x) {
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         // the shared expert's row is loaded with the first batch, added last
-        const uint4 sv = shared_out ? *(const uint4 *)(shared_out + (size_t)t * H + c * 8) : make_uint4(0, 0, 0, 0);
+        const uint4 sv = shared_out ? __ldcs((const uint4 *)(shared_out + (size_t)t * H + c * 8)) : make_uint4(0, 0, 0, 0);
         // batches of 8 rows: all loads of a batch are in flight together
         for (int j0 = 0; j0 < k; j0 += 8) {
             uint4 v[8];
@@ -57,7 +57,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict
                 const int p = j0 + j < k ? dp[j0 + j] : -1;
                 const bool ok = p >= 0 && p < S;
                 wj[j] = ok ? wt[j0 + j] : 0.f;
-                v[j] = ok ? *(const uint4 *)(y_perm + (size_t)p * H + c * 8) : make_uint4(0, 0, 0, 0);
+                // each row is read once: streaming loads keep it out of the way in L1 and L2
+                v[j] = ok ? __ldcs((const uint4 *)(y_perm + (size_t)p * H + c * 8)) : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
             for (int j = 0; j < 8; ++j)
