@@ -219,6 +219,8 @@ SMALL_LAYERS = [
     small_cfg("wide_down", T=300, H=256, E=8, k=2, I=640, has_shared=True, G=128, wr_std=0.03),
     # the same with Q4K super-blocks (12 k-steps)
     small_cfg("wide_down_q4k", T=200, H=512, E=4, k=2, I=768, G=256, wfmt=synth.WFMT_Q4K),
+    # 1024 routed experts + shared: schedules over more experts than threads, eight router expert tiles
+    small_cfg("many_experts", T=600, H=256, E=1024, k=4, I=128, has_shared=True, G=64, wr_std=0.05),
 ]
 
 
