@@ -129,41 +129,56 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float *__restri
 }
 
 // gate_out[t] = x[t] . g in fp32: one warp per token, lane l takes the
-// 8-element chunks l, l + 32, ... in order (four in flight), then a
-// butterfly sum over the lanes.
+// 8-element chunks l, l + 32, ... in order, then a butterfly sum over the
+// lanes.  A warp takes two tokens at a time, and a token's whole row (up to
+// 2048 elements: eight 16-byte loads per lane) is loaded before its FMAs.
 __device__ void gate_logits(const RouterArgs &p, int worker, int nworkers)
 {
     const int lane = threadIdx.x % 32;
-    for (int t = worker; t < p.T; t += nworkers) {
-        const uint16_t *xr = p.x + (size_t)t * p.H;
-        float acc = 0.f;
-        for (int base = lane * 8; base < p.H; base += 4 * 256) {
-            uint4 v[4];
+    constexpr int kChunks = 8;   // 16-byte loads in flight per lane and token
+    for (int t0 = 2 * worker; t0 < p.T; t0 += 2 * nworkers) {
+        float acc[2] = {0.f, 0.f};
+        for (int base = lane * 8; base < p.H; base += kChunks * 256) {
+            uint4 v[2][kChunks];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                v[q] = base + q * 256 < p.H ? *(const uint4 *)(xr + base + q * 256) : make_uint4(0, 0, 0, 0);
+            for (int u = 0; u < 2; ++u) {
+                const int t = t0 + u;
+                const uint16_t *xr = p.x + (size_t)(t < p.T ? t : t0) * p.H;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < kChunks; ++q)
+                    v[u][q] = base + q * 256 < p.H ? *(const uint4 *)(xr + base + q * 256) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int q = 0; q < kChunks; ++q) {
                 const int c0 = base + q * 256;
                 if (c0 < p.H) {
                     const float4 g0 = *(const float4 *)(p.gate_w + c0);
                     const float4 g1 = *(const float4 *)(p.gate_w + c0 + 4);
-                    acc = fmaf(__uint_as_float(v[q].x << 16), g0.x, acc);
-                    acc = fmaf(__uint_as_float(v[q].x & 0xFFFF0000u), g0.y, acc);
-                    acc = fmaf(__uint_as_float(v[q].y << 16), g0.z, acc);
-                    acc = fmaf(__uint_as_float(v[q].y & 0xFFFF0000u), g0.w, acc);
-                    acc = fmaf(__uint_as_float(v[q].z << 16), g1.x, acc);
-                    acc = fmaf(__uint_as_float(v[q].z & 0xFFFF0000u), g1.y, acc);
-                    acc = fmaf(__uint_as_float(v[q].w << 16), g1.z, acc);
-                    acc = fmaf(__uint_as_float(v[q].w & 0xFFFF0000u), g1.w, acc);
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        acc[u] = fmaf(__uint_as_float(v[u][q].x << 16), g0.x, acc[u]);
+                        acc[u] = fmaf(__uint_as_float(v[u][q].x & 0xFFFF0000u), g0.y, acc[u]);
+                        acc[u] = fmaf(__uint_as_float(v[u][q].y << 16), g0.z, acc[u]);
+                        acc[u] = fmaf(__uint_as_float(v[u][q].y & 0xFFFF0000u), g0.w, acc[u]);
+                        acc[u] = fmaf(__uint_as_float(v[u][q].z << 16), g1.x, acc[u]);
+                        acc[u] = fmaf(__uint_as_float(v[u][q].z & 0xFFFF0000u), g1.y, acc[u]);
+                        acc[u] = fmaf(__uint_as_float(v[u][q].w << 16), g1.z, acc[u]);
+                        acc[u] = fmaf(__uint_as_float(v[u][q].w & 0xFFFF0000u), g1.w, acc[u]);
+                    }
                 }
             }
         }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-        if (lane == 0)
-            p.gate_out[t] = acc;
+        for (int u = 0; u < 2; ++u) {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                acc[u] += __shfl_xor_sync(0xFFFFFFFFu, acc[u], off);
+        }
+        if (lane == 0) {
+            p.gate_out[t0] = acc[0];
+            if (t0 + 1 < p.T)
+                p.gate_out[t0 + 1] = acc[1];
+        }
     }
 }
 

@@ -31,13 +31,19 @@ __device__ __forceinline__ float key_value(uint32_t key)
 
 // Lane j < k gets the j-th largest logit (my_val; a -0 logit as +0) and its
 // expert id (my_id; 0x7FFFFFFF and my_val = -inf where every remaining
-// logit is NaN); every lane gets the largest logit (top).  The selection
-// carries no per-lane value array: the owner lane marks its logit taken in
-// a bit mask, and the value is recovered from the winning key.
+// logit is NaN); every lane gets the largest logit (top).  The owner lane
+// marks its chosen logit in a bit mask, and the value is recovered from the
+// winning key.
 template <int NPL>
 __device__ __forceinline__ void warp_topk(const float (&v)[NPL], int E, int k, int lane, float &my_val, int &my_id,
                                           float &top)
 {
+    // order keys once; a chosen logit is masked through the taken bits (no
+    // write into the key array, which would need a dynamic index)
+    uint32_t key[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+        key[i] = i * 32 + lane < E ? order_key(v[i]) : 0u;
     uint32_t taken = 0u;   // bit i: logit i * 32 + lane already chosen
     top = 0.f;
     my_val = -CUDART_INF_F;
@@ -48,7 +54,7 @@ __device__ __forceinline__ void warp_topk(const float (&v)[NPL], int E, int k, i
         int bi = 0;
 #pragma unroll
         for (int i = 0; i < NPL; ++i) {
-            const uint32_t ki = i * 32 + lane < E && !((taken >> i) & 1u) ? order_key(v[i]) : 0u;
+            const uint32_t ki = (taken >> i) & 1u ? 0u : key[i];
             if (ki > bk) {
                 bk = ki;
                 bi = i;
