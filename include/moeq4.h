@@ -174,11 +174,12 @@ size_t moe_router_workspace_size(const moe_config_t *cfg, int T);
  * Router logits and the shared expert's gate logit.
  *   x [T, H] bf16, logits [T, E] fp32 (bias added when L->router_bias),
  *   gate_logit [T] fp32 = x . shared_gate (may be NULL; ignored without a
- *   shared expert).  fp32 accumulation.  For small T the reduction over H
- *   is cut into slices that run on separate SMs; their partial logits live
- *   in the caller's workspace ws (at least moe_router_workspace_size bytes,
- *   256-byte aligned; MOE_ERR_WORKSPACE if smaller) and are summed in slice
- *   order.
+ *   shared expert).  fp32 accumulation.  The caller's workspace ws (at
+ *   least moe_router_workspace_size bytes, 256-byte aligned;
+ *   MOE_ERR_WORKSPACE if smaller) receives the router weights split into
+ *   two bf16 matrices (hi = bf16(w), lo = bf16(w - hi); rewritten by every
+ *   call) and, for small T, the partial logits of the slices of H that run
+ *   on separate SMs, summed in slice order.
  * Source: the router of the Qwen3.6-35B-A3B layer the hipfire 0.4.3
  * benchmarks measure ("Qwen3.6-35B-A3B prefill on the R9700" table); the
  * pages give no formula, so logits = x Wr^T + bias is this library's reading.
