@@ -327,7 +327,7 @@ int run_expert_ffn(const moe_layer_t *L, const uint16_t *x, int T, const int32_t
         a.out = h;
         a.out_shared = h + (size_t)Tk * c.I;
         a.ldo = c.I;
-        CUDA_TRY(launch_grouped_gemm(a, 2, c.wfmt, gemm_tile_tokens(T, c.E, c.k), num_sms(), st), "gate/up GEMM");
+        CUDA_TRY(launch_grouped_gemm(a, 2, c.wfmt, gemm_tile_tokens(T, c.E, c.k, c.wfmt), num_sms(), st), "gate/up GEMM");
         g_launches += 1;
     }
     if (pass & 2) {

@@ -892,17 +892,22 @@ size_t gemm_smem_required(int nmat, int meta_bytes, int E_total)
     return a > b ? (a > c ? a : c) : (b > c ? b : c);
 }
 
-// Gate/up token tiles: 64 when experts average at most 64 rows, 192 when
-// they average at least 128 (one accumulator of 2 x 192 columns and two A
-// stages fill TMEM: half again the MMA work per dequantised k-step), else 128.
+// Gate/up token tiles: 64 when experts average at most 64 rows; when they
+// average at least 128, 192 (one accumulator of 2 x 192 columns and two A
+// stages fill TMEM: half again the MMA work per dequantised k-step), or 160
+// for Q4K super-blocks, whose heavier dequantisation gains more from a
+// third A stage than from the wider tile (measured: 4096 tokens 266 -> 257
+// us; int4-sym at 8192 tokens prefers 192, 397 vs 425 us); else 128.
 #ifndef MOEQ4_GU_TILE_MAX
 #define MOEQ4_GU_TILE_MAX 192
 #endif
-int gemm_tile_tokens(int T, int E, int k)
+int gemm_tile_tokens(int T, int E, int k, int wfmt)
 {
     if ((long long)T * k <= 64LL * E)
         return 64;
-    return MOEQ4_GU_TILE_MAX >= 192 && (long long)T * k >= 128LL * E ? 192 : 128;
+    if (MOEQ4_GU_TILE_MAX < 192 || (long long)T * k < 128LL * E)
+        return 128;
+    return wfmt == MOE_WFMT_Q4K ? 160 : 192;
 }
 
 // The down pass reads its token rows with TMA and has a single matrix, so
@@ -932,6 +937,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int tile_
     if (nmat == 2)
         return tile_tokens == 64    ? launch_fmt<MODE_GATE_UP, 64>(a, wfmt, num_sms, st)
                : tile_tokens == 192 ? launch_fmt<MODE_GATE_UP, 192>(a, wfmt, num_sms, st)
+               : tile_tokens == 160 ? launch_one<MODE_GATE_UP, MOE_WFMT_Q4K, 160>(a, num_sms, st)
                                     : launch_fmt<MODE_GATE_UP, 128>(a, wfmt, num_sms, st);
     return tile_tokens == 64    ? launch_fmt<MODE_DOWN, 64>(a, wfmt, num_sms, st)
            : tile_tokens == 128 ? launch_fmt<MODE_DOWN, 128>(a, wfmt, num_sms, st)

@@ -72,9 +72,8 @@ struct GemmArgs {
     int *status;                // [code, detail]
 };
 
-// Token-tile width of the gate/up GEMM: 64 when experts average at most 64
-// rows (T k <= 64 E), else 128.
-int gemm_tile_tokens(int T, int E, int k);
+// Token-tile width of the gate/up GEMM (64, 128, 160 or 192; see gemm.cu).
+int gemm_tile_tokens(int T, int E, int k, int wfmt);
 // Token-tile width of the down pass: 256 when experts average >= 128 rows, else as above.
 int gemm_down_tile_tokens(int T, int E, int k);
 cudaError_t launch_grouped_gemm(const GemmArgs &a, int nmat, int wfmt, int tile_tokens, int num_sms, cudaStream_t st);

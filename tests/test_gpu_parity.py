@@ -219,6 +219,8 @@ SMALL_LAYERS = [
     small_cfg("wide_down", T=300, H=256, E=8, k=2, I=640, has_shared=True, G=128, wr_std=0.03),
     # the same with Q4K super-blocks (12 k-steps)
     small_cfg("wide_down_q4k", T=200, H=512, E=4, k=2, I=768, G=256, wfmt=synth.WFMT_Q4K),
+    # Q4K experts averaging more than 128 rows: 160-token gate/up tiles with a ragged tail
+    small_cfg("q4k_wide_tiles", T=700, H=512, E=4, k=2, I=256, G=256, wfmt=synth.WFMT_Q4K, wr_std=0.03),
     # 1024 routed experts + shared: schedules over more experts than threads, eight router expert tiles
     small_cfg("many_experts", T=600, H=256, E=1024, k=4, I=128, has_shared=True, G=64, wr_std=0.05),
 ]
@@ -277,8 +279,8 @@ def test_fused_equals_composed_bitwise(dev, cfg):
     assert torch.equal(y.view(torch.int16), fused["y_bf16"].view(torch.int16))
 
 
-@pytest.mark.parametrize("cfg", [SMALL_LAYERS[5], SMALL_LAYERS[3], SMALL_LAYERS[1], SMALL_LAYERS[7], SMALL_LAYERS[8]],
-                         ids=lambda c: c.name)
+@pytest.mark.parametrize("cfg", [SMALL_LAYERS[5], SMALL_LAYERS[3], SMALL_LAYERS[1], SMALL_LAYERS[7], SMALL_LAYERS[8],
+                                 SMALL_LAYERS[10]], ids=lambda c: c.name)
 @pytest.mark.parametrize("ctas", [1, 3])
 def test_layer_on_few_ctas_is_bitwise_equal(dev, cfg, ctas, monkeypatch):
     """Each work unit is computed the same way whichever CTA takes it, so a
