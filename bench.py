@@ -529,26 +529,59 @@ def main():
     roofline, layer_roof = b.rooflines(ms, per_kernel_ms, touched)
 
     # ------------------------------------------------------------------ e2e
+    # Through the public call with host buffers: every step copies its input
+    # from pinned host memory and its result back to pinned host memory.  The
+    # steps are pipelined the way a serving loop runs them: the copies in and
+    # out go on their own streams, two device buffers each, so that step i's
+    # copies overlap the layer of its neighbours; the timed region runs from
+    # the first copy in to the last copy out.
     e2e = None
     if not args.profile:
         x_host = torch.from_numpy(np.ascontiguousarray(b.layer["x"]).view(np.int16)).pin_memory()
-        y_host = torch.empty((T, H), dtype=torch.int16).pin_memory()
-        x_in = torch.empty((T, H), dtype=torch.int16, device=dev)
-        y_out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        y_host = [torch.empty((T, H), dtype=torch.int16).pin_memory() for _ in range(2)]
+        x_in = [torch.empty((T, H), dtype=torch.int16, device=dev) for _ in range(2)]
+        y_out = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-        def e2e_step():
-            x_in.copy_(x_host, non_blocking=True)
-            b.call(b.packed, x_in, T, y_out, b.ws, b.nbytes, stream)
-            y_host.copy_(y_out.view(torch.int16), non_blocking=True)
+        def e2e_run(n):
+            ev = lambda: torch.cuda.Event(enable_timing=False)
+            start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            start.record(s_in)
+            comp_done, out_done = [], []
+            for i in range(n):
+                j = i % 2
+                if i >= 2:
+                    s_in.wait_event(comp_done[i - 2])   # x_in[j] is no longer read
+                with torch.cuda.stream(s_in):
+                    x_in[j].copy_(x_host, non_blocking=True)
+                e_in = ev()
+                e_in.record(s_in)
+                stream.wait_event(e_in)
+                if i >= 2:
+                    stream.wait_event(out_done[i - 2])   # y_out[j] has been copied out
+                b.call(b.packed, x_in[j], T, y_out[j], b.ws, b.nbytes, stream)
+                e_c = ev()
+                e_c.record(stream)
+                comp_done.append(e_c)
+                s_out.wait_event(e_c)
+                with torch.cuda.stream(s_out):
+                    y_host[j].copy_(y_out[j].view(torch.int16), non_blocking=True)
+                e_o = ev()
+                e_o.record(s_out)
+                out_done.append(e_o)
+            end.record(s_out)
+            end.synchronize()
+            return start.elapsed_time(end)
 
-        for _ in range(3):
-            e2e_step()
+        e2e_run(3)
         torch.cuda.synchronize(dev)
         barrier(world)
-        _, e_total = b.timed(e2e_step, args.steps)
+        e_total = e2e_run(args.steps)
+        torch.cuda.synchronize(dev)
         e_ms = max_over_ranks(e_total / args.steps, world, dev)
         e2e = {"value": world * T / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
-               "d2h_bytes_per_step": T * H * 2, "ms_per_step": e_ms}
+               "d2h_bytes_per_step": T * H * 2, "ms_per_step": e_ms,
+               "mode": "pipelined: copies in and out on their own streams overlap the layer (two buffers each)"}
 
     # ------------------------------------------------ other workloads (N = 1)
     extras = None
