@@ -58,10 +58,18 @@ __device__ unsigned long long g_dec_trace[4][16];
         if (blockIdx.x < 4 && threadIdx.x == 0)                       \
             g_dec_trace[blockIdx.x][(i)] = moeq4::globaltimer_ns();    \
     } while (0)
+// entries 7 .. 10: steps inside the routing phase; 15: warp 0's cycles
+// waiting for its staged down items
+#define DEC_CLK(v) const long long v = clock64()
+#define DEC_ACC(a, since) (a) += clock64() - (since)
+#define DEC_DECL(a) long long a = 0
 #else
 #define DEC_MARK(i) \
     do {            \
     } while (0)
+#define DEC_CLK(v)
+#define DEC_ACC(a, since)
+#define DEC_DECL(a)
 #endif
 
 namespace moeq4 {
@@ -74,6 +82,10 @@ constexpr int kN = kDecodeMaxT;
 constexpr int kFeat = 16;   // features per gate/up unit: 16 gate rows + 16 up rows, one per lane
 constexpr int kCols = 16;   // output columns per down unit
 constexpr int kCodeBuf = 2048; // staged codes of one warp item
+// row stride (floats) of the 16-wide rows of the gate/up partials and the
+// down outputs in shared memory: 20 puts the 4 column pairs a warp's MMA
+// fragment writes on distinct banks
+constexpr int kRedLd = 20;
 // bytes of one row's scale entry: bf16 scale (int4-sym), bf16 scale and
 // minimum (int4-asym), 16-byte super-block header (Q4K)
 __host__ __device__ constexpr int meta_row_bytes(int wfmt)
@@ -98,44 +110,38 @@ __device__ __forceinline__ unsigned ld_relaxed(const unsigned *p)
     return v;
 }
 
-__device__ __forceinline__ void st_release(unsigned *p, unsigned v)
-{
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Grid barrier over all CTAs of a cooperative launch.  bar[0] counts
-// arrivals (back to 0 after every barrier), bar[1] is the generation,
-// bar[2] the abort flag.  Waits are bounded by the workspace's wait budget
-// (status word 20, microseconds; 0 = 2 s): on timeout the CTA records
-// MOE_ERR_TIMEOUT, raises the abort flag (so the others stop waiting) and
-// the caller returns.  Returns false when the kernel must stop.
+// Grid barrier over all CTAs of a cooperative launch.  bar[0] is the
+// arrival word: CTA 0 adds 2^31 - (n - 1) and every other CTA adds 1, so
+// its top bit flips exactly when the last of the n CTAs arrives and its low
+// bits come back to where they were (no reset step, and one atomic on the
+// critical path); a CTA waits for the flip relative to the word it saw when
+// it arrived.  bar[2] is the abort flag.  Waits are bounded by wait_ns (the
+// workspace's wait budget, status word 20, microseconds; 0 = 2 s): on
+// timeout the CTA records MOE_ERR_TIMEOUT, raises the abort flag (so the
+// others stop waiting) and the caller returns.  Returns false when the
+// kernel must stop.  Only thread 0's skip and wait_ns are read.
 //
 // Test knob (status word 21): when it holds c > 0, CTA c - 1 waits at the
-// first barrier without arriving, so that every CTA's wait runs out of its
-// budget (the way a lost arrival would); the kernel then returns with
-// MOE_ERR_TIMEOUT and a usable context.
-__device__ bool grid_sync(unsigned *bar, int *status, int where, int *s_flag)
+// first barrier without arriving (skip), so that every CTA's wait runs out
+// of its budget (the way a lost arrival would); the kernel then returns
+// with MOE_ERR_TIMEOUT and a usable context.
+__device__ bool grid_sync(unsigned *bar, int *status, int where, int *s_flag, bool skip, uint64_t wait_ns)
 {
     __syncthreads();
     if (threadIdx.x == 0) {
         int ok = 1;
-        __threadfence();
-        const unsigned gen = ld_acquire(bar + 1);   // read before arriving: it cannot move until we do
-        const bool skip = where == 91 && test_knob_hits_this_cta(status);
-        const unsigned prev = skip ? 0u : atomicAdd(bar, 1u);
-        if (!skip && prev == gridDim.x - 1) {
-            atomicExch(bar, 0u);
-            __threadfence();
-            st_release(bar + 1, gen + 1);
-        } else {
-            const uint64_t t0 = globaltimer_ns(), limit = wait_limit_ns(status);
+        __threadfence();   // this CTA's global writes before its arrival
+        const unsigned add = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1) : 1u;
+        const unsigned seen = skip ? ld_acquire(bar) : atomicAdd(bar, add);
+        if (skip || (((seen + add) ^ seen) & 0x80000000u) == 0) {   // not the last arrival
+            const uint64_t t0 = globaltimer_ns();
             uint32_t spins = 0;
-            while (ld_acquire(bar + 1) == gen) {
+            while (((ld_acquire(bar) ^ seen) & 0x80000000u) == 0) {
                 if (ld_relaxed(bar + 2)) {
                     ok = 0;
                     break;
                 }
-                if ((++spins & 63u) == 0 && globaltimer_ns() - t0 > limit) {
+                if ((++spins & 63u) == 0 && globaltimer_ns() - t0 > wait_ns) {
                     atomicExch(bar + 2, 1u);
                     record_error(status, MOE_ERR_TIMEOUT, where);
                     ok = 0;
@@ -251,6 +257,49 @@ __device__ __forceinline__ void cp_async_wait_upto(int n)
         cp_async_wait_group<0>();
 }
 
+// Rows 0 .. n - 1 of a row-major bf16 matrix (row length len, a multiple
+// of 32) into shared rows of stride ld elements, then a zero row at shared
+// row zrow: 16-byte cp.async (L2 only: the rows may have been written by
+// other CTAs of this launch), all issued at once, as one commit group.
+__device__ __forceinline__ void issue_rows(const uint16_t *src, int len, int n, int zrow, uint32_t dst, int ld,
+                                           int tid)
+{
+    const int per_row = len / 8;
+    for (int i = tid; i < (n + 1) * per_row; i += kThreads) {
+        const int r = i / per_row, kk = (i % per_row) * 8;
+        const bool real = r < n;
+        cp_async_16(dst + 2u * (uint32_t)((real ? r : zrow) * ld + kk), real ? src + (size_t)r * len + kk : src,
+                    real ? 16u : 0u);
+    }
+    cp_async_commit();
+}
+
+// The fp32 sum of every 32-element chunk of shared rows 0 .. n - 1 (stride
+// ld) into sums[row][chunk].  Thread i reads 16 bytes (8 elements, summed
+// in order; a warp reads consecutive bytes); the 4 threads of a chunk are
+// consecutive lanes and add their parts with two shuffles.  The loop runs
+// in whole warps so every shuffle is complete.
+__device__ __forceinline__ void row_sums(const uint16_t *rows, int len, int n, int ld, float *sums, int tid)
+{
+    const int per_row = len / 8, nch = len / 32;
+    const int rounded = (n * per_row + 31) & ~31;
+    for (int i = tid; i < rounded; i += kThreads) {
+        const int r = i / per_row, kk = (i % per_row) * 8;
+        const uint4 v = r < n ? *(const uint4 *)(rows + (size_t)r * ld + kk) : make_uint4(0, 0, 0, 0);
+        float s = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t w = word_of(v, q);
+            s += __uint_as_float(w << 16);
+            s += __uint_as_float(w & 0xFFFF0000u);
+        }
+        s += __shfl_xor_sync(0xFFFFFFFFu, s, 1);
+        s += __shfl_xor_sync(0xFFFFFFFFu, s, 2);
+        if (r < n && (i & 3) == 0)
+            sums[(size_t)r * nch + kk / 32] = s;
+    }
+}
+
 // One 32-element chunk of a 16-row tile against an 8-column B operand: the
 // two k16 slices of the chunk.  lo / hi: this lane's codes of rows gid and
 // gid + 8; brow: this lane's B column (a row of 16-bit values in shared
@@ -272,45 +321,65 @@ __device__ __forceinline__ void chunk_mma(float (&d)[4], const uint4 &lo, const 
 
 DecodeSmem decode_smem_layout(int T, int k, int H, int I, int has_shared, int wfmt)
 {
-    DecodeSmem s{};
     const int tk = T * k;
     const int np = tk + (has_shared ? T : 0);
-    const int nd = tk + (has_shared ? 1 : 0);
-    size_t off = 0;
-    auto take = [&](size_t bytes) {
-        const size_t o = off;
-        off += (bytes + 15) & ~(size_t)15;
-        return (int)o;
-    };
-    // phases A-C: x as bf16 rows (kN + 1, the last one zero) and its chunk
-    // sums; phase D reuses the space for h (np + 1 rows) and its chunk sums
-    const size_t xbytes = sizeof(uint16_t) * (size_t)(kN + 1) * (H + 8) + sizeof(float) * (size_t)kN * (H / 32) + 16;
-    const size_t hbytes = sizeof(uint16_t) * (size_t)(np + 1) * (I + 8) + sizeof(float) * (size_t)np * (I / 32) + 16;
-    s.big = take(xbytes > hbytes ? xbytes : hbytes);
-    s.sums = 0;   // placed inside big by the kernel
-    // gate/up partials [warp][matrix][row][token]; reused for the down outputs [pair][column]
-    const size_t red = (size_t)kWarps * 2 * 16 * kN > (size_t)np * kCols ? (size_t)kWarps * 2 * 16 * kN
-                                                                         : (size_t)np * kCols;
-    s.red = take(sizeof(float) * red);
-    s.ids = take(sizeof(int) * (tk > 0 ? tk : 1));
-    s.w = take(sizeof(float) * np);
-    s.pidx = take(sizeof(int) * (tk > 0 ? tk : 1));
-    s.pair_tok = take(sizeof(int) * np);
-    s.pair_w = take(sizeof(float) * np);
-    s.slot_e = take(sizeof(int) * nd);
-    s.slot_base = take(sizeof(int) * nd);
-    s.slot_cnt = take(sizeof(int) * nd);
-    s.bitmap = take(sizeof(uint32_t) * 32);
-    s.wprefix = take(sizeof(int) * 33);
-    s.flag = take(sizeof(int) * 4);
-    // the warps' staging rings take what is left, 2 to 4 items deep (a
-    // shape whose 2-deep rings do not fit is refused by the caller)
+    const int nd = tk + (has_shared ? 1 : 0);   // slots of at most 8 pairs: at most one per pair
+    const int ntok = tk < kN ? (tk > 0 ? tk : 1) : kN;   // pairs (MMA columns) of one slot
+    auto up16 = [](size_t b) { return (b + 15) & ~(size_t)15; };
     const size_t ring = (size_t)kWarps * item_buf_bytes(wfmt);
-    const size_t left = off < kDecodeSmemLimit ? kDecodeSmemLimit - off : 0;
-    s.nstage = left / ring >= 4 ? 4 : left / ring >= 3 ? 3 : 2;
-    s.cbuf = take(ring * s.nstage);
-    s.bytes = off;
-    return s;
+    auto build = [&](int nred) {
+        DecodeSmem s{};
+        size_t off = 0;
+        auto take = [&](size_t bytes) {
+            const size_t o = off;
+            off += up16(bytes);
+            return (int)o;
+        };
+        // phases A-C: x as bf16 rows (kN + 1, the last one zero) and its
+        // chunk sums, then nred buffers of gate/up partials
+        // [warp][matrix][pair < ntok][row] (the router's per-warp sums in
+        // phase A use the first); phase D reuses the space for h (np + 1
+        // rows), its chunk sums and the down outputs [pair][column]
+        const size_t xbytes = up16(sizeof(uint16_t) * (size_t)(kN + 1) * (H + 8) + sizeof(float) * (size_t)kN * (H / 32));
+        const size_t hbytes = up16(sizeof(uint16_t) * (size_t)(np + 1) * (I + 8) + sizeof(float) * (size_t)np * (I / 32));
+        size_t redc = sizeof(float) * (size_t)kWarps * 2 * ntok * kRedLd;
+        if ((size_t)nred * redc < sizeof(float) * kWarps * kN)
+            redc = sizeof(float) * kWarps * kN;
+        const size_t outd = up16(sizeof(float) * (size_t)np * kRedLd);
+        s.big = take(xbytes + nred * redc > hbytes + outd ? xbytes + nred * redc : hbytes + outd);
+        s.sums = 0;   // placed inside big by the kernel
+        s.red = s.big + (int)xbytes;
+        s.nred = nred;
+        s.ntok = ntok;
+        s.ored = s.big + (int)hbytes;
+        s.ids = take(sizeof(int) * (tk > 0 ? tk : 1));
+        s.w = take(sizeof(float) * np);
+        s.pidx = take(sizeof(int) * (tk > 0 ? tk : 1));
+        s.pair_tok = take(sizeof(int) * np);
+        s.pair_w = take(sizeof(float) * np);
+        s.slot_e = take(sizeof(int) * nd);
+        s.slot_base = take(sizeof(int) * nd);
+        s.slot_cnt = take(sizeof(int) * nd);
+        // per chosen expert (rank d): its pairs per token (one byte per
+        // token, 4 tokens a word), its expert id and its first pair
+        s.tcount = take(sizeof(uint32_t) * 2 * (tk > 0 ? tk : 1));
+        s.dexp = take(sizeof(int) * (tk > 0 ? tk : 1));
+        s.dbase = take(sizeof(int) * (tk > 0 ? tk : 1));
+        s.bitmap = take(sizeof(uint32_t) * 32);
+        s.wprefix = take(sizeof(int) * 33);
+        s.flag = take(sizeof(int) * 4);
+        // the warps' staging rings take what is left, 2 to 4 items deep (a
+        // shape whose 2-deep rings do not fit is refused by the caller)
+        const size_t left = off < kDecodeSmemLimit ? kDecodeSmemLimit - off : 0;
+        s.nstage = left / ring >= 4 ? 4 : left / ring >= 3 ? 3 : 2;
+        s.cbuf = take(ring * s.nstage);
+        s.bytes = off;
+        return s;
+    };
+    // two partials buffers (one block barrier per gate/up unit) where they
+    // fit beside 2-deep rings, else one (two barriers per unit)
+    const DecodeSmem two = build(2);
+    return two.bytes <= kDecodeSmemLimit ? two : build(1);
 }
 
 namespace {
@@ -408,6 +477,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     int *slot_e = (int *)(smem + L.slot_e);
     int *slot_base = (int *)(smem + L.slot_base);
     int *slot_cnt = (int *)(smem + L.slot_cnt);
+    uint32_t *tcount = (uint32_t *)(smem + L.tcount);
+    int *dexp = (int *)(smem + L.dexp);
+    int *dbase = (int *)(smem + L.dbase);
     uint32_t *bitmap = (uint32_t *)(smem + L.bitmap);
     int *wprefix = (int *)(smem + L.wprefix);
     int *flag = (int *)(smem + L.flag);
@@ -432,6 +504,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     // the abort flag of a previous launch, and this warp's first router row,
     // are requested before anything else so that their latencies overlap
     const unsigned aborted = ld_relaxed(A.bar + 2);
+    // rows t < T of x, then the zero row kN (rows T .. kN - 1 are never read)
+    issue_rows(A.x, H, T, kN, smem_u32(xb), XS, tid);
+    bool knob_skip = false;   // thread 0's barrier inputs, read early for the same reason
+    uint64_t wait_ns = 0;
+    if (tid == 0) {
+        knob_skip = test_knob_hits_this_cta(A.status);
+        wait_ns = wait_limit_ns(A.status);
+    }
     const int rows = E + (A.has_shared ? 1 : 0);
     const int e_first = blockIdx.x + gridDim.x * warp;
     float4 wv[16];
@@ -445,6 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     }
     // a previous launch on this workspace gave up in a barrier: stop before touching it
     if (aborted) {
+        cp_async_wait_group<0>();
         if (blockIdx.x == 0 && tid == 0)
             record_error(A.status, MOE_ERR_TIMEOUT, 90);
         return;
@@ -452,22 +533,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     DEC_MARK(0);
     if (tid < 32)
         bitmap[tid] = 0;
+    for (int i = tid; i < 2 * A.T * A.k; i += kThreads)
+        tcount[i] = 0;
 
     // ------------------------------------------------ A: x -> smem, router
     {
-        for (int i = tid; i < (kN + 1) * (H / 8); i += kThreads) {
-            const int t = i / (H / 8), kk = (i % (H / 8)) * 8;
-            const uint4 v = t < T ? *(const uint4 *)(A.x + (size_t)t * H + kk) : make_uint4(0, 0, 0, 0);
-            *(uint4 *)(xb + (size_t)t * XS + kk) = v;
-        }
+        cp_async_wait_group<0>();
         __syncthreads();
-        for (int i = tid; i < kN * nchH; i += kThreads) {
-            const uint16_t *c = xb + (size_t)(i / nchH) * XS + (i % nchH) * 32;
-            float s = 0.f;
-            for (int q = 0; q < 32; ++q)
-                s += __uint_as_float((uint32_t)c[q] << 16);
-            xsum[i] = s;
-        }
+        row_sums(xb, H, T, XS, xsum, tid);   // read in phase C, after two more block barriers
         // one warp per router row (and the shared gate vector); a lane holds
         // 16 float4 of a 2048-wide slice of the row, loaded before any use
         float *racc = red + warp * kN;
@@ -481,26 +554,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
                         wv[q] = kk < H ? __ldg((const float4 *)(wrow + kk)) : make_float4(0.f, 0.f, 0.f, 0.f);
                     }
                 }
-                for (int t = 0; t < T; ++t) {
-                    const uint16_t *xt = xb + (size_t)t * XS;
-                    float a0 = 0.f, a1 = 0.f;
+                // two tokens against the slice at a time: 4 independent
+                // chains, each summed in the same order as for one token
+                for (int t0 = 0; t0 < T; t0 += 2) {
+                    float a0[2] = {0.f, 0.f}, a1[2] = {0.f, 0.f};
+                    const bool two = t0 + 1 < T;
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
                         const int kk = seg + (q * 32 + lane) * 4;
                         if (kk < H) {
-                            const uint2 xv = *(const uint2 *)(xt + kk);
-                            a0 = fmaf(wv[q].x, __uint_as_float(xv.x << 16), a0);
-                            a1 = fmaf(wv[q].y, __uint_as_float(xv.x & 0xFFFF0000u), a1);
-                            a0 = fmaf(wv[q].z, __uint_as_float(xv.y << 16), a0);
-                            a1 = fmaf(wv[q].w, __uint_as_float(xv.y & 0xFFFF0000u), a1);
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                if (u == 0 || two) {
+                                    const uint2 xv = *(const uint2 *)(xb + (size_t)(t0 + u) * XS + kk);
+                                    a0[u] = fmaf(wv[q].x, __uint_as_float(xv.x << 16), a0[u]);
+                                    a1[u] = fmaf(wv[q].y, __uint_as_float(xv.x & 0xFFFF0000u), a1[u]);
+                                    a0[u] = fmaf(wv[q].z, __uint_as_float(xv.y << 16), a0[u]);
+                                    a1[u] = fmaf(wv[q].w, __uint_as_float(xv.y & 0xFFFF0000u), a1[u]);
+                                }
+                            }
                         }
                     }
-                    float v = a0 + a1;
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1)
-                        v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-                    if (lane == 0)
-                        racc[t] = seg == 0 ? v : racc[t] + v;
+                    for (int u = 0; u < 2; ++u) {
+                        float v = a0[u] + a1[u];
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1)
+                            v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+                        if (lane == 0 && (u == 0 || two))
+                            racc[t0 + u] = seg == 0 ? v : racc[t0 + u] + v;
+                    }
                 }
             }
             __syncwarp();
@@ -515,13 +598,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
         }
     }
     DEC_MARK(1);
-    if (!grid_sync(A.bar, A.status, 91, flag))
+    if (!grid_sync(A.bar, A.status, 91, flag, knob_skip, wait_ns))
         return;
     DEC_MARK(2);
 
     // ------------------------------------------------ B: routing, pair lists
     if (warp < T) {
         const int t = warp;
+        // the shared expert's gate logit is requested with the logits
+        const float glog = lane == 0 && A.has_shared ? __ldcg(A.gate_logit + t) : 0.f;
         int my_id = 0;
         float my_w = 0.f;
         if (A.override_ids) {
@@ -547,8 +632,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
             w_s[t * k + lane] = my_w;
         }
         if (lane == 0 && A.has_shared)
-            w_s[tk + t] = 1.0f / (1.0f + expf(-__ldcg(A.gate_logit + t)));
+            w_s[tk + t] = 1.0f / (1.0f + expf(-glog));
     }
+    DEC_MARK(7);
     __syncthreads();
     if (blockIdx.x == 0) {
         for (int i = tid; i < tk; i += kThreads) {
@@ -573,28 +659,73 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
             wprefix[32] = incl;
     }
     __syncthreads();
-    // pair p of (t, j): pairs ordered by expert, then by t k + j
+    DEC_MARK(8);
+    // pair p of (t, j): pairs ordered by expert, then by t k + j.  Chosen
+    // expert d (its rank among the chosen ones) counts its pairs per token;
+    // its first pair is the sum of the counts of the experts below it, and
+    // a pair's rank among its expert's pairs is that expert's count in the
+    // tokens before t plus its earlier places in token t (a token lists an
+    // expert twice only through given or replaced ids).  Each expert's
+    // pairs are then cut into slots of at most 8 (the columns of one MMA).
+    auto rank_of = [&](int e) { return wprefix[e >> 5] + __popc(bitmap[e >> 5] & ((1u << (e & 31)) - 1u)); };
     for (int i = tid; i < tk; i += kThreads) {
-        const int e = ids_s[i];
-        int below = 0, before = 0, same = 0;
-        for (int i2 = 0; i2 < tk; ++i2) {
-            const int e2 = ids_s[i2];
-            below += e2 < e;
-            same += e2 == e;
-            before += (e2 == e) & (i2 < i);
+        const int e = ids_s[i], t = i / k, d = rank_of(e);
+        atomicAdd(&tcount[2 * d + (t >> 2)], 1u << (8 * (t & 3)));
+        dexp[d] = e;
+    }
+    __syncthreads();
+    DEC_MARK(9);
+    if (warp == 0) {
+        const int nchosen = wprefix[32];
+        int carry = 0;   // (pairs << 16) | slots of the experts so far
+        for (int d0 = 0; d0 < nchosen; d0 += 32) {
+            const int d = d0 + lane;
+            int c = 0;
+            if (d < nchosen) {
+                const uint64_t v = (uint64_t)tcount[2 * d] | (uint64_t)tcount[2 * d + 1] << 32;
+#pragma unroll
+                for (int b = 0; b < kN; ++b)
+                    c += (int)((v >> (8 * b)) & 0xFFu);
+            }
+            const int mine = (c << 16) | ((c + 7) >> 3);   // both sums stay below 2^16
+            int incl = mine;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o)
+                    incl += n;
+            }
+            if (d < nchosen) {
+                const int excl = carry + incl - mine;
+                const int base = excl >> 16, sl0 = excl & 0xFFFF, e = dexp[d];
+                dbase[d] = base;
+                for (int q = 0; 8 * q < c; ++q) {
+                    slot_e[sl0 + q] = e;
+                    slot_base[sl0 + q] = base + 8 * q;
+                    slot_cnt[sl0 + q] = c - 8 * q < 8 ? c - 8 * q : 8;
+                }
+            }
+            carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
         }
-        const int p = below + before;
-        const int d = wprefix[e >> 5] + __popc(bitmap[e >> 5] & ((1u << (e & 31)) - 1u));
-        pair_tok[p] = i / k;
+        if (lane == 0)
+            flag[2] = carry & 0xFFFF;   // routed slots
+    }
+    __syncthreads();
+    DEC_MARK(10);
+    const int nd_routed = flag[2];
+    for (int i = tid; i < tk; i += kThreads) {
+        const int e = ids_s[i], t = i / k, j = i % k, d = rank_of(e);
+        const uint64_t v = (uint64_t)tcount[2 * d] | (uint64_t)tcount[2 * d + 1] << 32;
+        int before = 0;
+        for (int t2 = 0; t2 < t; ++t2)
+            before += (int)((v >> (8 * t2)) & 0xFFu);
+        for (int j2 = 0; j2 < j; ++j2)
+            before += ids_s[t * k + j2] == e;
+        const int p = dbase[d] + before;
+        pair_tok[p] = t;
         pair_w[p] = w_s[i];
         pidx[i] = p;
-        if (before == 0) {
-            slot_e[d] = e;
-            slot_base[d] = below;
-            slot_cnt[d] = same;
-        }
     }
-    const int nd_routed = wprefix[32];
     if (A.has_shared) {
         for (int t = tid; t < T; t += kThreads) {
             pair_tok[tk + t] = t;
@@ -632,6 +763,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
         for (int it2 = 0; it2 < NS - 1; ++it2)
             stage(it2);
         float acc[2][4];
+        int ru = 0;   // units reduced so far: picks the partials buffer
         for (int it = 0; it < nitems; ++it) {
             const int u = unit_of(it), pass = it % npass;
             const int d = u / per_slot, f0 = (u % per_slot) * kFeat;
@@ -651,10 +783,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
             cp_async_wait_upto(NS - 1);   // item it's copies have landed
             __syncwarp();
             const uint8_t *buf = mybuf + (it % NS) * kIB;
+            // the 4 chunks are independent MMA chains: unrolled so that they
+            // overlap; a chunk past the end reads a valid one and is not added
+#pragma unroll
             for (int n = 0; n < 4; ++n) {
-                const int j = pass * 4 * kWarps + warp + kWarps * n;
-                if (j >= nchH)
-                    break;
+                const int jr = pass * 4 * kWarps + warp + kWarps * n;
+                const bool valid = jr < nchH;
+                const int j = valid ? jr : nchH - 1;
                 float cs[2][2][2];   // [matrix][row lo/hi][a, b]
 #pragma unroll
                 for (int m = 0; m < 2; ++m) {
@@ -676,37 +811,49 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
                     for (int v = 0; v < 4; ++v) {
                         const float sx = (v & 1) ? sB : sA;
                         const float a = cs[m][v >> 1][0], b = cs[m][v >> 1][1];
-                        acc[m][v] = fmaf(a, fmaf(-kOff, sx, dd[v]), fmaf(b, sx, acc[m][v]));
+                        const float nv = fmaf(a, fmaf(-kOff, sx, dd[v]), fmaf(b, sx, acc[m][v]));
+                        acc[m][v] = valid ? nv : acc[m][v];
                     }
                 }
             }
             __syncwarp();
             if (pass == npass - 1) {
-                // the unit is complete in every warp: gate and up summed over the warps, in order
+                // the unit is complete in every warp: gate and up summed over
+                // the warps, in order.  The partials alternate between two
+                // buffers: a buffer is written again two units later, after a
+                // block barrier that its readers pass only once they are done,
+                // so one barrier per unit suffices and the other warps go on
+                // to the next unit while the sums are formed.
+                float *rb = red + (size_t)(ru & (L.nred - 1)) * kWarps * 2 * L.ntok * kRedLd;
+                ++ru;
+                if (L.nred == 1)
+                    __syncthreads();   // the previous unit's sums are formed
 #pragma unroll
                 for (int m = 0; m < 2; ++m)
 #pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        red[((warp * 2 + m) * 16 + gid + 8 * (v >> 1)) * kN + 2 * tid4 + (v & 1)] = acc[m][v];
+                    for (int v = 0; v < 4; ++v) {
+                        const int nn = 2 * tid4 + (v & 1);
+                        if (nn < cnt)
+                            rb[((warp * 2 + m) * L.ntok + nn) * kRedLd + gid + 8 * (v >> 1)] = acc[m][v];
+                    }
                 __syncthreads();
                 if (tid < kFeat * cnt) {
                     const int nn = tid / kFeat, f = tid % kFeat;
                     float g = 0.f, uu = 0.f;
                     for (int w = 0; w < kWarps; ++w) {
-                        g += red[((w * 2 + 0) * 16 + f) * kN + nn];
-                        uu += red[((w * 2 + 1) * 16 + f) * kN + nn];
+                        g += rb[((w * 2 + 0) * L.ntok + nn) * kRedLd + f];
+                        uu += rb[((w * 2 + 1) * L.ntok + nn) * kRedLd + f];
                     }
                     const float hv = g / (1.0f + expf(-g)) * uu;
                     A.h[(size_t)(base + nn) * I + f0 + f] = (uint16_t)(pack_bf16x2(hv, 0.f) & 0xFFFFu);
                 }
-                __syncthreads();
             }
         }
         cp_async_wait_group<0>();
         __syncwarp();
     }
     DEC_MARK(4);
-    if (!grid_sync(A.bar, A.status, 92, flag))
+    if (!grid_sync(A.bar, A.status, 92, flag, false, wait_ns))
         return;
     DEC_MARK(5);
 
@@ -716,36 +863,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
         const int HS = I + 8;
         uint16_t *hb = (uint16_t *)(smem + L.big);
         float *hsum = (float *)(hb + (size_t)(NP + 1) * HS);
-        for (int i = tid; i < (NP + 1) * (I / 8); i += kThreads) {
-            const int p = i / (I / 8), kk = (i % (I / 8)) * 8;
-            const uint4 v = p < NP ? __ldcg((const uint4 *)(A.h + (size_t)p * I + kk)) : make_uint4(0, 0, 0, 0);
-            *(uint4 *)(hb + (size_t)p * HS + kk) = v;
-        }
-        __syncthreads();
-        for (int i = tid; i < NP * nchI; i += kThreads) {
-            const uint16_t *c = hb + (size_t)(i / nchI) * HS + (i % nchI) * 32;
-            float s = 0.f;
-            for (int q = 0; q < 32; ++q)
-                s += __uint_as_float((uint32_t)c[q] << 16);
-            hsum[i] = s;
-        }
-        __syncthreads();
+        issue_rows(A.h, I, NP, NP, smem_u32(hb), HS, tid);
         const int gsh = WFMT == MOE_WFMT_Q4K ? 8 : gshift;
         const int nparts = (nchI + 7) / 8;
-        float *o_s = red;   // [pair][column]
+        float *o_s = (float *)(smem + L.ored);   // [pair][column]
         // this warp's slots: d = warp + kWarps i; items (slot, part)
         const int nslots = Nd > warp ? (Nd - 1 - warp) / kWarps + 1 : 0;
         const int nitems = nslots * nparts;
+        auto stage_for = [&](int c0, int it2) {
+            if (it2 < nitems)
+                dn_stage<WFMT>(A, slot_e[warp + kWarps * (it2 / nparts)], c0, it2 % nparts, nchI, gsh, lane,
+                               mybuf_s + (it2 % NS) * kIB);
+            cp_async_commit();
+        };
+        // the first column block's weights are requested before h is waited for
+        const int c_first = (int)blockIdx.x * kCols;
+        for (int it2 = 0; it2 < NS - 1; ++it2)
+            stage_for(c_first < H ? c_first : 0, c_first < H ? it2 : nitems);
+        cp_async_wait_upto(NS - 1);   // h (the oldest group) has landed
+        __syncthreads();
+        row_sums(hb, I, NP, HS, hsum, tid);
+        __syncthreads();
+        DEC_DECL(tdw);
         for (int u = blockIdx.x; u < H / kCols; u += gridDim.x) {
             const int c0 = u * kCols;
-            auto stage = [&](int it2) {
-                if (it2 < nitems)
-                    dn_stage<WFMT>(A, slot_e[warp + kWarps * (it2 / nparts)], c0, it2 % nparts, nchI, gsh, lane,
-                                   mybuf_s + (it2 % NS) * kIB);
-                cp_async_commit();
-            };
-            for (int it2 = 0; it2 < NS - 1; ++it2)
-                stage(it2);
+            auto stage = [&](int it2) { stage_for(c0, it2); };
+            if (u != (int)blockIdx.x)
+                for (int it2 = 0; it2 < NS - 1; ++it2)
+                    stage(it2);
             float acc[4];
             for (int it = 0; it < nitems; ++it) {
                 const int d = warp + kWarps * (it / nparts), q = it % nparts;
@@ -759,13 +904,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
                 const int prow = gid < cnt ? base + gid : NP;
                 const int pA = 2 * tid4 < cnt ? base + 2 * tid4 : -1;
                 const int pB = 2 * tid4 + 1 < cnt ? base + 2 * tid4 + 1 : -1;
+                DEC_CLK(c0);
                 cp_async_wait_upto(NS - 1);
                 __syncwarp();
+                DEC_ACC(tdw, c0);
                 const uint8_t *buf = mybuf + (it % NS) * kIB;
+                // independent chunks, partly unrolled as in the gate/up loop
+#pragma unroll 4
                 for (int n = 0; n < 8; ++n) {
-                    const int j = 8 * q + n;
-                    if (j >= nchI)
-                        break;
+                    const int jr = 8 * q + n;
+                    const bool valid = jr < nchI;
+                    const int j = valid ? jr : nchI - 1;
                     float clo_a, clo_b, chi_a, chi_b;
                     const uint8_t *mrow = buf + kCodeBuf + (n * 16 + gid) * kMB;
                     staged_coeffs<WFMT>(mrow, j * 32, clo_a, clo_b);
@@ -780,7 +929,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
                     for (int v = 0; v < 4; ++v) {
                         const float sx = (v & 1) ? sB : sA;
                         const float a = (v >> 1) ? chi_a : clo_a, b = (v >> 1) ? chi_b : clo_b;
-                        acc[v] = fmaf(a, fmaf(-kOff, sx, dd[v]), fmaf(b, sx, acc[v]));
+                        const float nv = fmaf(a, fmaf(-kOff, sx, dd[v]), fmaf(b, sx, acc[v]));
+                        acc[v] = valid ? nv : acc[v];
                     }
                 }
                 __syncwarp();
@@ -790,7 +940,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
                     for (int v = 0; v < 4; ++v) {
                         const int nn = 2 * tid4 + (v & 1);
                         if (nn < cnt)
-                            o_s[(base + nn) * kCols + gid + 8 * (v >> 1)] = acc[v];
+                            o_s[(base + nn) * kRedLd + gid + 8 * (v >> 1)] = acc[v];
                     }
                 }
             }
@@ -801,13 +951,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
                 const int t = tid / kCols, c2 = tid % kCols;
                 float y = 0.f;
                 for (int jj = 0; jj < k; ++jj)
-                    y = fmaf(w_s[t * k + jj], o_s[pidx[t * k + jj] * kCols + c2], y);
+                    y = fmaf(w_s[t * k + jj], o_s[pidx[t * k + jj] * kRedLd + c2], y);
                 if (A.has_shared)
-                    y = fmaf(w_s[tk + t], o_s[(tk + t) * kCols + c2], y);
+                    y = fmaf(w_s[tk + t], o_s[(tk + t) * kRedLd + c2], y);
                 A.y[(size_t)t * H + c0 + c2] = (uint16_t)(pack_bf16x2(y, 0.f) & 0xFFFFu);
             }
             __syncthreads();
         }
+#ifdef MOEQ4_TRACE
+        if (blockIdx.x < 4 && threadIdx.x == 0)
+            g_dec_trace[blockIdx.x][15] = (unsigned long long)tdw;
+#endif
     }
     DEC_MARK(6);
 }

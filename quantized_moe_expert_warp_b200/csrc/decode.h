@@ -34,7 +34,10 @@ struct DecodeArgs {
 
 // Byte offsets of the decode kernel's dynamic shared memory.
 struct DecodeSmem {
-    int big, sums, red, cbuf, ids, w, pidx, pair_tok, pair_w, slot_e, slot_base, slot_cnt, bitmap, wprefix, flag;
+    int big, sums, red, ored, cbuf, ids, w, pidx, pair_tok, pair_w, slot_e, slot_base, slot_cnt, tcount, dexp, dbase,
+        bitmap, wprefix, flag;
+    int nred;     // gate/up partials buffers (1 or 2)
+    int ntok;     // pairs (MMA columns) a slot holds at most: min(8, T k)
     int nstage;   // depth of each warp's staging ring
     size_t bytes;
 };

@@ -11,7 +11,7 @@ import pytest
 
 import oracle
 import synth
-from gpu_util import bf16_to_f32, check_close, compare_layer
+from gpu_util import bf16_to_f32, check_close, compare_layer, run_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -110,6 +110,24 @@ def test_decode_with_oracle_routing(dev):
     check_close(got["y"], ref["y"], cfg.name)
 
 
+def test_decode_duplicate_ids_cut_into_slots(dev):
+    """A token may list an expert more than once (given ids, or NaN logits
+    whose places are replaced by expert 0): every listed place is a pair of
+    its own.  Expert 2 here has 14 pairs, more than the 8 columns of one
+    MMA, so the kernel cuts its pairs into two slots."""
+    cfg = small_cfg("duplicate_ids", T=3, H=256, E=8, k=6, I=128, has_shared=True, G=32)
+    layer = synth.make_layer(cfg)
+    ids = np.array([[2, 2, 2, 5, 2, 2], [2, 0, 2, 2, 7, 2], [2, 2, 1, 2, 2, 2]], np.int32)
+    w = np.random.RandomState(5).uniform(0.05, 0.3, ids.shape).astype(np.float32)
+    ref = oracle.layer_forward(layer, override_ids=ids, override_w=w)
+    got = run_decode(layer, dev, override_ids=ids, override_w=w)
+    assert np.array_equal(got["topk_ids"], ids)
+    check_close(got["y"], ref["y"], cfg.name)
+    # the kernel chain takes the same routing
+    chain = run_layer(layer, dev, override_ids=ids, override_w=w)
+    check_close(chain["y"], ref["y"], cfg.name + " (chain)")
+
+
 @pytest.mark.parametrize("ctas", [1, 5])
 def test_decode_independent_of_grid(dev, ctas, monkeypatch):
     from quantized_moe_expert_warp_b200.host import upload_layer
@@ -138,7 +156,7 @@ def test_decode_repeated_calls_and_abort_flag(dev):
     b = run_decode(layer, dev, packed=packed, ws=ws)["y_bf16"]
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     words = ws[:256].view(torch.int32)
-    assert int(words[16].item()) == 0          # barrier count back at zero
+    assert int(words[16].item()) == 0          # barrier word back at zero (its top bit flips twice a call)
     words[18] = 1                              # abort flag, as a timed-out launch leaves it
     x = torch.zeros((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
     y = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
