@@ -338,11 +338,15 @@ int moe_layer_forward_chunked(const moe_layer_t *L, const uint16_t *x, int T, ui
  * them); at such sizes the separate kernels of moe_layer_forward cost more
  * in launches and pipeline fill than in memory traffic.
  *
- * Results: routing as in moe_route (on this kernel's fp32 logits), expert
- * FFNs with the exact dequantised weights in fp32 on CUDA cores, no
- * intermediate rounded to bf16 before y.  Within the layer tolerance of
- * the oracle, but not bitwise equal to moe_layer_forward.  Independent of
- * the number of CTAs (work is split by output rows only).
+ * Results: routing as in moe_route (on this kernel's fp32 logits); expert
+ * FFNs on warp-level tensor-core MMAs with fp32 accumulation, the codes
+ * entering exactly and each 32-weight chunk's scale applied to the fp32
+ * result, so the weights take their exact dequantised values; h rounded to
+ * bf16 once, as in moe_layer_forward.  Within the layer tolerance of the
+ * oracle, but not bitwise equal to moe_layer_forward (other summation
+ * order).  Independent of the number of CTAs (work is split by output rows
+ * and columns with fixed K slices).  A token may list an expert more than
+ * once (given ids): every place is a pair of its own.
  *
  * ws: moe_layer_decode_workspace_size(cfg, T) bytes (0 = shape or T not
  * admitted: T > 8, or x or the expert intermediates do not fit in shared
@@ -367,8 +371,8 @@ int moe_layer_decode(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *y
  * kernel recorded; *detail (optional) = where it was recorded.
  *
  * The status block (the first 256 bytes of those workspaces), as int32
- * words: [0] status, [1] detail, [16..18] the decode kernel's grid barrier
- * (count, generation, abort flag), [20] the wait budget in microseconds of
+ * words: [0] status, [1] detail, [16] and [18] the decode kernel's grid
+ * barrier (arrival word, abort flag), [20] the wait budget in microseconds of
  * every bounded device wait of the kernels reading this workspace (0: 2 s;
  * a wait that runs out records MOE_ERR_TIMEOUT and its kernel returns with
  * its TMEM freed and its copies landed), [21] a test knob: c > 0 makes

@@ -214,8 +214,9 @@ LayerWs layer_layout(const moe_config_t *c, int T, uint8_t *base)
 }
 
 // Workspace of the fused decode kernel: the 256-byte status block (status
-// word, detail, and at byte 64 the grid barrier's count, generation and
-// abort flag), then logits, gate logits, routing and the fp32 expert outputs.
+// word, detail, and at byte 64 the grid barrier's arrival word, an unused
+// word and the abort flag), then logits, gate logits, routing and the bf16
+// gate/up outputs h.
 struct DecodeWs {
     int *status;
     unsigned *bar;

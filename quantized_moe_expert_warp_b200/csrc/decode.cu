@@ -9,15 +9,16 @@
 //   A  router: logits[t, e] = x[t] . Wr[e] (+ bias), gate[t] = x[t] . g;
 //      one warp per router row (fp32 FMAs), rows spread over the CTAs
 //   B  every CTA routes all T tokens itself (top-k as in route.cu) and
-//      groups the (token, expert) pairs by expert
-//   C  gate/up + SwiGLU: a unit is (expert, 16 features), i.e. a 16-row tile
+//      groups the (token, expert) pairs by expert, in slots of at most 8
+//      pairs (the columns of one MMA)
+//   C  gate/up + SwiGLU: a unit is (slot, 16 features), i.e. a 16-row tile
 //      of Wg and the matching tile of Wu; the 16 warps split K = H, each
-//      runs warp-level m16n8k16 tensor-core MMAs against the expert's tokens
+//      runs warp-level m16n8k16 tensor-core MMAs against the slot's tokens
 //      (up to 8 columns), and the warps' sums are added in a fixed order:
 //          h[p, i] = bf16( silu(x[t] . Wg_e[i]) * (x[t] . Wu_e[i]) )
 //   D  down and combine: a unit is 16 output columns (a 16-row tile of Wd)
-//      of every chosen expert, one warp per expert, MMAs against the
-//      expert's h rows; the combine of those columns happens in the CTA:
+//      of every slot, one warp per slot, MMAs against the slot's h rows;
+//      the combine of those columns happens in the CTA:
 //          y[t, c] = bf16( sum_j w[t,j] (h[p(t,j)] . Wd_e[c])
 //                          + sigmoid(gate[t]) (h[shared t] . Wd_s[c]) )
 //
@@ -32,9 +33,10 @@
 // so the weights enter at their exact dequantised values; x is bf16 (exact)
 // and h is rounded to bf16 once, as on the prefill path.
 //
-// Each phase runs its code a few times per launch at most, so instruction
-// fetch is a large share of its time: loops over tokens, chunks and items
-// stay rolled, and the kernel is instantiated per weight format.
+// The chunks of one staged item are unrolled so that their MMA chains
+// overlap; loops over tokens, items and units stay rolled, which keeps the
+// code that runs once per launch small, and the kernel is instantiated per
+// weight format.
 //
 // Work is split by output rows and columns with fixed K slices, and every
 // sum runs in a fixed order, so the result does not depend on the number of
@@ -347,7 +349,6 @@ DecodeSmem decode_smem_layout(int T, int k, int H, int I, int has_shared, int wf
             redc = sizeof(float) * kWarps * kN;
         const size_t outd = up16(sizeof(float) * (size_t)np * kRedLd);
         s.big = take(xbytes + nred * redc > hbytes + outd ? xbytes + nred * redc : hbytes + outd);
-        s.sums = 0;   // placed inside big by the kernel
         s.red = s.big + (int)xbytes;
         s.nred = nred;
         s.ntok = ntok;

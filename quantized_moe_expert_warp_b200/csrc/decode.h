@@ -29,12 +29,12 @@ struct DecodeArgs {
     uint16_t *h;                // [NP, I] gate/up outputs (bf16), NP = T k (+ T)
     uint16_t *y;                // [T, H] bf16
     int *status;                // [code, detail]
-    unsigned *bar;              // [count, generation, abort] of the grid barrier
+    unsigned *bar;              // [arrival word, unused, abort flag] of the grid barrier
 };
 
 // Byte offsets of the decode kernel's dynamic shared memory.
 struct DecodeSmem {
-    int big, sums, red, ored, cbuf, ids, w, pidx, pair_tok, pair_w, slot_e, slot_base, slot_cnt, tcount, dexp, dbase,
+    int big, red, ored, cbuf, ids, w, pidx, pair_tok, pair_w, slot_e, slot_base, slot_cnt, tcount, dexp, dbase,
         bitmap, wprefix, flag;
     int nred;     // gate/up partials buffers (1 or 2)
     int ntok;     // pairs (MMA columns) a slot holds at most: min(8, T k)
