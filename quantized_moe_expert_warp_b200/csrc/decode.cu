@@ -184,6 +184,17 @@ __device__ __forceinline__ void staged_coeffs(const uint8_t *mrow, int kpos, flo
     }
 }
 
+// 32-weight chunks that share one scale entry, capped at 4 (the chunks one
+// warp takes together): G / 32 for the int4 formats, 1 for Q4K (its
+// sub-block scales change every 32 weights).
+template <int WFMT>
+__device__ __forceinline__ int chunks_per_group(int G)
+{
+    if (WFMT == MOE_WFMT_Q4K)
+        return 1;
+    return G >= 128 ? 4 : G >= 64 ? 2 : 1;
+}
+
 // Top-k of one token by one warp (lane l holds logits l, l + 32, ...):
 // ties to the lower id, weights softmax over the kept k (renorm) or over
 // all E.  Lane j < k returns the j-th id and weight; a position left
@@ -386,7 +397,7 @@ DecodeSmem decode_smem_layout(int T, int k, int H, int I, int has_shared, int wf
 namespace {
 
 // Gate/up staging of one unit pass for this warp, with 16-byte cp.async:
-// chunks j = j0 + warp + 16 n (n < 4) of the 16 gate and 16 up rows of the
+// chunks j = j0 + 4 warp + n (n < 4) of the 16 gate and 16 up rows of the
 // unit, as codes [n][matrix][row][16 bytes] (2 KB), then the rows' scale
 // entries of each (n, matrix) [n][matrix][row][entry].  gsh: log2 of the
 // positions along K that share one entry.
@@ -405,7 +416,7 @@ __device__ __forceinline__ void gu_stage(const DecodeArgs &A, int e, int f0, int
         const int idx = lane + 32 * q;   // 8 MB pieces of 16 bytes
         if (idx < 8 * MB) {
             const int nm = idx / MB, pi = idx % MB, n = nm >> 1, m = nm & 1;
-            const int j = j0 + warp + kWarps * n;
+            const int j = j0 + 4 * warp + n;
             if (j < nchH) {
                 const uint8_t *src = mb + ((size_t)(m * ngroups + ((j * 32) >> gsh)) * kTileRows + r0) * MB + 16 * pi;
                 cp_async_16(dst + kCodeBuf + idx * 16, src, 16);
@@ -417,7 +428,7 @@ __device__ __forceinline__ void gu_stage(const DecodeArgs &A, int e, int f0, int
     for (int q = 0; q < 4; ++q) {
         const int idx = lane + 32 * q;    // 128 pieces of 16 bytes
         const int n = idx >> 5, m = (idx >> 4) & 1, row = idx & 15;
-        const int j = j0 + warp + kWarps * n;
+        const int j = j0 + 4 * warp + n;
         if (j < nchH) {
             const uint8_t *src = base + (size_t)(j >> 1) * code_block_bytes(2) +
                                  ((size_t)(m * 2 + (j & 1)) * kTileRows + r0 + row) * kChunkBytes;
@@ -746,6 +757,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
     // ------------------------------------------------ C: gate/up + SwiGLU (tensor cores)
     {
         const int gsh = WFMT == MOE_WFMT_Q4K ? 8 : gshift;
+        const int cpg = chunks_per_group<WFMT>(A.G);
         const int per_slot = I / kFeat;
         const int U = Nd * per_slot;
         const int npass = (nchH + 4 * kWarps - 1) / (4 * kWarps);
@@ -784,36 +796,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
             cp_async_wait_upto(NS - 1);   // item it's copies have landed
             __syncwarp();
             const uint8_t *buf = mybuf + (it % NS) * kIB;
-            // the 4 chunks are independent MMA chains: unrolled so that they
-            // overlap; a chunk past the end reads a valid one and is not added
+            // the warp's 4 consecutive chunks (all past the end or none: H is
+            // a multiple of 128); the MMAs of one scale group accumulate in
+            // dd and the group's scale and offset are applied once
+            const int j0 = pass * 4 * kWarps + 4 * warp;
+            if (j0 < nchH) {
+                float dd[2][4] = {};
+                float sA = 0.f, sB = 0.f;
 #pragma unroll
-            for (int n = 0; n < 4; ++n) {
-                const int jr = pass * 4 * kWarps + warp + kWarps * n;
-                const bool valid = jr < nchH;
-                const int j = valid ? jr : nchH - 1;
-                float cs[2][2][2];   // [matrix][row lo/hi][a, b]
+                for (int n = 0; n < 4; ++n) {
+                    const int j = j0 + n;
+                    sA += tA >= 0 ? xsum[tA * nchH + j] : 0.f;
+                    sB += tB >= 0 ? xsum[tB * nchH + j] : 0.f;
+                    const uint16_t *brow = xb + (size_t)trow * XS + j * 32;
 #pragma unroll
-                for (int m = 0; m < 2; ++m) {
-                    const uint8_t *mrow = buf + kCodeBuf + ((n * 2 + m) * 16 + gid) * kMB;
-                    staged_coeffs<WFMT>(mrow, j * 32, cs[m][0][0], cs[m][0][1]);
-                    staged_coeffs<WFMT>(mrow + 8 * kMB, j * 32, cs[m][1][0], cs[m][1][1]);
-                }
-                const float sA = tA >= 0 ? xsum[tA * nchH + j] : 0.f;
-                const float sB = tB >= 0 ? xsum[tB * nchH + j] : 0.f;
-                const uint16_t *brow = xb + (size_t)trow * XS + j * 32;
+                    for (int m = 0; m < 2; ++m) {
+                        const uint4 lo = *(const uint4 *)(buf + ((n * 2 + m) * 16 + gid) * 16);
+                        const uint4 hi = *(const uint4 *)(buf + ((n * 2 + m) * 16 + gid + 8) * 16);
+                        chunk_mma(dd[m], lo, hi, brow, tid4);
+                    }
+                    if (((n + 1) & (cpg - 1)) == 0) {   // the last chunk of a scale group
+                        // rows gid (v = 0, 1) and gid + 8 (v = 2, 3); tokens 2 tid4 + (v & 1)
 #pragma unroll
-                for (int m = 0; m < 2; ++m) {
-                    const uint4 lo = *(const uint4 *)(buf + ((n * 2 + m) * 16 + gid) * 16);
-                    const uint4 hi = *(const uint4 *)(buf + ((n * 2 + m) * 16 + gid + 8) * 16);
-                    float dd[4] = {0.f, 0.f, 0.f, 0.f};
-                    chunk_mma(dd, lo, hi, brow, tid4);
-                    // rows gid (v = 0, 1) and gid + 8 (v = 2, 3); tokens 2 tid4 + (v & 1)
+                        for (int m = 0; m < 2; ++m) {
+                            const uint8_t *mrow = buf + kCodeBuf + ((n * 2 + m) * 16 + gid) * kMB;
+                            float alo, blo, ahi, bhi;
+                            staged_coeffs<WFMT>(mrow, j * 32, alo, blo);
+                            staged_coeffs<WFMT>(mrow + 8 * kMB, j * 32, ahi, bhi);
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        const float sx = (v & 1) ? sB : sA;
-                        const float a = cs[m][v >> 1][0], b = cs[m][v >> 1][1];
-                        const float nv = fmaf(a, fmaf(-kOff, sx, dd[v]), fmaf(b, sx, acc[m][v]));
-                        acc[m][v] = valid ? nv : acc[m][v];
+                            for (int v = 0; v < 4; ++v) {
+                                const float sx = (v & 1) ? sB : sA;
+                                const float a = (v >> 1) ? ahi : alo, b = (v >> 1) ? bhi : blo;
+                                acc[m][v] = fmaf(a, fmaf(-kOff, sx, dd[m][v]), fmaf(b, sx, acc[m][v]));
+                                dd[m][v] = 0.f;
+                            }
+                        }
+                        sA = 0.f;
+                        sB = 0.f;
                     }
                 }
             }
@@ -866,6 +885,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
         float *hsum = (float *)(hb + (size_t)(NP + 1) * HS);
         issue_rows(A.h, I, NP, NP, smem_u32(hb), HS, tid);
         const int gsh = WFMT == MOE_WFMT_Q4K ? 8 : gshift;
+        const int cpg = chunks_per_group<WFMT>(A.G);
         const int nparts = (nchI + 7) / 8;
         float *o_s = (float *)(smem + L.ored);   // [pair][column]
         // this warp's slots: d = warp + kWarps i; items (slot, part)
@@ -910,28 +930,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
                 __syncwarp();
                 DEC_ACC(tdw, c0);
                 const uint8_t *buf = mybuf + (it % NS) * kIB;
-                // independent chunks, partly unrolled as in the gate/up loop
+                // the item's chunks (past the end in whole groups of 4: I is a
+                // multiple of 128); the MMAs of one scale group accumulate in
+                // dd and the group's scale and offset are applied once
+                float dd[4] = {0.f, 0.f, 0.f, 0.f};
+                float sA = 0.f, sB = 0.f;
 #pragma unroll 4
                 for (int n = 0; n < 8; ++n) {
-                    const int jr = 8 * q + n;
-                    const bool valid = jr < nchI;
-                    const int j = valid ? jr : nchI - 1;
-                    float clo_a, clo_b, chi_a, chi_b;
-                    const uint8_t *mrow = buf + kCodeBuf + (n * 16 + gid) * kMB;
-                    staged_coeffs<WFMT>(mrow, j * 32, clo_a, clo_b);
-                    staged_coeffs<WFMT>(mrow + 8 * kMB, j * 32, chi_a, chi_b);
-                    const float sA = pA >= 0 ? hsum[pA * nchI + j] : 0.f;
-                    const float sB = pB >= 0 ? hsum[pB * nchI + j] : 0.f;
-                    const uint4 lo = *(const uint4 *)(buf + (n * 16 + gid) * 16);
-                    const uint4 hi = *(const uint4 *)(buf + (n * 16 + gid + 8) * 16);
-                    float dd[4] = {0.f, 0.f, 0.f, 0.f};
-                    chunk_mma(dd, lo, hi, hb + (size_t)prow * HS + j * 32, tid4);
+                    const int j = 8 * q + n;
+                    if (j < nchI) {
+                        sA += pA >= 0 ? hsum[pA * nchI + j] : 0.f;
+                        sB += pB >= 0 ? hsum[pB * nchI + j] : 0.f;
+                        const uint4 lo = *(const uint4 *)(buf + (n * 16 + gid) * 16);
+                        const uint4 hi = *(const uint4 *)(buf + (n * 16 + gid + 8) * 16);
+                        chunk_mma(dd, lo, hi, hb + (size_t)prow * HS + j * 32, tid4);
+                        if (((n + 1) & (cpg - 1)) == 0) {   // the last chunk of a scale group
+                            float clo_a, clo_b, chi_a, chi_b;
+                            const uint8_t *mrow = buf + kCodeBuf + (n * 16 + gid) * kMB;
+                            staged_coeffs<WFMT>(mrow, j * 32, clo_a, clo_b);
+                            staged_coeffs<WFMT>(mrow + 8 * kMB, j * 32, chi_a, chi_b);
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        const float sx = (v & 1) ? sB : sA;
-                        const float a = (v >> 1) ? chi_a : clo_a, b = (v >> 1) ? chi_b : clo_b;
-                        const float nv = fmaf(a, fmaf(-kOff, sx, dd[v]), fmaf(b, sx, acc[v]));
-                        acc[v] = valid ? nv : acc[v];
+                            for (int v = 0; v < 4; ++v) {
+                                const float sx = (v & 1) ? sB : sA;
+                                const float a = (v >> 1) ? chi_a : clo_a, b = (v >> 1) ? chi_b : clo_b;
+                                acc[v] = fmaf(a, fmaf(-kOff, sx, dd[v]), fmaf(b, sx, acc[v]));
+                                dd[v] = 0.f;
+                            }
+                            sA = 0.f;
+                            sB = 0.f;
+                        }
                     }
                 }
                 __syncwarp();
