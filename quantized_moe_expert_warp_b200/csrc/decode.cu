@@ -54,14 +54,16 @@
 
 #ifdef MOEQ4_TRACE
 // phase timestamps (%globaltimer) of the first four CTAs, thread 0
-__device__ unsigned long long g_dec_trace[4][16];
+__device__ unsigned long long g_dec_trace[4][24];
 #define DEC_MARK(i)                                                   \
     do {                                                              \
         if (blockIdx.x < 4 && threadIdx.x == 0)                       \
             g_dec_trace[blockIdx.x][(i)] = moeq4::globaltimer_ns();    \
     } while (0)
-// entries 7 .. 10: steps inside the routing phase; 15: warp 0's cycles
-// waiting for its staged down items
+// entries 7 .. 10: steps inside the routing phase; 11 .. 14: warp 0's
+// cycles in the gate/up phase issuing copies, waiting for them, in the MMA
+// loop and in the hand-off; 15: warp 0's cycles waiting for its staged down
+// items; 16, 17: clock64 at the start and the end of the gate/up phase
 #define DEC_CLK(v) const long long v = clock64()
 #define DEC_ACC(a, since) (a) += clock64() - (since)
 #define DEC_DECL(a) long long a = 0
@@ -777,11 +779,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
             stage(it2);
         float acc[2][4];
         int ru = 0;   // units reduced so far: picks the partials buffer
+        DEC_DECL(ts);
+        DEC_DECL(tw);
+        DEC_DECL(tc);
+        DEC_DECL(tr);
+#ifdef MOEQ4_TRACE
+        if (blockIdx.x < 4 && threadIdx.x == 0)
+            g_dec_trace[blockIdx.x][16] = (unsigned long long)clock64();
+#endif
         for (int it = 0; it < nitems; ++it) {
             const int u = unit_of(it), pass = it % npass;
             const int d = u / per_slot, f0 = (u % per_slot) * kFeat;
             const int base = slot_base[d], cnt = slot_cnt[d];
+            DEC_CLK(c_s);
             stage(it + NS - 1);
+            DEC_ACC(ts, c_s);
             if (pass == 0) {
 #pragma unroll
                 for (int m = 0; m < 2; ++m)
@@ -793,8 +805,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
             const int trow = gid < cnt ? pair_tok[base + gid] : kN;
             const int tA = 2 * tid4 < cnt ? pair_tok[base + 2 * tid4] : -1;
             const int tB = 2 * tid4 + 1 < cnt ? pair_tok[base + 2 * tid4 + 1] : -1;
+            DEC_CLK(c_w);
             cp_async_wait_upto(NS - 1);   // item it's copies have landed
             __syncwarp();
+            DEC_ACC(tw, c_w);
+            DEC_CLK(c_c);
             const uint8_t *buf = mybuf + (it % NS) * kIB;
             // the warp's 4 consecutive chunks (all past the end or none: H is
             // a multiple of 128); the MMAs of one scale group accumulate in
@@ -837,6 +852,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
                 }
             }
             __syncwarp();
+            DEC_ACC(tc, c_c);
+            DEC_CLK(c_r);
             if (pass == npass - 1) {
                 // the unit is complete in every warp: gate and up summed over
                 // the warps, in order.  The partials alternate between two
@@ -868,9 +885,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const DecodeA
                     A.h[(size_t)(base + nn) * I + f0 + f] = (uint16_t)(pack_bf16x2(hv, 0.f) & 0xFFFFu);
                 }
             }
+            DEC_ACC(tr, c_r);
         }
         cp_async_wait_group<0>();
         __syncwarp();
+#ifdef MOEQ4_TRACE
+        if (blockIdx.x < 4 && threadIdx.x == 0) {
+            g_dec_trace[blockIdx.x][11] = (unsigned long long)ts;
+            g_dec_trace[blockIdx.x][12] = (unsigned long long)tw;
+            g_dec_trace[blockIdx.x][13] = (unsigned long long)tc;
+            g_dec_trace[blockIdx.x][14] = (unsigned long long)tr;
+            g_dec_trace[blockIdx.x][17] = (unsigned long long)clock64();
+        }
+#endif
     }
     DEC_MARK(4);
     if (!grid_sync(A.bar, A.status, 92, flag, false, wait_ns))
