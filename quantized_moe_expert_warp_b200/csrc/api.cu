@@ -650,7 +650,8 @@ int moe_combine(const uint16_t *y_perm, const int32_t *dest_pos, const float *to
         REQUIRE_PTR(shared_out);
     if (shared_gate_logit)
         REQUIRE_PTR(shared_gate_logit);
-    CUDA_TRY(launch_combine(y_perm, dest_pos, topk_w, shared_out, shared_gate_logit, T, H, k, y, (cudaStream_t)stream),
+    CUDA_TRY(launch_combine(y_perm, dest_pos, topk_w, shared_out, shared_gate_logit, T, H, k, y, num_sms(),
+                            (cudaStream_t)stream),
              "combine");
     g_launches += 1;
     return ok();
@@ -734,7 +735,7 @@ int moe_layer_forward(const moe_layer_t *L, const uint16_t *x, int T, uint16_t *
     if (rc)
         return rc;
     CUDA_TRY(launch_combine(w.y_perm, w.dest_pos, tw, c.has_shared ? w.shared_out : nullptr,
-                            c.has_shared ? w.gate_logit : nullptr, T, c.H, c.k, y, st),
+                            c.has_shared ? w.gate_logit : nullptr, T, c.H, c.k, y, num_sms(), st),
              "combine");
     g_launches += 1;
     if (dbg) {

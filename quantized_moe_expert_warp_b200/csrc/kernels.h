@@ -129,7 +129,7 @@ cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *sorted_slot, in
                                int *status = nullptr);
 
 cudaError_t launch_combine(const uint16_t *y_perm, const int32_t *dest_pos, const float *w, const uint16_t *shared_out,
-                           const float *gate_logit, int T, int H, int k, uint16_t *y, cudaStream_t st);
+                           const float *gate_logit, int T, int H, int k, uint16_t *y, int num_sms, cudaStream_t st);
 
 cudaError_t launch_pack_codes(const moe_config_t &cfg, int which, const uint8_t *canon, uint8_t *out,
                               cudaStream_t st);
